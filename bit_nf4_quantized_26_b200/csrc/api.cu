@@ -1,0 +1,564 @@
+// api.cu — the C ABI declared in include/qlora_nf4.h: argument checks,
+// workspace planning, TMA descriptor creation and kernel launches.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "kernels.h"
+
+using namespace qnf4;
+
+namespace {
+
+// ------------------------------------------------------------ NF4 constants
+//
+// "QLoRA" encyclopedia entry (tonho.wtf), section "como funciona": a 4-bit
+// type from standard-normal quantiles, normalised to [-1, 1] by the absolute
+// maximum, asymmetric so that zero is exact.  Positive levels are the N(0,1)
+// quantiles at 8 probabilities evenly spaced from DELTA towards 1/2, negative
+// levels minus the quantiles at 7 such probabilities, plus 0; all divided by
+// the largest magnitude.  DELTA is the mean of 1-1/30 and 1-1/32.  The
+// quantile is found by bisection on Phi(x) = erfc(-x/sqrt 2)/2 in double
+// precision, then rounded once to fp32.
+
+double normal_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double normal_quantile(double p) {
+  double lo = -12.0, hi = 12.0;
+  for (int i = 0; i < 200; ++i) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (normal_cdf(mid) < p) lo = mid;
+    else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+Nf4Tables build_tables() {
+  const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+  std::vector<double> lv;
+  const double step_pos = (0.5 - delta) / 8.0, step_neg = (0.5 - delta) / 7.0;
+  for (int i = 0; i < 8; ++i) lv.push_back(normal_quantile(i * step_pos + delta));
+  for (int i = 0; i < 7; ++i) lv.push_back(-normal_quantile(i * step_neg + delta));
+  lv.push_back(0.0);
+  std::sort(lv.begin(), lv.end());
+  double amax = 0.0;
+  for (double v : lv) amax = std::max(amax, std::fabs(v));
+  Nf4Tables t{};
+  for (int i = 0; i < 16; ++i) t.q[i] = static_cast<float>(lv[i] / amax);
+  float mid[15];
+  for (int i = 0; i < 15; ++i)
+    mid[i] = static_cast<float>((static_cast<double>(t.q[i]) + static_cast<double>(t.q[i + 1])) / 2.0);
+  for (int b = 0; b < 64; ++b) {
+    t.thr[b] = INFINITY;
+    t.base[b] = 0;
+  }
+  for (int b = 0; b <= 32; ++b) {
+    const double lo = -1.0 + (b - 0.5) / 16.0, hi = -1.0 + (b + 0.5) / 16.0;
+    int below = 0, inside = 0;
+    float thr = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      const double m = mid[i];
+      if (m < lo) ++below;
+      else if (m <= hi) { ++inside; thr = mid[i]; }
+      // A midpoint on (or next to) a bucket edge would make the bucket
+      // choice matter; the NF4 midpoints sit at least 4e-3 from every edge.
+      if (std::fabs(m - lo) < 1e-6 || std::fabs(m - hi) < 1e-6) std::abort();
+    }
+    if (inside > 1) std::abort();
+    t.base[b] = below;
+    t.thr[b] = thr;
+  }
+  return t;
+}
+
+const Nf4Tables& tables() {
+  static const Nf4Tables t = build_tables();
+  return t;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] of elements of `esize` bytes, row
+// stride `row_bytes`, copied in boxes of [box_outer, box_inner].
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows, true);
+}
+
+bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, false);
+}
+
+// ------------------------------------------------------------ checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qlora_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  static int arch_ok[64] = {0};  // 0 unknown, 1 ok, 2 not sm_100
+  if (dev < 0 || dev >= 64) return QLORA_ERR_ARCH;
+  if (arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return arch_ok[dev] == 1 ? QLORA_OK : QLORA_ERR_ARCH;
+}
+
+qlora_status check_linear_shape(int64_t M, const nf4_weight& W, int32_t r) {
+  const int64_t N = W.n_out, K = W.k_in;
+  if (M < 0 || M >= (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
+  if (N < 64 || K < 64 || N % 64 != 0 || K % 64 != 0) return QLORA_ERR_SHAPE;
+  if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N * K >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  if (r < 16 || r > 64 || r % 16 != 0) return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+qlora_status check_weight_ptrs(const nf4_weight& W) {
+  if (!W.codes || !W.c8 || !W.s2) return QLORA_ERR_NULL;
+  if (!aligned16(W.codes) || !aligned16(W.c8) || !aligned16(W.s2)) return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+// ------------------------------------------------------------ kernel timing
+
+enum KernelId {
+  kKQuantize = 0, kKDequantize, kKDown, kKFinishDown, kKFusedFwd, kKFinishFwd, kKPrepSU, kKDU, kKFinishDU,
+  kKDB, kKFinishDB, kKFusedDX, kKDA, kKFinishDA, kKCount
+};
+const char* const kKernelNames[kKCount] = {
+    "nf4_quantize", "nf4_dequantize", "lora_down", "finish_down", "fused_fwd", "finish_fwd", "prep_su",
+    "lora_du", "finish_du", "lora_db", "finish_db", "fused_dx", "lora_da", "finish_da"};
+
+struct ProfRecord {
+  int id;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one kernel launch with events on its stream while profiling is on.
+class ProfScope {
+ public:
+  ProfScope(int id, cudaStream_t s) : s_(s) {
+    if (!g_prof_on) return;
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    rec_.id = id;
+    rec_.start = prof_event();
+    rec_.stop = prof_event();
+    if (rec_.start && rec_.stop) {
+      cudaEventRecord(rec_.start, s_);
+      active_ = true;
+    }
+  }
+  ~ProfScope() {
+    if (!active_) return;
+    cudaEventRecord(rec_.stop, s_);
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    g_prof_records.push_back(rec_);
+  }
+
+ private:
+  cudaStream_t s_;
+  ProfRecord rec_{};
+  bool active_ = false;
+};
+
+// ------------------------------------------------------------ planning
+//
+// Split counts depend only on the shape (aim: about two CTAs per SM of a
+// 148-SM B200), so the workspace query is a pure host function.
+
+constexpr int kTargetCtas = 296;
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Number of slices for `stages` contraction steps over `tiles` output tiles,
+// with at least `min_per` steps per slice; every slice is non-empty.
+void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int& splits, int& per) {
+  int64_t s = std::max<int64_t>(1, cdiv(kTargetCtas, std::max<int64_t>(tiles, 1)));
+  s = std::min<int64_t>(s, std::max<int64_t>(1, stages / std::max<int64_t>(min_per, 1)));
+  const int64_t p = cdiv(stages, s);
+  per = static_cast<int>(p);
+  splits = static_cast<int>(cdiv(stages, p));
+}
+
+struct FwdPlan {
+  int s_down, per_down;
+  int bn, s_fwd, per_fwd;
+  size_t off_ucat, off_pfwd, total;
+};
+
+FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
+  FwdPlan p{};
+  const int64_t kst = K / 64;
+  split_plan(cdiv(M, 128), kst, 4, p.s_down, p.per_down);
+  p.bn = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
+  const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
+  if (M <= 256) split_plan(tiles, kst, 8, p.s_fwd, p.per_fwd);
+  else { p.s_fwd = 1; p.per_fwd = static_cast<int>(kst); }
+  size_t off = align256(static_cast<size_t>(p.s_down) * M * r * 4);
+  p.off_ucat = off;
+  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  p.off_pfwd = off;
+  if (p.s_fwd > 1) off += align256(static_cast<size_t>(p.s_fwd) * M * N * 4);
+  p.total = off;
+  return p;
+}
+
+struct BwdPlan {
+  int s_du, per_du, s_db, per_db, s_da, per_da, bn;
+  size_t off_sucat, off_pdu, off_ducat, off_pdb, off_pda, total;
+};
+
+BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
+  BwdPlan p{};
+  split_plan(cdiv(M, 128), N / 64, 4, p.s_du, p.per_du);
+  split_plan(cdiv(N, 128), cdiv(M, 64), 4, p.s_db, p.per_db);
+  split_plan(cdiv(K, 256), cdiv(M, 64), 4, p.s_da, p.per_da);
+  p.bn = M > 128 ? 256 : 128;
+  size_t off = 0;
+  p.off_sucat = off;
+  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  p.off_pdu = off;
+  off += align256(static_cast<size_t>(p.s_du) * M * r * 4);
+  p.off_ducat = off;
+  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  p.off_pdb = off;
+  off += align256(static_cast<size_t>(p.s_db) * N * r * 4);
+  p.off_pda = off;
+  off += align256(static_cast<size_t>(p.s_da) * r * K * 4);
+  p.total = off;
+  return p;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+void qlora_profile_enable(int32_t enable) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = enable != 0;
+}
+
+int32_t qlora_profile_collect(int32_t* kernel_ids, float* ms, int32_t capacity) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  int32_t n = 0;
+  bool ok = true;
+  for (const ProfRecord& r : g_prof_records) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+      ok = false;
+    if (n < capacity) {
+      if (kernel_ids) kernel_ids[n] = r.id;
+      if (ms) ms[n] = t;
+    }
+    ++n;
+    g_prof_pool.push_back(r.start);
+    g_prof_pool.push_back(r.stop);
+  }
+  g_prof_records.clear();
+  return ok ? n : -1;
+}
+
+const char* qlora_kernel_name(int32_t id) {
+  return (id >= 0 && id < kKCount) ? kKernelNames[id] : "unknown";
+}
+
+const char* qlora_strerror(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_NULL: return "a required pointer is NULL";
+    case QLORA_ERR_SHAPE: return "a size violates the documented constraints";
+    case QLORA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_NONFINITE: return "non-finite input";
+    case QLORA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case QLORA_ERR_CUDA: return "a CUDA call failed";
+    case QLORA_ERR_ARCH: return "the current device is not sm_100";
+    case QLORA_ERR_DTYPE: return "unknown output dtype";
+  }
+  return "unknown status";
+}
+
+void nf4_levels(float out[16]) {
+  if (out) std::memcpy(out, tables().q, sizeof(float) * 16);
+}
+
+size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+  return plan_fwd(M, N, K, r).total;
+}
+
+size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+  return plan_bwd(M, N, K, r).total;
+}
+
+qlora_status nf4_quantize(const uint16_t* w_bf16, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                          int32_t* d_status, void* stream) {
+  if (numel < 0 || numel >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  if (numel == 0) return QLORA_OK;
+  if (!w_bf16 || !codes || !c8 || !s2) return QLORA_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(c8) || !aligned16(s2) ||
+      (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  ProfScope ps(kKQuantize, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_nf4_quantize(w_bf16, numel, codes, c8, s2, d_status, tables(),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
+                            uint16_t* w_bf16, void* stream) {
+  if (numel < 0 || numel >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  if (numel == 0) return QLORA_OK;
+  if (!w_bf16 || !codes || !c8 || !s2) return QLORA_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(c8) || !aligned16(s2)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  ProfScope ps(kKDequantize, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_nf4_dequantize(codes, c8, s2, numel, w_bf16, tables(), static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
+                              int32_t r, float s, void* Y, int32_t y_dtype, float* U_out, void* ws,
+                              size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
+  if (M == 0) return QLORA_OK;
+  if (!X || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;
+  if (qlora_status st = check_weight_ptrs(W)) return st;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(U_out) ||
+      (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  const int64_t N = W.n_out, K = W.k_in;
+  const FwdPlan p = plan_fwd(M, N, K, r);
+  if (!ws || ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* pdown = reinterpret_cast<float*>(wsb);
+  uint16_t* ucat = reinterpret_cast<uint16_t*>(wsb + p.off_ucat);
+  float* pfwd = reinterpret_cast<float*>(wsb + p.off_pfwd);
+
+  // U = X A^T  (split over K, fixed-order finish), then s*U as bf16 hi/lo.
+  CUtensorMap mx_down, ma_down;
+  if (!map_bf16(&mx_down, X, M, K, 64, 128) || !map_bf16(&ma_down, A, r, K, 64, 64)) return QLORA_ERR_CUDA;
+  SkinnyArgs sa{};
+  sa.partial = pdown;
+  sa.M = static_cast<int>(M);
+  sa.N = static_cast<int>(N);
+  sa.K = static_cast<int>(K);
+  sa.r = r;
+  sa.stages_total = static_cast<int>(K / 64);
+  sa.stages_per_split = p.per_down;
+  sa.status = d_status;
+  {
+    ProfScope ps(kKDown, cs);
+    if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa, static_cast<int>(cdiv(M, 128)),
+                                                  p.s_down, cs)))
+      return st;
+  }
+  {
+    ProfScope ps(kKFinishDown, cs);
+    if (qlora_status st = from_cuda(launch_finish_down(pdown, p.s_down, static_cast<int>(M), r, s, U_out, ucat, cs)))
+      return st;
+  }
+
+  // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
+  CUtensorMap mx, mc, mu, mb;
+  if (!map_bf16(&mx, X, M, K, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 32, 128) ||
+      !map_bf16(&mu, ucat, M, 2 * r, 64, p.bn) || !map_bf16(&mb, B, N, r, 64, 128))
+    return QLORA_ERR_CUDA;
+  FusedArgs fa{};
+  fa.c8 = W.c8;
+  fa.s2 = W.s2;
+  fa.out = p.s_fwd > 1 ? static_cast<void*>(pfwd) : Y;
+  fa.out_f32 = y_dtype == QLORA_DTYPE_F32;
+  fa.ld_out = N;
+  fa.split_stride = p.s_fwd > 1 ? M * N : 0;
+  fa.M = static_cast<int>(M);
+  fa.rows = static_cast<int>(N);
+  fa.n_out = static_cast<int>(N);
+  fa.k_in = static_cast<int>(K);
+  fa.r = r;
+  fa.kt_total = static_cast<int>(K / 64);
+  fa.kt_per_split = p.per_fwd;
+  fa.status = d_status;
+  fa.tab = tables();
+  {
+    ProfScope ps(kKFusedFwd, cs);
+    if (qlora_status st = from_cuda(launch_fused_fwd(p.bn, mx, mc, mu, mb, fa, p.s_fwd, cs))) return st;
+  }
+  if (p.s_fwd > 1) {
+    ProfScope ps(kKFinishFwd, cs);
+    return from_cuda(launch_finish_out(pfwd, p.s_fwd, M * N, Y, y_dtype == QLORA_DTYPE_F32, cs));
+  }
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
+                              const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX, int32_t dx_dtype,
+                              float* dA, float* dB, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
+  if (M == 0) return QLORA_OK;
+  if (!dY || !X || !U || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
+  if (qlora_status st = check_weight_ptrs(W)) return st;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(U) || !aligned16(A) || !aligned16(B) || !aligned16(dX) ||
+      !aligned16(dA) || !aligned16(dB) || (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  const int64_t N = W.n_out, K = W.k_in;
+  const BwdPlan p = plan_bwd(M, N, K, r);
+  if (!ws || ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* sucat = reinterpret_cast<uint16_t*>(wsb + p.off_sucat);
+  float* pdu = reinterpret_cast<float*>(wsb + p.off_pdu);
+  uint16_t* ducat = reinterpret_cast<uint16_t*>(wsb + p.off_ducat);
+  float* pdb = reinterpret_cast<float*>(wsb + p.off_pdb);
+  float* pda = reinterpret_cast<float*>(wsb + p.off_pda);
+  const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
+
+  SkinnyArgs sa{};
+  sa.M = Mi;
+  sa.N = Ni;
+  sa.K = Ki;
+  sa.r = r;
+  sa.status = d_status;
+
+  {
+    ProfScope ps(kKPrepSU, cs);
+    if (qlora_status st = from_cuda(launch_prep_su(U, Mi, r, s, sucat, cs))) return st;
+  }
+
+  // dU = s dY B  (split over N)
+  CUtensorMap mdy128, mbl;
+  if (!map_bf16(&mdy128, dY, M, N, 64, 128) || !map_bf16(&mbl, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
+  sa.partial = pdu;
+  sa.stages_total = static_cast<int>(N / 64);
+  sa.stages_per_split = p.per_du;
+  {
+    ProfScope ps(kKDU, cs);
+    if (qlora_status st = from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)), p.s_du, cs)))
+      return st;
+  }
+  {
+    ProfScope ps(kKFinishDU, cs);
+    if (qlora_status st = from_cuda(launch_finish_du(pdu, p.s_du, Mi, r, s, ducat, cs))) return st;
+  }
+
+  // dB = dY^T (sU)  (split over M)
+  CUtensorMap mdy64, msu;
+  if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * r, 64, 64)) return QLORA_ERR_CUDA;
+  sa.partial = pdb;
+  sa.stages_total = static_cast<int>(cdiv(M, 64));
+  sa.stages_per_split = p.per_db;
+  {
+    ProfScope ps(kKDB, cs);
+    if (qlora_status st = from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, cs)))
+      return st;
+  }
+  {
+    ProfScope ps(kKFinishDB, cs);
+    if (qlora_status st = from_cuda(launch_finish_sum(pdb, p.s_db, N * r, 1.0f, dB, cs))) return st;
+  }
+
+  // dX = dY W' + dU A, W' dequantised inside the GEMM.
+  CUtensorMap mdy, mc, mdu, mal;
+  if (!map_bf16(&mdy, dY, M, N, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 64, 64) ||
+      !map_bf16(&mdu, ducat, M, 2 * r, 64, p.bn) || !map_bf16(&mal, A, r, K, 64, 64))
+    return QLORA_ERR_CUDA;
+  FusedArgs fa{};
+  fa.c8 = W.c8;
+  fa.s2 = W.s2;
+  fa.out = dX;
+  fa.out_f32 = dx_dtype == QLORA_DTYPE_F32;
+  fa.ld_out = K;
+  fa.split_stride = 0;
+  fa.M = Mi;
+  fa.rows = Ki;
+  fa.n_out = Ni;
+  fa.k_in = Ki;
+  fa.r = r;
+  fa.kt_total = static_cast<int>(N / 64);
+  fa.kt_per_split = static_cast<int>(N / 64);
+  fa.status = d_status;
+  fa.tab = tables();
+  {
+    ProfScope ps(kKFusedDX, cs);
+    if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, cs))) return st;
+  }
+
+  // dA = dU^T X  (split over M)
+  CUtensorMap mduc, mx;
+  if (!map_bf16(&mduc, ducat, M, 2 * r, 64, 64) || !map_bf16(&mx, X, M, K, 64, 64)) return QLORA_ERR_CUDA;
+  sa.partial = pda;
+  sa.stages_total = static_cast<int>(cdiv(M, 64));
+  sa.stages_per_split = p.per_da;
+  {
+    ProfScope ps(kKDA, cs);
+    if (qlora_status st = from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 256)), p.s_da, cs)))
+      return st;
+  }
+  ProfScope ps(kKFinishDA, cs);
+  return from_cuda(launch_finish_sum(pda, p.s_da, static_cast<int64_t>(r) * K, 1.0f, dA, cs));
+}
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+// kernels.h — host-side launch functions of the CUDA kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "nf4_lut.cuh"
+
+namespace qnf4 {
+
+// Arguments shared by the fused dequantise-in-GEMM kernels.  The W side of the
+// product (dequantised NF4 rows: output features in the forward, input
+// features in dX) is the MMA's M dimension; tokens are its N dimension.
+struct FusedArgs {
+  const uint8_t* c8;   // FP8 block constants of W [n_out * k_in / 64]
+  const float* s2;     // group scales of W
+  void* out;           // out[m * ld_out + row]
+  int out_f32;         // 1: fp32 output, 0: bf16 output
+  int64_t ld_out;      // row stride of out (elements)
+  int64_t split_stride;// elements between split-K partial slices (0: no split)
+  int M;               // tokens
+  int rows;            // extent of the W-side index (N for fwd, K for dX)
+  int n_out, k_in;     // shape of W
+  int r;               // LoRA rank
+  int kt_total;        // main contraction stages (64 each)
+  int kt_per_split;    // stages per blockIdx.z slice
+  int32_t* status;
+  Nf4Tables tab;
+};
+
+enum SkinnyMode { kSkDown = 0, kSkDU = 1, kSkDB = 2, kSkDA = 3 };
+
+struct SkinnyArgs {
+  float* partial;      // [splits][rows][cols] fp32 partial sums
+  int M, N, K, r;
+  int stages_total;    // contraction stages (64 each)
+  int stages_per_split;
+  int32_t* status;
+};
+
+cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                                int32_t* status, const Nf4Tables& tab, cudaStream_t stream);
+cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
+                                  uint16_t* out, const Nf4Tables& tab, cudaStream_t stream);
+
+// Forward: Y[m, n] (+)= sum_k X[m,k] W'[n,k]  (+ LoRA extension in split 0).
+//   tm_x: X [M,K] box {64, BN} SW128; tm_codes: codes [N, K/2] box {32, 128};
+//   tm_uc: Ucat [M, 2r] box {64, BN} SW128; tm_bl: B [N, r] box {64, 128} SW128.
+cudaError_t launch_fused_fwd(int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_codes,
+                             const CUtensorMap& tm_uc, const CUtensorMap& tm_bl, const FusedArgs& a,
+                             int splits, cudaStream_t stream);
+
+// dX: dX[m, k] = sum_n dY[m,n] W'[n,k] + LoRA extension.
+//   tm_dy: dY [M,N] box {64, BN} SW128; tm_codes: codes [N, K/2] box {64, 64};
+//   tm_duc: dUcat [M, 2r] box {64, BN} SW128; tm_al: A [r, K] box {64, 64} SW128.
+cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap& tm_codes,
+                            const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a,
+                            cudaStream_t stream);
+
+// Skinny LoRA products with split contraction; see skinny.cu for the maps.
+cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
+                          int grid_rows, int splits, cudaStream_t stream);
+
+// Elementwise finishers (fixed-order sums over split partials).
+cudaError_t launch_finish_down(const float* P, int S, int M, int r, float s, float* U, uint16_t* ucat,
+                               cudaStream_t stream);
+cudaError_t launch_finish_du(const float* P, int S, int M, int r, float s, uint16_t* ducat, cudaStream_t stream);
+cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream);
+cudaError_t launch_finish_sum(const float* P, int S, int64_t count, float scale, float* out, cudaStream_t stream);
+cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32,
+                              cudaStream_t stream);
+
+}  // namespace qnf4

@@ -1,0 +1,106 @@
+// nf4_lut.cuh — NF4 level tables and the register lookups used by every kernel
+// that turns 4-bit codes into bf16 weights ("QLoRA" encyclopedia entry,
+// tonho.wtf, sections "a ideia" and "como funciona").
+#pragma once
+
+#include "sm100.cuh"
+
+namespace qnf4 {
+
+// Host-computed constants, passed to kernels by value (constant bank).
+//   q[16]     NF4 levels, ascending, fp32 (code i -> q[i]; q[7] = 0)
+//   thr/base  bucket table of the quantiser: bucket b = RNE(16 x + 16) covers
+//             x in [-1 + (b - 0.5)/16, -1 + (b + 0.5)/16], b = 0..32 (entry 63
+//             guards x < -1 - 1/32, which cannot occur); every bucket holds at
+//             most one midpoint m_i and none lies on a bucket edge, so
+//             code(x) = base[b] + (x > thr[b]).
+struct Nf4Tables {
+  float q[16];
+  float thr[64];
+  int base[64];
+};
+
+// Byte planes of a 16-entry bf16 table T[i] = bf16(RN32(q[i] * chat)):
+// L[k] holds the low bytes of T[4k..4k+3], H[k] the high bytes.
+struct Nf4Lut {
+  uint32_t L[4];
+  uint32_t H[4];
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Dequantised block constant chat = RN32(e4m3(c8) * s2).
+__device__ __forceinline__ float nf4_block_scale(uint32_t c8_byte, float s2) {
+  return __fmul_rn(e4m3_to_float(c8_byte), s2);
+}
+
+// The 16 dequantised values of one block, as byte planes.  Two separate
+// roundings per value: RN32 product, then RNE to bf16.
+__device__ __forceinline__ Nf4Lut nf4_make_lut(const Nf4Tables& tab, float chat) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    P[j] = pack_bf16x2(__fmul_rn(tab.q[2 * j], chat), __fmul_rn(tab.q[2 * j + 1], chat));
+  }
+  Nf4Lut t;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t.L[k] = prmt(P[2 * k], P[2 * k + 1], 0x6420u);
+    t.H[k] = prmt(P[2 * k], P[2 * k + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Four codes (nibbles 0..3 of c, element i in nibble i) -> four bf16 values,
+// returned as two packed pairs (element 0 in the low half of o01).
+__device__ __forceinline__ void nf4_lookup4(uint32_t c, const Nf4Lut& t, uint32_t& o01, uint32_t& o23) {
+  const uint32_t idx = c & 0x7777u;                                // entry within a half table
+  const uint32_t msk = prmt(0x0000FF00u, 0u, (c >> 3) & 0x1111u);  // 0xFF where code >= 8
+  const uint32_t la = prmt(t.L[0], t.L[1], idx);
+  const uint32_t lb = prmt(t.L[2], t.L[3], idx);
+  const uint32_t ha = prmt(t.H[0], t.H[1], idx);
+  const uint32_t hb = prmt(t.H[2], t.H[3], idx);
+  const uint32_t lo = (lb & msk) | (la & ~msk);
+  const uint32_t hi = (hb & msk) | (ha & ~msk);
+  o01 = prmt(lo, hi, 0x5140u);
+  o23 = prmt(lo, hi, 0x7362u);
+}
+
+// Eight codes (one 32-bit word of packed codes) -> eight bf16 values in a uint4.
+__device__ __forceinline__ uint4 nf4_lookup8(uint32_t w, const Nf4Lut& t) {
+  uint4 o;
+  nf4_lookup4(w, t, o.x, o.y);
+  nf4_lookup4(w >> 16, t, o.z, o.w);
+  return o;
+}
+
+// Dequantise one 64-element block (32 bytes of codes at `src`, 16-byte aligned)
+// into one 128-byte row of a 128-byte-swizzled shared-memory tile: the 16-byte
+// chunk j (elements 8j..8j+7) goes to position (j ^ swz).
+__device__ __forceinline__ void nf4_block_to_swizzled_row(const uint8_t* src, const Nf4Lut& t, uint8_t* dst_row,
+                                                          uint32_t swz) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(src);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (uint32_t j = 0; j < 8; ++j) {
+    *reinterpret_cast<uint4*>(dst_row + ((j ^ swz) << 4)) = nf4_lookup8(cw[j], t);
+  }
+}
+
+// Nearest-level code of a normalised value through the bucket table in shared
+// memory (lut[b] = (thr, base as int bits)).  The bucket is
+// b = RNE(16 x + 16), read from the low bits of a float whose ulp is 1
+// (1.5 * 2^23 + 16 is exact in fp32; the fma rounds once).
+__device__ __forceinline__ uint32_t nf4_code_of(float x, const float2* lut) {
+  const float t = fmaf(x, 16.0f, 12582928.0f);
+  const uint32_t b = __float_as_uint(t) & 63u;
+  const float2 e = lut[b];
+  return static_cast<uint32_t>(__float_as_int(e.y)) + (x > e.x ? 1u : 0u);
+}
+
+}  // namespace qnf4

@@ -1,0 +1,184 @@
+// quant.cu — NF4 blockwise quantisation with FP8 double quantisation, and the
+// standalone dequantisation ("QLoRA" encyclopedia entry, tonho.wtf, sections
+// "como funciona" and "a ideia").  Both kernels are HBM-bound streams.
+#include "kernels.h"
+#include "nf4_lut.cuh"
+
+namespace qnf4 {
+
+// ------------------------------------------------------------------ quantize
+//
+// One CTA (256 threads) owns one double-quantisation group: 256 blocks of 64
+// elements = 32 KB of bf16 input.  Eight threads share a block (8 elements,
+// 16 bytes each), so a warp reads 512 contiguous bytes per pass and writes
+// 128 contiguous bytes of codes; 8 passes cover the group.  All 8 loads of a
+// thread are issued before any arithmetic.  The block absmax is a max over
+// the bf16 magnitude bits (non-negative floats order like unsigned ints)
+// reduced across the 8 lanes with shuffles; the code search uses a bucket
+// table in shared memory (one fma, one load, one compare per element).
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ uint32_t max_abs_bits(uint4 v) {
+  // bf16 magnitudes of 8 elements, max over pairs with SIMD u16 max.
+  uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ uint32_t code_pair(uint32_t word, float rc, const float2* lut, uint32_t shift) {
+  const float a = __uint_as_float(word << 16);
+  const float b = __uint_as_float(word & 0xFFFF0000u);
+  const uint32_t ca = nf4_code_of(__fmul_rn(a, rc), lut);
+  const uint32_t cb = nf4_code_of(__fmul_rn(b, rc), lut);
+  return (ca | (cb << 4)) << shift;
+}
+
+// Codes of 8 elements where 1/c is not finite (c = 0, or c so small that the
+// reciprocal overflows): zero -> 7, positive -> 15, negative -> 0.
+__device__ __forceinline__ uint32_t codes_degenerate(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t b = (w[i] >> (16 * h)) & 0xFFFFu;
+      const uint32_t code = (b & 0x7FFFu) == 0 ? 7u : ((b & 0x8000u) ? 0u : 15u);
+      out |= code << (4 * (2 * i + h));
+    }
+  }
+  return out;
+}
+
+__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint16_t* __restrict__ w,
+                                                                      int64_t numel, uint8_t* __restrict__ codes,
+                                                                      uint8_t* __restrict__ c8,
+                                                                      float* __restrict__ s2, int32_t* status,
+                                                                      Nf4Tables tab) {
+  __shared__ float2 lut[64];
+  __shared__ uint32_t cblk[256];
+  __shared__ uint32_t wmax[kQuantThreads / 32];
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, sub = lane & 7;
+  if (tid < 64) lut[tid] = make_float2(tab.thr[tid], __int_as_float(tab.base[tid]));
+
+  const int64_t nblocks = (numel + 63) / 64;
+  const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * 256;
+  const bool full_group = (blk0 + 256) * 64 <= numel;
+
+  uint4 v[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int64_t e0 = (blk0 + p * 32 + warp * 4 + (lane >> 3)) * 64 + sub * 8;
+    if (full_group) {
+      v[p] = __ldg(reinterpret_cast<const uint4*>(w + e0));
+    } else {
+      uint32_t t[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (e0 + i < numel) t[i >> 1] |= static_cast<uint32_t>(w[e0 + i]) << (16 * (i & 1));
+      }
+      v[p] = make_uint4(t[0], t[1], t[2], t[3]);
+    }
+  }
+  __syncthreads();  // lut ready
+
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int lb = p * 32 + warp * 4 + (lane >> 3);
+    uint32_t m = max_abs_bits(v[p]);
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+    if (m > 0x7F7Fu && sub == 0 && status) atomicOr(status, QLORA_DEV_NONFINITE);
+    const float c = __uint_as_float(m << 16);
+    const float rc = __frcp_rn(c);
+    uint32_t out;
+    if (rc < __int_as_float(0x7F800000)) {
+      out = code_pair(v[p].x, rc, lut, 0) | code_pair(v[p].y, rc, lut, 8) | code_pair(v[p].z, rc, lut, 16) |
+            code_pair(v[p].w, rc, lut, 24);
+    } else {
+      out = codes_degenerate(v[p]);
+    }
+    const int64_t b = blk0 + lb;
+    if (b < nblocks) *reinterpret_cast<uint32_t*>(codes + b * 32 + sub * 4) = out;
+    if (sub == 0) cblk[lb] = m << 16;  // c as fp32 bits (0 for padding blocks)
+  }
+  __syncthreads();
+
+  // Double quantisation of the 256 constants of this group.
+  const uint32_t cbits = cblk[tid];
+  uint32_t amax = __reduce_max_sync(0xFFFFFFFFu, cbits);  // c >= 0: bit order = value order
+  if (lane == 0) wmax[warp] = amax;
+  __syncthreads();
+  amax = wmax[0];
+#pragma unroll
+  for (int i = 1; i < kQuantThreads / 32; ++i) amax = max(amax, wmax[i]);
+  const float scale = __fdiv_rn(__uint_as_float(amax), 448.0f);
+  const float y = scale > 0.0f ? __fdiv_rn(__uint_as_float(cbits), scale) : 0.0f;
+  const int64_t b = blk0 + tid;
+  if (b < nblocks) c8[b] = static_cast<uint8_t>(float_to_e4m3_satfinite(y));
+  if (tid == 0) s2[blockIdx.x] = scale;
+}
+
+// ---------------------------------------------------------------- dequantize
+//
+// One thread per half block: 16 bytes of codes in (a coalesced 128-bit load
+// across the warp), 64 bytes of bf16 out (four 128-bit stores).  The 16
+// dequantised values of the block are built once per thread as byte planes
+// and looked up with byte permutes (no per-element multiply).
+
+constexpr int kDequantThreads = 256;
+
+__global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                                          const uint8_t* __restrict__ c8,
+                                                                          const float* __restrict__ s2,
+                                                                          int64_t numel, uint16_t* __restrict__ out,
+                                                                          Nf4Tables tab) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDequantThreads + threadIdx.x;
+  const int64_t b = t >> 1;
+  const int h = static_cast<int>(t & 1);
+  const int64_t nblocks = (numel + 63) / 64;
+  if (b >= nblocks) return;
+  const float chat = nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8)));
+  const Nf4Lut lut = nf4_make_lut(tab, chat);
+  const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + b * 32 + h * 16));
+  uint4 o[4];
+  o[0] = nf4_lookup8(cw.x, lut);
+  o[1] = nf4_lookup8(cw.y, lut);
+  o[2] = nf4_lookup8(cw.z, lut);
+  o[3] = nf4_lookup8(cw.w, lut);
+  const int64_t e0 = b * 64 + h * 32;
+  if (e0 + 32 <= numel) {
+    uint4* dst = reinterpret_cast<uint4*>(out + e0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = o[i];
+  } else {
+    const uint16_t* vals = reinterpret_cast<const uint16_t*>(o);
+    for (int i = 0; i < 32; ++i)
+      if (e0 + i < numel) out[e0 + i] = vals[i];
+  }
+}
+
+// ------------------------------------------------------------------ launches
+
+cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                                int32_t* status, const Nf4Tables& tab, cudaStream_t stream) {
+  const int64_t ngroups = (numel + 16383) / 16384;
+  nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, stream>>>(w, numel, codes, c8, s2,
+                                                                                    status, tab);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
+                                  uint16_t* out, const Nf4Tables& tab, cudaStream_t stream) {
+  const int64_t nhalf = ((numel + 63) / 64) * 2;
+  const int64_t grid = (nhalf + kDequantThreads - 1) / kDequantThreads;
+  nf4_dequantize_kernel<<<static_cast<unsigned>(grid), kDequantThreads, 0, stream>>>(codes, c8, s2, numel, out,
+                                                                                      tab);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

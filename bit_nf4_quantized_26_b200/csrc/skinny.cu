@@ -1,0 +1,325 @@
+// skinny.cu — the rank-r products of the LoRA adapter path ("QLoRA"
+// encyclopedia entry, tonho.wtf, section "a ideia": the adapters stay in 16 bit
+// and are the only parameters that receive gradients).
+//
+//   mode DOWN:  P[m, j]  = sum_k X[m,k]  A[j,k]      (U = X A^T)
+//   mode DU:    P[m, j]  = sum_n dY[m,n] B[n,j]      (dU = s dY B)
+//   mode DB:    P[n, j]  = sum_m dY[m,n] sU[m,j]     (dB = s dY^T U)
+//   mode DA:    P[j, k]  = sum_m dU[m,j] X[m,k]      (dA = dU^T X)
+//
+// Each is a tcgen05 GEMM with M = 128 rows and a narrow N, streaming its long
+// operand through a TMA ring; the contraction is split across blockIdx.y
+// slices and the fp32 partials are summed in a fixed order by a finisher, so
+// results are deterministic.  The fp32 operands (sU, dU) enter the tensor core
+// as a bf16 hi/lo pair in the interleaved "hi/lo per 16" column layout:
+// column c holds part (c/16)%2 (0 = hi, 1 = lo) of j = 16*(c/32) + c%16.
+#include "kernels.h"
+
+namespace qnf4 {
+
+__device__ __forceinline__ void sk_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
+  }
+}
+
+template <int MODE>
+struct SkPlan {
+  static constexpr uint32_t kA = 16384;
+  static constexpr uint32_t kB = MODE == kSkDA ? 32768 : (MODE == kSkDB ? 16384 : 8192);
+  static constexpr uint32_t kStage = kA + kB;
+  static constexpr uint32_t kFit = (232448u - 2048u) / kStage;
+  static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
+  static constexpr uint32_t kBarOff = kStages * kStage;
+  static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
+  static constexpr uint32_t kTmemCols = MODE == kSkDA ? 256 : (MODE == kSkDB ? 128 : 64);
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(192, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const SkinnyArgs a) {
+  using P = SkPlan<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
+  uint64_t* empty = full + P::kStages;
+  uint64_t* accf = empty + P::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Tile origin: DOWN/DU rows are tokens, DB rows are output features, DA's
+  // 128 rows are the hi/lo columns of dU and blockIdx.x walks K in 256s.
+  const int row0 = blockIdx.x * (MODE == kSkDA ? 256 : 128);
+  const int z = blockIdx.y;
+  const int st0 = z * a.stages_per_split;
+  const int T = min(a.stages_total, st0 + a.stages_per_split) - st0;
+  const int nc = (2 * a.r > 64) ? 128 : 64;  // DB: width of the sU operand
+
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < P::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, P::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  const WaitCtx wc{abort_flag, a.status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (t >= static_cast<int>(P::kStages) && !mbar_wait(&empty[s], (u - 1) & 1, wc)) break;
+        uint8_t* sa = smem + s * P::kStage;
+        uint8_t* sb = sa + P::kA;
+        const int kt = st0 + t;
+        if (MODE == kSkDown || MODE == kSkDU) {
+          mbar_arrive_expect_tx(&full[s], 16384 + 8192);
+          tma_load_2d(sa, &tmA, &full[s], kt * 64, row0);
+          if (MODE == kSkDown) tma_load_2d(sb, &tmB, &full[s], kt * 64, 0);
+          else tma_load_2d(sb, &tmB, &full[s], 0, kt * 64);
+        } else if (MODE == kSkDB) {
+          const bool a2 = row0 + 64 < a.N;
+          mbar_arrive_expect_tx(&full[s], 8192u * ((a2 ? 2 : 1) + nc / 64));
+          tma_load_2d(sa, &tmA, &full[s], row0, kt * 64);
+          if (a2) tma_load_2d(sa + 8192, &tmA, &full[s], row0 + 64, kt * 64);
+          tma_load_2d(sb, &tmB, &full[s], 0, kt * 64);
+          if (nc == 128) tma_load_2d(sb + 8192, &tmB, &full[s], 64, kt * 64);
+        } else {  // DA
+          int nb = 0;
+          for (int i = 0; i < 4; ++i) nb += (row0 + 64 * i < a.K) ? 1 : 0;
+          mbar_arrive_expect_tx(&full[s], 8192u * ((nc / 64) + nb));
+          tma_load_2d(sa, &tmA, &full[s], 0, kt * 64);
+          if (nc == 128) tma_load_2d(sa + 8192, &tmA, &full[s], 64, kt * 64);
+          for (int i = 0; i < nb; ++i) tma_load_2d(sb + 8192 * i, &tmB, &full[s], row0 + 64 * i, kt * 64);
+        }
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
+        sk_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool a_mn = (MODE == kSkDB || MODE == kSkDA);
+      const bool b_mn = (MODE != kSkDown);
+      const int n = MODE == kSkDA ? 256 : (MODE == kSkDB ? nc : 64);
+      const uint32_t idesc = idesc_bf16_f32(128, n, a_mn ? 1 : 0, b_mn ? 1 : 0);
+      const uint32_t a_step = a_mn ? (2048u >> 4) : (32u >> 4);
+      const uint32_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
+      bool aborted = false;
+      for (int t = 0; t < T; ++t) {
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * P::kStage), sb = sa + P::kA;
+        const uint64_t adesc = a_mn ? sdesc_sw128(sa, 8192, 1024) : sdesc_sw128(sa, 16, 1024);
+        const uint64_t bdesc = b_mn ? sdesc_sw128(sb, 8192, 1024) : sdesc_sw128(sb, 16, 1024);
+#pragma unroll
+        for (uint32_t kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem_d, adesc + kk * a_step, bdesc + kk * b_step, idesc, (t | kk) != 0 ? 1u : 0u);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+      if (aborted) sk_wait_drain(accf, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    const int rl = q * 32 + lane;
+    if (mbar_wait(accf, 0, wc)) {
+      tc_fence_after();
+      const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+      if (MODE == kSkDown || MODE == kSkDU) {
+        const int m = row0 + rl;
+        float* out = a.partial + (static_cast<int64_t>(z) * a.M + m) * a.r;
+        for (int cb = 0; cb < (a.r + 31) / 32; ++cb) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tq + cb * 32, v);
+          tmem_ld_wait();
+          if (m < a.M) {
+            const int nv = min(32, a.r - cb * 32);
+            for (int j = 0; j < nv; j += 4)
+              *reinterpret_cast<float4*>(out + cb * 32 + j) =
+                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                              __uint_as_float(v[j + 3]));
+          }
+        }
+      } else if (MODE == kSkDB) {
+        const int n = row0 + rl;
+        float* out = a.partial + (static_cast<int64_t>(z) * a.N + n) * a.r;
+        for (int g = 0; g < a.r / 16; ++g) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tq + g * 32, v);
+          tmem_ld_wait();
+          if (n < a.N) {
+            for (int j = 0; j < 16; j += 4)
+              *reinterpret_cast<float4*>(out + g * 16 + j) = make_float4(
+                  __uint_as_float(v[j]) + __uint_as_float(v[j + 16]),
+                  __uint_as_float(v[j + 1]) + __uint_as_float(v[j + 17]),
+                  __uint_as_float(v[j + 2]) + __uint_as_float(v[j + 18]),
+                  __uint_as_float(v[j + 3]) + __uint_as_float(v[j + 19]));
+          }
+        }
+      } else {  // DA: rows c = 32q + lane; hi row (lane < 16) plus lo row (lane + 16)
+        const int j = 16 * q + lane;
+        const bool jok = lane < 16 && j < a.r;
+        for (int cb = 0; cb < 8; ++cb) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tq + cb * 32, v);
+          tmem_ld_wait();
+          float sum[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float lo = __shfl_down_sync(0xFFFFFFFFu, __uint_as_float(v[i]), 16);
+            sum[i] = __uint_as_float(v[i]) + lo;
+          }
+          const int k = row0 + cb * 32;
+          if (jok && k < a.K) {
+            float* out = a.partial + (static_cast<int64_t>(z) * a.r + j) * a.K + k;
+            const int nv = min(32, a.K - k);
+            for (int i = 0; i < nv; i += 4)
+              *reinterpret_cast<float4*>(out + i) = make_float4(sum[i], sum[i + 1], sum[i + 2], sum[i + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, P::kTmemCols);
+  }
+}
+
+template <int MODE>
+static cudaError_t launch_skinny_impl(const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
+                                      int grid_rows, int splits, cudaStream_t stream) {
+  using P = SkPlan<MODE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(skinny_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(P::kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  skinny_kernel<MODE><<<dim3(grid_rows, splits), 192, P::kSmem, stream>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
+                          int grid_rows, int splits, cudaStream_t stream) {
+  switch (mode) {
+    case kSkDown: return launch_skinny_impl<kSkDown>(tmA, tmB, a, grid_rows, splits, stream);
+    case kSkDU: return launch_skinny_impl<kSkDU>(tmA, tmB, a, grid_rows, splits, stream);
+    case kSkDB: return launch_skinny_impl<kSkDB>(tmA, tmB, a, grid_rows, splits, stream);
+    case kSkDA: return launch_skinny_impl<kSkDA>(tmA, tmB, a, grid_rows, splits, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ------------------------------------------------------------------ finishers
+
+__device__ __forceinline__ int hilo_col(int j) { return 32 * (j >> 4) + (j & 15); }
+
+// v -> (bf16(v), bf16(v - bf16(v))) at the interleaved hi/lo columns of row m.
+__device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int r, int j, float v) {
+  const uint16_t hi = bf16_bits(v);
+  const uint16_t lo = bf16_bits(__fsub_rn(v, bf16_bits_to_float(hi)));
+  uint16_t* row = cat + static_cast<int64_t>(m) * 2 * r;
+  row[hilo_col(j)] = hi;
+  row[hilo_col(j) + 16] = lo;
+}
+
+__global__ void finish_down_kernel(const float* __restrict__ P, int S, int M, int r, float s, float* __restrict__ U,
+                                   uint16_t* __restrict__ ucat) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(M) * r;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  U[i] = acc;
+  store_hilo(ucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
+}
+
+__global__ void finish_du_kernel(const float* __restrict__ P, int S, int M, int r, float s,
+                                 uint16_t* __restrict__ ducat) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(M) * r;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  store_hilo(ducat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
+}
+
+__global__ void prep_su_kernel(const float* __restrict__ U, int M, int r, float s, uint16_t* __restrict__ sucat) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n = static_cast<int64_t>(M) * r;
+  if (i >= n) return;
+  store_hilo(sucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, U[i]));
+}
+
+__global__ void finish_sum_kernel(const float* __restrict__ P, int S, int64_t n, float scale,
+                                  float* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  out[i] = scale == 1.0f ? acc : __fmul_rn(scale, acc);
+}
+
+__global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n, void* __restrict__ out,
+                                  int out_f32) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = 0.f;
+  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  if (out_f32) reinterpret_cast<float*>(out)[i] = acc;
+  else reinterpret_cast<uint16_t*>(out)[i] = bf16_bits(acc);
+}
+
+static inline unsigned blocks_for(int64_t n) { return static_cast<unsigned>((n + 255) / 256); }
+
+cudaError_t launch_finish_down(const float* P, int S, int M, int r, float s, float* U, uint16_t* ucat,
+                               cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(M) * r;
+  finish_down_kernel<<<blocks_for(n), 256, 0, stream>>>(P, S, M, r, s, U, ucat);
+  return cudaGetLastError();
+}
+cudaError_t launch_finish_du(const float* P, int S, int M, int r, float s, uint16_t* ducat, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(M) * r;
+  finish_du_kernel<<<blocks_for(n), 256, 0, stream>>>(P, S, M, r, s, ducat);
+  return cudaGetLastError();
+}
+cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(M) * r;
+  prep_su_kernel<<<blocks_for(n), 256, 0, stream>>>(U, M, r, s, sucat);
+  return cudaGetLastError();
+}
+cudaError_t launch_finish_sum(const float* P, int S, int64_t count, float scale, float* out, cudaStream_t stream) {
+  finish_sum_kernel<<<blocks_for(count), 256, 0, stream>>>(P, S, count, scale, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32, cudaStream_t stream) {
+  finish_out_kernel<<<blocks_for(count), 256, 0, stream>>>(P, S, count, out, out_f32);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

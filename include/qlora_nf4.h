@@ -1,0 +1,198 @@
+/*
+ * qlora_nf4.h — C ABI of the NF4 / QLoRA linear-layer library for sm_100a (B200).
+ *
+ * What the library computes (sources are web pages, cited by title and section):
+ *
+ *  - "QLoRA" encyclopedia entry (tonho.wtf), section "como funciona": a 4-bit
+ *    storage type (NF4) built from standard-normal quantiles, asymmetric so that
+ *    zero is exact; blockwise absmax quantisation with one constant per 64
+ *    elements; the constants themselves quantised to FP8 in blocks of 256.
+ *  - same entry, section "a ideia": weights are stored in 4 bit and dequantised
+ *    to BFloat16 only when used in a matmul; the gradient crosses the frozen
+ *    weight and lands in the 16-bit LoRA adapters, the only trainable parameters.
+ *  - "Tutorial fine-tuning LLM LoRA/QLoRA 2026" (nexusinovation), section
+ *    "LoRA: O Padrão Ouro de Eficiência": the adapter adds a scaled low-rank
+ *    product to the frozen weight; "Mão na Massa" shows the knobs
+ *    (r, lora_alpha, nf4, bf16 compute, double quant).
+ *
+ * Notation: W is [N = out, K = in] row-major (PyTorch Linear layout); X is
+ * [M, K]; Y is [M, N]; the adapters are A [r, K] and B [N, r], all row-major;
+ * s = alpha / r.  bf16 tensors are passed as uint16_t bit patterns.
+ *
+ *   forward:   U = X A^T (fp32)           Y = X W'^T + s U B^T
+ *   backward:  dU = s dY B                dX = dY W' + dU A
+ *              dA = dU^T X                dB = s dY^T U
+ *
+ * where W' = dequantize(NF4(W)) in bf16.  There is no dW (the base is frozen).
+ *
+ * NF4 storage of a tensor of `numel` elements (flattened row-major):
+ *   codes  uint8[ceil(numel/64)*32]  two 4-bit codes per byte; element 2j in
+ *                                    the low nibble of byte j; code i is the
+ *                                    i-th NF4 level in ascending order
+ *                                    (code 7 is the exact zero)
+ *   c8     uint8[ceil(numel/64)]     FP8 E4M3 absmax constant per 64 elements
+ *   s2     float[ceil(numel/16384)]  fp32 scale per group of 256 constants
+ *
+ * Conventions common to every entry point:
+ *  - Ownership: the caller allocates and owns every buffer (device memory
+ *    unless stated).  The library never allocates or frees device memory and
+ *    keeps no state beyond host-side constant tables and cached device
+ *    attributes.
+ *  - Asynchrony: every compute call only enqueues work on `stream` (a
+ *    cudaStream_t; NULL = legacy default stream) and returns.  The returned
+ *    status covers the synchronous argument checks and launch errors only.
+ *  - Device-side conditions (non-finite input, a bounded wait that ran out)
+ *    are OR-ed into the optional device word `d_status` (int32, caller
+ *    zeroes it; NULL = not reported): bit 0 = QLORA_DEV_NONFINITE,
+ *    bit 1 = QLORA_DEV_TIMEOUT.
+ *  - Alignment: every pointer must be 16-byte aligned (QLORA_ERR_ALIGN).
+ *  - Errors are reported before any work is enqueued; on error nothing runs.
+ *  - Only sm_100 devices are supported (QLORA_ERR_ARCH); there is no fallback.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_NULL = 1,       /* a required pointer is NULL                       */
+  QLORA_ERR_SHAPE = 2,      /* a size violates the documented constraints      */
+  QLORA_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned                */
+  QLORA_ERR_WORKSPACE = 4,  /* workspace NULL or smaller than the size query   */
+  QLORA_ERR_NONFINITE = 5,  /* (reserved for host-visible non-finite reports)  */
+  QLORA_ERR_TIMEOUT = 6,    /* (reserved for host-visible timeout reports)     */
+  QLORA_ERR_CUDA = 7,       /* a CUDA runtime/driver call failed               */
+  QLORA_ERR_ARCH = 8,       /* current device is not sm_100                    */
+  QLORA_ERR_DTYPE = 9       /* unknown output dtype code                       */
+} qlora_status;
+
+/* Device status bits OR-ed into d_status by the kernels. */
+#define QLORA_DEV_NONFINITE 1
+#define QLORA_DEV_TIMEOUT 2
+
+/* Output dtype codes for Y and dX. */
+#define QLORA_DTYPE_BF16 0
+#define QLORA_DTYPE_F32 1
+
+/* A quantised weight [n_out, k_in]: views into caller-owned device memory. */
+typedef struct {
+  const uint8_t* codes; /* uint8[n_out*k_in/2]           */
+  const uint8_t* c8;    /* uint8[n_out*k_in/64]          */
+  const float* s2;      /* float[ceil(n_out*k_in/16384)] */
+  int64_t n_out;
+  int64_t k_in;
+} nf4_weight;
+
+/*
+ * nf4_quantize — NF4 blockwise quantisation with FP8 double quantisation
+ * ("QLoRA" entry, "como funciona").
+ *
+ *  w_bf16  [numel] bf16 input (device)
+ *  numel   > 0, any value; the last 64-block is padded with +0 (code 7) and
+ *          the last 256-constant group with zero constants
+ *  codes   [ceil(numel/64)*32] out; c8 [ceil(numel/64)] out; s2 [ceil(numel/16384)] out
+ *  d_status optional device word (see above); a non-finite input sets
+ *          QLORA_DEV_NONFINITE and leaves the affected outputs unspecified
+ *
+ * Per block of 64: c = max|w|; x = RN32(w * RN32(1/c)); code = #{i: x > m_i}
+ * with m_i the fp32 midpoints of adjacent levels (ties go to the lower code;
+ * zero is always code 7).  Per group of 256 constants: s2 = RN32(amax/448);
+ * c8 = E4M3 round-to-nearest-even, saturating (RN32(c/s2)).  Bit-exact with
+ * the CPU oracle.  numel == 0 is a no-op.
+ */
+QLORA_API qlora_status nf4_quantize(const uint16_t* w_bf16, int64_t numel, uint8_t* codes, uint8_t* c8,
+                          float* s2, int32_t* d_status, void* stream);
+
+/*
+ * nf4_dequantize — bf16 weights from NF4 storage ("a ideia": dequantised to
+ * BFloat16 at use).  w' = bf16(RN32(q[code] * RN32(e4m3(c8) * s2))), two
+ * separate roundings.  Writes exactly numel bf16 values.  numel == 0 is a
+ * no-op.
+ */
+QLORA_API qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2,
+                            int64_t numel, uint16_t* w_bf16, void* stream);
+
+/*
+ * qlora_linear_fwd — Y = X W'^T + s (X A^T) B^T with W' dequantised inside the
+ * tensor-core GEMM (the bf16 weight never reaches global memory).
+ *
+ *  X      [M, K] bf16;  W: NF4 weight with n_out = N, k_in = K
+ *  A      [r, K] bf16;  B [N, r] bf16;  s scalar (alpha / r)
+ *  Y      [M, N] out, bf16 or fp32 per y_dtype
+ *  U_out  [M, r] fp32 out: U = X A^T, to be passed back to qlora_linear_bwd
+ *  ws     device workspace of at least qlora_fwd_workspace_size(M, N, K, r) bytes
+ *
+ * Constraints: M >= 0 (0 = no-op), K % 64 == 0, N % 64 == 0, K >= 64,
+ * N >= 64, r % 16 == 0 and 16 <= r <= 64, M < 2^31, N*K < 2^40.
+ * Accuracy: fp32 accumulation over exact bf16 inputs; relative Frobenius
+ * error of Y within 2e-3 of the fp64 product on the same dequantised weights.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A,
+                              const uint16_t* B, int32_t r, float s, void* Y, int32_t y_dtype,
+                              float* U_out, void* ws, size_t ws_bytes, int32_t* d_status,
+                              void* stream);
+
+/*
+ * qlora_linear_bwd — gradients through the frozen NF4 weight into the adapters.
+ *
+ *  dY [M, N] bf16; X [M, K] bf16; U [M, r] fp32 (from qlora_linear_fwd)
+ *  dX [M, K] out (bf16 or fp32 per dx_dtype) = dY W' + (s dY B) A
+ *  dA [r, K] fp32 out = (s dY B)^T X;  dB [N, r] fp32 out = s dY^T U
+ *  ws device workspace of at least qlora_bwd_workspace_size(M, N, K, r) bytes
+ *
+ * Same constraints as the forward.  dA and dB are overwritten (not
+ * accumulated); their reductions over tokens run in a fixed order, so repeated
+ * calls give bitwise-identical results.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M,
+                              nf4_weight W, const uint16_t* A, const uint16_t* B, int32_t r,
+                              float s, void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws,
+                              size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* Workspace sizes in bytes (0 when M == 0).  Pure host functions. */
+QLORA_API size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
+QLORA_API size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
+
+/*
+ * nf4_levels — the 16 fp32 NF4 levels the kernels use, ascending (code i ->
+ * out[i]; out[7] == 0).  Host-only, needs no device.  The library derives
+ * them itself from the standard-normal quantile construction of "como
+ * funciona" (outermost probability (1-1/30 + 1-1/32)/2, the reading also used
+ * by the CPU oracle), by bisection on the normal CDF in double precision.
+ */
+QLORA_API void nf4_levels(float out[16]);
+
+/*
+ * Kernel timing (diagnostics).  While enabled, every kernel this library
+ * launches is bracketed by a pair of CUDA events recorded on the launch
+ * stream (the events are library-owned host objects; no device memory is
+ * allocated).  qlora_profile_collect waits for the recorded events, writes up
+ * to `capacity` (kernel id, milliseconds) pairs in launch order, clears the
+ * record list and returns the number of records (or -1 on a CUDA error).
+ * qlora_kernel_name maps an id to a static name.  Not thread-safe with
+ * respect to concurrent launches from several host threads.
+ */
+QLORA_API void qlora_profile_enable(int32_t enable);
+QLORA_API int32_t qlora_profile_collect(int32_t* kernel_ids, float* ms, int32_t capacity);
+QLORA_API const char* qlora_kernel_name(int32_t kernel_id);
+
+/* Static, NUL-terminated description of a status code. */
+QLORA_API const char* qlora_strerror(qlora_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

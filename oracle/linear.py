@@ -52,13 +52,13 @@ def linear_fwd(X, Wd, A, B, s):
     return U, Y
 
 
-def linear_bwd(dY, X, Wd, A, B, s):
-    """Return (dX, dA, dB, dU) in fp64."""
-    dY, X, Wd, A, B = _f64(dY), _f64(X), _f64(Wd), _f64(A), _f64(B)
+def linear_bwd(dY, X, Wd, A, B, s, want_dx=True):
+    """Return (dX, dA, dB, dU) in fp64 (dX is None when ``want_dx`` is False)."""
+    dY, X, A, B = _f64(dY), _f64(X), _f64(A), _f64(B)
     s = float(s)
     U = X @ A.T
     dU = s * (dY @ B)
-    dX = dY @ Wd + dU @ A
+    dX = dY @ _f64(Wd) + dU @ A if want_dx else None
     dA = dU.T @ X
     dB = s * (dY.T @ U)
     return dX, dA, dB, dU

@@ -118,15 +118,18 @@ def encode_codes(w_bits, numel, c):
     block, then one rounded product per element (the page says "normalise by
     the absolute maximum" without fixing the arithmetic; this is the reading).
     Nearest level: code = #{i : x > m_i}.  A value exactly on a midpoint goes
-    to the lower code; -0 goes to code 7.  A block with c = 0 is all code 7.
+    to the lower code.  A zero weight (+0 or -0) is always code 7, the exact
+    zero level ("como funciona": zero padding quantises without error); this
+    also covers blocks with c = 0 and blocks so small that RN32(1/c)
+    overflows, where the product would be 0 * inf.
     """
     w = _blocks(w_bits, numel)
     c = np.asarray(c, dtype=np.float32)
-    with np.errstate(divide="ignore", invalid="ignore"):
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
         rc = np.float32(1.0) / c
         x = (w * rc[:, None]).astype(np.float32)
     codes = nearest_code(x)
-    codes[c == 0] = 7
+    codes[w == 0] = 7
     return codes
 
 

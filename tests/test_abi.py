@@ -1,0 +1,124 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared
+symbol, derives the same NF4 levels as the oracle, sizes its workspaces, and
+rejects bad arguments before touching a device.  No GPU needed; no test here
+enqueues device work."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import bit_nf4_quantized_26_b200 as q
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+OK, NULL, SHAPE, ALIGN, WS, CUDA, ARCH, DTYPE = 0, 1, 2, 3, 4, 7, 8, 9
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert len(names) == 11
+    lib = q.raw()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(q.EXPORTED) == names
+
+
+def test_library_levels_equal_oracle_codebook():
+    """The library's codebook (bisection on erfc, C++) and the oracle's
+    (Wichura AS241, Python) are independent derivations of the same levels."""
+    lib_levels = np.array(q.nf4_levels(), dtype=np.float32)
+    assert np.array_equal(lib_levels.view(np.uint32), nf4.codebook().view(np.uint32))
+
+
+def test_strerror():
+    for code in range(10):
+        assert isinstance(q.qlora_strerror(code), str) and q.qlora_strerror(code)
+    assert q.qlora_strerror(0) == "ok"
+
+
+def test_workspace_sizes():
+    assert q.qlora_fwd_workspace_size(0, 4096, 4096, 64) == 0
+    assert q.qlora_bwd_workspace_size(0, 4096, 4096, 64) == 0
+    a = q.qlora_fwd_workspace_size(4096, 4096, 4096, 64)
+    b = q.qlora_fwd_workspace_size(8192, 4096, 4096, 64)
+    assert 0 < a <= b
+    assert q.qlora_fwd_workspace_size(4096, 4096, 4096, 64) % 256 == 0
+    assert q.qlora_bwd_workspace_size(4096, 4096, 4096, 64) >= 4096 * 2 * 64 * 2 * 2
+    # small M uses split-K partials: still bounded by S * M * N * 4
+    assert q.qlora_fwd_workspace_size(1, 22016, 8192, 64) < 300 * 22016 * 4 + (1 << 20)
+
+
+# ----------------------------------------------------------- argument checks
+
+FAKE = 1 << 20  # a 16-byte aligned non-null value; never dereferenced
+
+
+def _w(codes=FAKE, c8=FAKE, s2=FAKE, n=4096, k=4096):
+    return q._NF4Weight(codes, c8, s2, n, k)
+
+
+def _fwd(X=FAKE, M=64, W=None, A=FAKE, B=FAKE, r=64, Y=FAKE, ydt=0, U=FAKE, ws=FAKE, wsb=1 << 40,
+         status=None):
+    W = _w() if W is None else W
+    return q.raw().qlora_linear_fwd(X, M, W, A, B, r, 0.25, Y, ydt, U, ws, wsb, status, None)
+
+
+def _bwd(dY=FAKE, X=FAKE, U=FAKE, M=64, W=None, A=FAKE, B=FAKE, r=64, dX=FAKE, dxdt=0, dA=FAKE, dB=FAKE,
+         ws=FAKE, wsb=1 << 40):
+    W = _w() if W is None else W
+    return q.raw().qlora_linear_bwd(dY, X, U, M, W, A, B, r, 0.25, dX, dxdt, dA, dB, ws, wsb, None, None)
+
+
+def test_fwd_argument_errors():
+    assert _fwd(X=None) == NULL
+    assert _fwd(W=_w(codes=None)) == NULL
+    assert _fwd(U=None) == NULL
+    assert _fwd(W=_w(k=4096 + 32)) == SHAPE          # K % 64 != 0
+    assert _fwd(W=_w(n=4096 + 16)) == SHAPE          # N % 64 != 0
+    assert _fwd(r=8) == SHAPE and _fwd(r=24) == SHAPE and _fwd(r=128) == SHAPE
+    assert _fwd(M=-1) == SHAPE
+    assert _fwd(X=FAKE + 8) == ALIGN
+    assert _fwd(W=_w(c8=FAKE + 4)) == ALIGN
+    assert _fwd(ydt=7) == DTYPE
+    assert _fwd(ws=None) == WS
+    assert _fwd(wsb=16) == WS
+    assert _fwd(M=0, X=None, Y=None, U=None, ws=None) == OK   # no-op
+
+
+def test_bwd_argument_errors():
+    assert _bwd(dY=None) == NULL
+    assert _bwd(dB=None) == NULL
+    assert _bwd(W=_w(k=100)) == SHAPE
+    assert _bwd(dA=FAKE + 2) == ALIGN
+    assert _bwd(dxdt=3) == DTYPE
+    assert _bwd(wsb=0) == WS
+    assert _bwd(M=0, dY=None) == OK
+
+
+def test_quantize_argument_errors():
+    lib = q.raw()
+    assert lib.nf4_quantize(None, 64, FAKE, FAKE, FAKE, None, None) == NULL
+    assert lib.nf4_quantize(FAKE, -5, FAKE, FAKE, FAKE, None, None) == SHAPE
+    assert lib.nf4_quantize(FAKE + 2, 64, FAKE, FAKE, FAKE, None, None) == ALIGN
+    assert lib.nf4_quantize(None, 0, None, None, None, None, None) == OK
+    assert lib.nf4_dequantize(FAKE, None, FAKE, 64, FAKE, None) == NULL
+    assert lib.nf4_dequantize(FAKE, FAKE, FAKE, 64, FAKE + 1, None) == ALIGN
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would reach the device with fake pointers")
+def test_valid_arguments_without_device_fail_cleanly():
+    """With every argument valid but no usable sm_100 device the call returns an
+    error status (never crashes, never falls back)."""
+    assert _fwd() in (CUDA, ARCH)
+    assert q.raw().nf4_quantize(FAKE, 64, FAKE, FAKE, FAKE, None, None) in (CUDA, ARCH)

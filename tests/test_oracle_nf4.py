@@ -149,6 +149,16 @@ def test_zero_block_and_padding_are_exact():
     assert np.all(nf4.dequantize(p2, c82, s22, 64) == 0x0000)
 
 
+def test_tiny_block_constant():
+    """A block whose absmax is so small that 1/c overflows still codes zero as 7."""
+    w = np.zeros(64, dtype=np.uint16)
+    w[0] = 0x0001                    # smallest positive bf16 subnormal: 1/c = inf
+    w[1] = 0x8001                    # its negative
+    packed, c8, s2 = nf4.quantize(w)
+    codes = nf4.unpack_codes(packed, 64)
+    assert codes[0] == 15 and codes[1] == 0 and np.all(codes[2:] == 7)
+
+
 def test_codebook_values_round_trip():
     q = nf4.codebook()
     qb = nm.f32_to_bf16_bits(q)
