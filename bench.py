@@ -190,7 +190,7 @@ def run_ours(args, rank, world):
     wl = synth.WORKLOADS[WORKLOAD]
     lin = wl.linears[0]
     M, N, K, r, s = wl.m_tokens, lin.n_out, lin.k_in, wl.r, wl.s
-    d = synth.linear_inputs(lin, M, r, seed=rank)
+    d = synth.dp_shard_inputs(lin, M, r, rank)
     g = {k: v.to(dev) for k, v in d.items()}
     W_bf16 = g["W"]
     nc, nb, ns = lib.nf4_sizes(N * K)

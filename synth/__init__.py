@@ -124,6 +124,15 @@ def linear_inputs(lin, m_tokens, r, seed, outliers=False, device="cpu"):
     }
 
 
+def dp_shard_inputs(lin, m_per_rank, r, rank, seed=0, outliers=False, device="cpu"):
+    """Data-parallel inputs: every rank holds the same frozen weight and
+    adapters (drawn with ``seed``) and its own batch of tokens (drawn with a
+    seed derived from ``rank``)."""
+    shared = linear_inputs(lin, 1, r, seed, outliers, device)
+    own = linear_inputs(lin, m_per_rank, r, seed + 1 + rank, outliers, device)
+    return {"W": shared["W"], "A": shared["A"], "B": shared["B"], "X": own["X"], "dY": own["dY"]}
+
+
 def workload_inputs(name, index=0, seed=0, device="cpu", m_tokens=None):
     """Inputs of linear ``index`` of workload ``name`` (seed offset per linear)."""
     wl = WORKLOADS[name]
