@@ -72,6 +72,9 @@ _lib.nf4_levels.argtypes = [_P]
 _lib.nf4_levels.restype = None
 _lib.qlora_strerror.argtypes = [ctypes.c_int]
 _lib.qlora_strerror.restype = ctypes.c_char_p
+_lib.qlora_linear_fwd_noalloc.argtypes = [_P, _I64, _NF4Weight, _P, _P, _I32, ctypes.c_float, _P, _I32, _P, _P,
+                                          _P]
+_lib.qlora_linear_fwd_noalloc.restype = ctypes.c_int
 _lib.qlora_profile_enable.argtypes = [_I32]
 _lib.qlora_profile_enable.restype = None
 _lib.qlora_profile_collect.argtypes = [_P, _P, _I32]
@@ -81,7 +84,7 @@ _lib.qlora_kernel_name.restype = ctypes.c_char_p
 
 EXPORTED = ("nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
             "qlora_fwd_workspace_size", "qlora_bwd_workspace_size", "nf4_levels", "qlora_strerror",
-            "qlora_profile_enable", "qlora_profile_collect", "qlora_kernel_name")
+            "qlora_profile_enable", "qlora_profile_collect", "qlora_kernel_name", "qlora_linear_fwd_noalloc")
 
 NF4Weight = namedtuple("NF4Weight", "codes c8 s2 n_out k_in")
 
@@ -171,6 +174,24 @@ def qlora_linear_fwd(X, W, A, B, s, y_dtype=DTYPE_BF16, Y=None, U=None, ws=None,
     _check(_lib.qlora_linear_fwd(_ptr(X), M, _weight(W), _ptr(A), _ptr(B), r, float(s), _ptr(Y), y_dtype,
                                  _ptr(U), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
            "qlora_linear_fwd")
+    return Y, U
+
+
+def qlora_linear_fwd_noalloc(X, W, A, B, s, y_dtype=DTYPE_BF16, Y=None, U=None, status=None, stream=None):
+    """Forward without a workspace, for callers that cannot allocate device
+    memory at call time (the library keeps a fixed 16 MiB scratch array per
+    device; problems that need more are rejected).  Returns ``(Y, U)``.  The
+    output tensors are allocated here only when not given."""
+    M = X.shape[0]
+    N, r = int(W.n_out), A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32 if y_dtype == DTYPE_F32 else torch.bfloat16, device=dev)
+    if U is None:
+        U = torch.empty((M, r), dtype=torch.float32, device=dev)
+    _check(_lib.qlora_linear_fwd_noalloc(_ptr(X), M, _weight(W), _ptr(A), _ptr(B), r, float(s), _ptr(Y), y_dtype,
+                                         _ptr(U), _ptr(status), _stream(stream)),
+           "qlora_linear_fwd_noalloc")
     return Y, U
 
 

@@ -166,6 +166,35 @@ QLORA_API size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32
 QLORA_API size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
 
 /*
+ * qlora_linear_fwd_noalloc — the forward of qlora_linear_fwd for callers that
+ * cannot provide a workspace.  The pages have no counterpart; it exists for
+ * callers that may not allocate device memory at call time: a plugin that a
+ * host framework hands only its input and output buffers (the framework owns
+ * the device memory pool), or a latency-critical loop that must not call
+ * cudaMalloc/cudaFree because they can synchronise the device.
+ *
+ * Same arguments, constraints, results and accuracy as qlora_linear_fwd
+ * (Y and U_out are caller-owned device buffers), minus the workspace: the
+ * scratch lives in a 16 MiB array of device memory declared statically by
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  The library allocates nothing here.
+ *  - Limit: problems whose qlora_fwd_workspace_size(M, N, K, r) exceeds
+ *    16 MiB (16777216 bytes) are rejected with QLORA_ERR_WORKSPACE before any
+ *    work is enqueued (e.g. 4096 tokens on 4096x4096 with r=64 fits).
+ *  - Set-up: the first call on each device (with that device current) looks
+ *    up the array's device address with cudaGetSymbolAddress and caches it;
+ *    make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array and leaves its last
+ *    contents behind (nothing in it needs to start at zero).  Calls whose
+ *    executions overlap on the GPU (different streams, or concurrent host
+ *    threads) race on the array and give undefined results; serialise them.
+ */
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight W,
+                                                const uint16_t* A, const uint16_t* B, int32_t r,
+                                                float s, void* Y, int32_t y_dtype, float* U_out,
+                                                int32_t* d_status, void* stream);
+
+/*
  * nf4_levels — the 16 fp32 NF4 levels the kernels use, ascending (code i ->
  * out[i]; out[7] == 0).  Host-only, needs no device.  The library derives
  * them itself from the standard-normal quantile construction of "como

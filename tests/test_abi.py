@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 11
+    assert len(names) == 12
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
