@@ -154,6 +154,50 @@ def cpu_cores():
 
 # ------------------------------------------------------------------ arms
 
+def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
+    """Forward of the 65B-shaped 8192<->22016 linears over M in {1,16,128,2048,16384}.
+
+    Per case: algorithmic bytes 0.5159 N K + 2 M K + 2 M N + 2 r (K + N) and
+    FLOPs 2 M N K + 2 M K r + 2 M N r, over the mean device time of the
+    forward call (L2 flushed before each run).
+    """
+    out = {}
+    r, s = 64, 0.25
+    for lin in synth.C5_SHAPES:
+        N, K = lin.n_out, lin.k_in
+        w = synth.weight_bf16(N, K, seed=650 + N, device=dev)
+        W = lib.quantize_weight(w)
+        del w
+        A = synth.normal_bf16((r, K), 1.0 / K, seed=651, device=dev)
+        B = synth.normal_bf16((N, r), synth.B_STD, seed=652, device=dev)
+        for M in synth.C5_M:
+            X = synth.normal_bf16((M, K), 1.0, seed=653 + M, device=dev)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            U = torch.empty((M, r), dtype=torch.float32, device=dev)
+            ws = torch.empty(max(lib.qlora_fwd_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+            for _ in range(2):
+                lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
+            ts = []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
+                e1.record()
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            ms = float(np.mean(ts))
+            byts = 0.51587 * N * K + 2 * M * K + 2 * M * N + 2 * r * (K + N)
+            fl = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
+            out[f"{lin.name}_{N}x{K}_M{M}"] = {
+                "ms": round(ms, 5), "tflops": round(fl / ms / 1e9, 2), "gbs": round(byts / ms / 1e6, 1),
+                "hbm_frac": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
+                "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+            del X, Y, U, ws
+        del W, A, B
+    return out
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -277,6 +321,11 @@ def run_ours(args, rank, world):
             kf = kernel_flops(n, M, N, K, r)
             kern[n]["tflops"] = kf / (kern[n]["ms_avg"] * 1e-3) / 1e12
 
+    if args.kernels_only:
+        if rank == 0:
+            print(json.dumps({"kernels_only": True, "ms_per_step": ms, "kernels": kern}), flush=True)
+        return
+
     # ------------------------------------------------ NF4 stream bandwidth
     # Separate launches on a weight larger than L2 (22016x8192, 65B-shaped).
     big = synth.weight_bf16(22016, 8192, seed=99, device=dev)
@@ -297,6 +346,9 @@ def run_ours(args, rank, world):
     quant_gbs = bytes_nf4 / (statistics.median(qt) * 1e-3) / 1e9
     dequant_gbs = bytes_nf4 / (statistics.median(dqt) * 1e-3) / 1e9
     del big, bcodes, bc8, bs2, bout
+
+    # ------------------------------------------- 65B-shaped forward sweep
+    c5 = c5_forward_sweep(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
 
     # ------------------------------------------------------------- e2e
     host = {k: torch.empty_like(g[k], device="cpu").pin_memory() for k in ("W", "X", "dY")}
@@ -353,6 +405,7 @@ def run_ours(args, rank, world):
             "kernels": {n: {kk: round(vv, 5) if isinstance(vv, float) else vv for kk, vv in k.items()}
                         for n, k in sorted(kern.items(), key=lambda x: -x[1]["ms_total"])},
             "nf4_quantize_gbs": quant_gbs, "nf4_dequantize_gbs": dequant_gbs,
+            "c5_forward": c5,
             "nf4_hbm_frac": {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
                              "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
         }
@@ -366,6 +419,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 65B-shaped forward sweep")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="only the timed steps (for profiler captures): no e2e, no NF4 stream test, no CPU baseline")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -101,25 +101,34 @@ EncodeTiledFn encode_fn() {
 // 2-D row-major tensor [outer, inner] of elements of `esize` bytes, row
 // stride `row_bytes`, copied in boxes of [box_outer, box_inner].
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, int swizzle_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                               : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                     : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
-  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows, true);
+// bf16 [rows, cols] row-major; the box's inner extent times 2 bytes must equal
+// the swizzle span (128 or 64 bytes).
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows,
+              int swizzle_bytes = 128) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows,
+                  swizzle_bytes);
 }
 
 bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
-  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, false);
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, 0);
 }
+
+// Token count above which the 512-token kernel runs.
+constexpr int64_t kWideM = 256;
 
 // ------------------------------------------------------------ checks
 
@@ -219,15 +228,16 @@ class ProfScope {
 // Split counts depend only on the shape (aim: about two CTAs per SM of a
 // 148-SM B200), so the workspace query is a pure host function.
 
-constexpr int kTargetCtas = 296;
+constexpr int kSms = 148;
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Number of slices for `stages` contraction steps over `tiles` output tiles,
-// with at least `min_per` steps per slice; every slice is non-empty.
-void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int& splits, int& per) {
-  int64_t s = std::max<int64_t>(1, cdiv(kTargetCtas, std::max<int64_t>(tiles, 1)));
+// Number of slices for `stages` contraction steps over `tiles` output tiles so
+// that tiles * slices fits in one wave of `ctas_per_sm` CTAs per SM, with at
+// least `min_per` steps per slice; every slice is non-empty.
+void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int ctas_per_sm, int& splits, int& per) {
+  int64_t s = std::max<int64_t>(1, (int64_t(kSms) * ctas_per_sm) / std::max<int64_t>(tiles, 1));
   s = std::min<int64_t>(s, std::max<int64_t>(1, stages / std::max<int64_t>(min_per, 1)));
   const int64_t p = cdiv(stages, s);
   per = static_cast<int>(p);
@@ -243,11 +253,23 @@ struct FwdPlan {
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   FwdPlan p{};
   const int64_t kst = K / 64;
-  split_plan(cdiv(M, 128), kst, 4, p.s_down, p.per_down);
+  split_plan(cdiv(M, 128), kst, 4, 2, p.s_down, p.per_down);
   p.bn = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
-  if (M <= 256) split_plan(tiles, kst, 8, p.s_fwd, p.per_fwd);
-  else { p.s_fwd = 1; p.per_fwd = static_cast<int>(kst); }
+  if (M <= 256) {
+    // The weight streams through once: spread it over several waves of CTAs
+    // (balanced SMs) while keeping the fp32 partials of Y under a quarter of
+    // the NF4 bytes (S * M * N * 4 <= N * K / 8).
+    int64_t s = cdiv(4 * kSms, tiles);
+    s = std::min<int64_t>(s, std::max<int64_t>(1, K / (8 * M)));
+    s = std::min<int64_t>(s, std::max<int64_t>(1, kst / 8));
+    s = std::max<int64_t>(s, 1);
+    p.per_fwd = static_cast<int>(cdiv(kst, s));
+    p.s_fwd = static_cast<int>(cdiv(kst, p.per_fwd));
+  } else {
+    p.s_fwd = 1;
+    p.per_fwd = static_cast<int>(kst);
+  }
   size_t off = align256(static_cast<size_t>(p.s_down) * M * r * 4);
   p.off_ucat = off;
   off += align256(static_cast<size_t>(M) * 2 * r * 2);
@@ -264,9 +286,9 @@ struct BwdPlan {
 
 BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   BwdPlan p{};
-  split_plan(cdiv(M, 128), N / 64, 4, p.s_du, p.per_du);
-  split_plan(cdiv(N, 128), cdiv(M, 64), 4, p.s_db, p.per_db);
-  split_plan(cdiv(K, 256), cdiv(M, 64), 4, p.s_da, p.per_da);
+  split_plan(cdiv(M, 128), N / 64, 4, 2, p.s_du, p.per_du);
+  split_plan(cdiv(N, 128), cdiv(M, 64), 4, 2, p.s_db, p.per_db);
+  split_plan(cdiv(K, 256), cdiv(M, 64), 4, 1, p.s_da, p.per_da);
   p.bn = M > 128 ? 256 : 128;
   size_t off = 0;
   p.off_sucat = off;
@@ -420,6 +442,29 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
   }
 
   // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
+  if (M > kWideM) {
+    CUtensorMap wx, wc, wu, wb;
+    if (!map_bf16(&wx, X, M, K, 32, 256, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
+        !map_bf16(&wu, ucat, M, 2 * r, 32, 256, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
+      return QLORA_ERR_CUDA;
+    FusedArgs fa{};
+    fa.c8 = W.c8;
+    fa.s2 = W.s2;
+    fa.out = Y;
+    fa.out_f32 = y_dtype == QLORA_DTYPE_F32;
+    fa.ld_out = N;
+    fa.M = static_cast<int>(M);
+    fa.rows = static_cast<int>(N);
+    fa.n_out = static_cast<int>(N);
+    fa.k_in = static_cast<int>(K);
+    fa.r = r;
+    fa.kt_total = static_cast<int>(K / 32);
+    fa.kt_per_split = fa.kt_total;
+    fa.status = d_status;
+    fa.tab = tables();
+    ProfScope ps(kKFusedFwd, cs);
+    return from_cuda(launch_fused2x(false, wx, wc, wu, wb, fa, cs));
+  }
   CUtensorMap mx, mc, mu, mb;
   if (!map_bf16(&mx, X, M, K, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 32, 128) ||
       !map_bf16(&mu, ucat, M, 2 * r, 64, p.bn) || !map_bf16(&mb, B, N, r, 64, 128))
@@ -521,6 +566,29 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   }
 
   // dX = dY W' + dU A, W' dequantised inside the GEMM.
+  if (M > kWideM) {
+    CUtensorMap wdy, wc, wdu, wal;
+    if (!map_bf16(&wdy, dY, M, N, 32, 256, 64) || !map_u8(&wc, W.codes, N, K / 2, 64, 32) ||
+        !map_bf16(&wdu, ducat, M, 2 * r, 32, 256, 64) || !map_bf16(&wal, A, r, K, 64, 16, 128))
+      return QLORA_ERR_CUDA;
+    FusedArgs fa{};
+    fa.c8 = W.c8;
+    fa.s2 = W.s2;
+    fa.out = dX;
+    fa.out_f32 = dx_dtype == QLORA_DTYPE_F32;
+    fa.ld_out = K;
+    fa.M = Mi;
+    fa.rows = Ki;
+    fa.n_out = Ni;
+    fa.k_in = Ki;
+    fa.r = r;
+    fa.kt_total = static_cast<int>(N / 32);
+    fa.kt_per_split = fa.kt_total;
+    fa.status = d_status;
+    fa.tab = tables();
+    ProfScope ps(kKFusedDX, cs);
+    if (qlora_status st = from_cuda(launch_fused2x(true, wdy, wc, wdu, wal, fa, cs))) return st;
+  } else {
   CUtensorMap mdy, mc, mdu, mal;
   if (!map_bf16(&mdy, dY, M, N, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 64, 64) ||
       !map_bf16(&mdu, ducat, M, 2 * r, 64, p.bn) || !map_bf16(&mal, A, r, K, 64, 64))
@@ -544,6 +612,7 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   {
     ProfScope ps(kKFusedDX, cs);
     if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, cs))) return st;
+  }
   }
 
   // dA = dU^T X  (split over M)

@@ -16,6 +16,8 @@
 // The LoRA up-projection is appended to the contraction as extra K steps over
 // the interleaved hi/lo bf16 split of the fp32 down-projection, accumulated in
 // the same TMEM accumulator (no second pass over Y).  No TMA multicast.
+#include <cstdlib>
+
 #include "kernels.h"
 
 namespace qnf4 {
@@ -41,8 +43,8 @@ struct FusedPlan {
   static_assert(kStages >= 3, "pipeline too shallow");
 };
 
-template <int BN, bool DX>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, bool DX, int DQW>
+__global__ void __launch_bounds__(64 + 32 * DQW, 1)
     fused_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
                  const FusedArgs a) {
@@ -69,7 +71,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&wfull[s], 128);
+      mbar_init(&wfull[s], 32 * DQW);
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -159,8 +161,11 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ dequantisers
-    const int q = warp & 3;
-    const int rl = q * 32 + lane;
+    // DQW == 4: thread dt owns tile row dt (one whole NF4 block per stage).
+    // DQW == 8: threads 2i and 2i+1 share tile row i, half a block each.
+    const int dt = threadIdx.x - 64;
+    const int rl = DQW == 4 ? dt : (dt >> 1);
+    const uint32_t half = DQW == 4 ? 0u : static_cast<uint32_t>(dt & 1);
     const int64_t kbpr = a.k_in / 64;  // NF4 blocks per W row
     auto block_of = [&](int t, int64_t& b) -> bool {
       const int kt = kt0 + t;
@@ -175,9 +180,11 @@ __global__ void __launch_bounds__(192, 1)
         return n < a.n_out && kb < kbpr;
       }
     };
-    // three-deep register prefetch of the block constants
-    uint32_t pc0 = 0, pc1 = 0, pc2 = 0;
-    float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f;
+    // six-deep register prefetch of the block constants (covers a DRAM miss
+    // when the weight streams through once, as for a handful of tokens)
+    constexpr int kPD = 6;
+    uint32_t pc[kPD];
+    float ps[kPD];
     auto fetch = [&](int t, uint32_t& c, float& sv) {
       int64_t b;
       if (t < nmain && block_of(t, b)) {
@@ -188,15 +195,17 @@ __global__ void __launch_bounds__(192, 1)
         sv = 0.f;
       }
     };
-    fetch(0, pc0, ps0);
-    fetch(1, pc1, ps1);
-    fetch(2, pc2, ps2);
+#pragma unroll
+    for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
     for (int t = 0; t < nmain; ++t) {
-      const uint32_t c8b = pc0;
-      const float s2v = ps0;
-      pc0 = pc1; ps0 = ps1;
-      pc1 = pc2; ps1 = ps2;
-      fetch(t + 3, pc2, ps2);
+      const uint32_t c8b = pc[0];
+      const float s2v = ps[0];
+#pragma unroll
+      for (int i = 0; i + 1 < kPD; ++i) {
+        pc[i] = pc[i + 1];
+        ps[i] = ps[i + 1];
+      }
+      fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
       int64_t bdummy;
       const bool valid = block_of(t, bdummy);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
@@ -215,42 +224,67 @@ __global__ void __launch_bounds__(192, 1)
         dst = st + P::kB + bs * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
         swz = nl & 7;
       }
-      if (valid) {
-        const Nf4Lut lut = nf4_make_lut(a.tab, nf4_block_scale(c8b, s2v));
-        nf4_block_to_swizzled_row(src, lut, dst, swz);
-      } else {
+      const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
+      if (DQW == 4) {
+        if (valid) {
+          nf4_block_to_swizzled_row(src, nf4_make_lut(a.tab, chat), dst, swz);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
+          for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
+        }
+      } else {
+        const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes: full-mask shuffle
+        if (valid) {
+          nf4_half_block_to_swizzled_row(src + 16 * half, lut, dst, swz, half);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(dst + (4 * half + j) * 16) = make_uint4(0, 0, 0, 0);
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&wfull[s]);
     }
 
     // ------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lane quadrant w % 4; with 8 dequant warps the two
+    // warps of a quadrant split the BN accumulator columns in halves.
     if (mbar_wait(accf, 0, wc)) {
       tc_fence_after();
-      const int orow = row0 + rl;
+      const int q = warp & 3;
+      const int erow = q * 32 + lane;
+      const int cgrp = DQW == 4 ? 0 : (warp - 2) / 4;
+      constexpr int kAll = BN / 32;                                  // 32-column chunks
+      constexpr int kChunks = DQW == 4 ? kAll : (kAll + 1) / 2;      // per column group
+      const int orow = row0 + erow;
       const bool rok = orow < a.rows;
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
+      for (int ci = 0; ci < kChunks; ++ci) {
+        const int cb = cgrp * kChunks + ci;
+        if (cb >= kAll) break;  // warp-uniform
         uint32_t v[32];
         tmem_ld_32x32b_x32(tq + cb * 32, v);
         tmem_ld_wait();
         if (rok) {
           const int mb = m0 + cb * 32;
           const int nv = min(32, a.M - mb);
+          const int64_t ld = a.ld_out;
           if (a.split_stride || a.out_f32) {
             float* o = reinterpret_cast<float*>(a.out) + static_cast<int64_t>(z) * a.split_stride + orow +
-                       static_cast<int64_t>(mb) * a.ld_out;
+                       static_cast<int64_t>(mb) * ld;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nv) o[static_cast<int64_t>(j) * a.ld_out] = __uint_as_float(v[j]);
+            for (int j = 0; j < 32; ++j) {
+              if (j < nv) *o = __uint_as_float(v[j]);
+              o += ld;
+            }
           } else {
-            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + orow + static_cast<int64_t>(mb) * a.ld_out;
+            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nv) o[static_cast<int64_t>(j) * a.ld_out] = bf16_bits(__uint_as_float(v[j]));
+            for (int j = 0; j < 32; ++j) {
+              if (j < nv) *o = bf16_bits(__uint_as_float(v[j]));
+              o += ld;
+            }
           }
         }
       }
@@ -265,30 +299,358 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int BN, bool DX>
+// ============================================================================
+// fused2x: large-M variant.  One CTA owns 128 W-side rows and 512 tokens in two
+// 128 x 256 fp32 TMEM accumulators (all 512 TMEM columns), so every
+// dequantised weight feeds 512 tokens: half the integer-pipe work per MMA
+// FLOP of the 256-token kernel.  Stages are 32 deep along the contraction
+// (64-byte swizzled token tiles) so that five stages fit in shared memory.
+//   forward: a thread owns one W row; an NF4 block spans two stages and its
+//            table is built once and reused for the second half.
+//   dX:      a stage covers 32 W rows x 128 columns = 64 blocks; a pair of
+//            adjacent lanes shares a block (table built jointly).
+// The LoRA extension adds r/16 stages, each one 16-wide j block as a hi and a
+// lo MMA.
+// ============================================================================
+
+struct Plan2x {
+  static constexpr uint32_t kBh = 256 * 64;   // 256 tokens x 32 bf16, one accumulator's operand
+  static constexpr uint32_t kB = 2 * kBh;     // 32 KB
+  static constexpr uint32_t kA = 8192;        // 128 x 32 bf16
+  static constexpr uint32_t kC = 2048;        // packed codes of the stage
+  static constexpr uint32_t kStage = kB + kA + kC;
+  static constexpr uint32_t kStages = 5;
+  static constexpr uint32_t kBarOff = kStages * kStage;
+  static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
+  static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kSmem <= 232448u, "too much shared memory");
+};
+
+template <bool DX>
+__global__ void __launch_bounds__(192, 1)
+    fused2x_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
+                   const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
+                   const FusedArgs a) {
+  using P = Plan2x;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
+  uint64_t* wfull = full + P::kStages;
+  uint64_t* empty = wfull + P::kStages;
+  uint64_t* accf = empty + P::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * 128;
+  const int m0 = blockIdx.y * 512;
+  const int nmain = a.kt_total;               // stages of 32
+  const int next = a.r / 16;                  // one per 16-wide j block
+  const int T = nmain + next;
+
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < P::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&wfull[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_uc);
+    tma_prefetch_desc(&tm_ext);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+  const WaitCtx wc{abort_flag, a.status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      const bool a2 = !DX || row0 + 64 < a.rows;  // dX ext: second 64-column half inside K
+      for (int t = 0; t < T; ++t) {
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (t >= static_cast<int>(P::kStages) && !mbar_wait(&empty[s], (u - 1) & 1, wc)) break;
+        uint8_t* st = smem + s * P::kStage;
+        if (t < nmain) {
+          mbar_arrive_expect_tx(&full[s], P::kB + P::kC);
+          tma_load_2d(st, &tm_b, &full[s], t * 32, m0);
+          tma_load_2d(st + P::kBh, &tm_b, &full[s], t * 32, m0 + 256);
+          if (!DX) tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], t * 16, row0);
+          else tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], row0 / 2, t * 32);
+        } else {
+          const int e = t - nmain;
+          if (!DX) {
+            mbar_arrive_expect_tx(&full[s], P::kB + P::kA);
+            tma_load_2d(st + P::kB, &tm_ext, &full[s], 16 * e, row0);  // B_lora [128 n x 32 j]
+          } else {
+            mbar_arrive_expect_tx(&full[s], P::kB + (a2 ? 4096u : 2048u));
+            tma_load_2d(st + P::kB, &tm_ext, &full[s], row0, 16 * e);  // A_lora [16 j x 64 k]
+            if (a2) tma_load_2d(st + P::kB + 4096, &tm_ext, &full[s], row0 + 64, 16 * e);
+          }
+          tma_load_2d(st, &tm_uc, &full[s], 32 * e, m0);
+          tma_load_2d(st + P::kBh, &tm_uc, &full[s], 32 * e, m0 + 256);
+        }
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
+        mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 256, DX ? 1 : 0, 0);
+      const uint32_t a_step = DX ? (2048u >> 4) : (32u >> 4);
+      bool aborted = false;
+      for (int t = 0; t < T; ++t) {
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
+        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) { aborted = true; break; }
+        tc_fence_after();
+        const uint32_t sb = smem_u32(smem + s * P::kStage);
+        const uint32_t sa = sb + P::kB;
+        const uint64_t b0 = sdesc_sw64(sb, 16, 512), b1 = sdesc_sw64(sb + P::kBh, 16, 512);
+        const uint64_t ad = DX ? sdesc_sw128(sa, 4096, 1024) : sdesc_sw64(sa, 16, 512);
+        if (t < nmain) {
+#pragma unroll
+          for (uint32_t kk = 0; kk < 2; ++kk) {
+            const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
+            umma_bf16(tmem_d, ad + kk * a_step, b0 + kk * 2, idesc, acc);
+            umma_bf16(tmem_d + 256, ad + kk * a_step, b1 + kk * 2, idesc, acc);
+          }
+        } else {
+#pragma unroll
+          for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
+            umma_bf16(tmem_d, ad, b0 + part * 2, idesc, 1u);
+            umma_bf16(tmem_d + 256, ad, b1 + part * 2, idesc, 1u);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+      if (aborted) mbar_wait_drain(accf, 0);
+    }
+  } else {
+    const int dt = threadIdx.x - 64;  // 0..127
+    const int64_t kbpr = a.k_in / 64;
+    if (!DX) {
+      // -------------------------------------------------- forward dequant
+      const int rl = dt;
+      const int n = row0 + rl;
+      const bool valid = n < a.n_out;
+      const int64_t rowb = static_cast<int64_t>(n) * kbpr;
+      const uint32_t swz = (rl >> 1) & 3;
+      constexpr int kPD = 4;  // blocks of prefetch (two stages each)
+      uint32_t pc[kPD];
+      float ps[kPD];
+      auto fetch = [&](int blk, uint32_t& c, float& sv) {
+        if (valid && 2 * blk < nmain) {
+          c = __ldg(a.c8 + rowb + blk);
+          sv = __ldg(a.s2 + ((rowb + blk) >> 8));
+        } else {
+          c = 0;
+          sv = 0.f;
+        }
+      };
+#pragma unroll
+      for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
+      Nf4Lut lut{};
+      for (int t = 0; t < nmain; ++t) {
+        if ((t & 1) == 0) {
+          const float chat = valid ? nf4_block_scale(pc[0], ps[0]) : 0.0f;
+#pragma unroll
+          for (int i = 0; i + 1 < kPD; ++i) {
+            pc[i] = pc[i + 1];
+            ps[i] = ps[i + 1];
+          }
+          fetch(t / 2 + kPD, pc[kPD - 1], ps[kPD - 1]);
+          lut = nf4_make_lut(a.tab, chat);
+        }
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (!mbar_wait(&full[s], u & 1, wc)) break;
+        uint8_t* st = smem + s * P::kStage;
+        uint8_t* dst = st + P::kB + rl * 64;
+        if (valid) {
+          const uint4 c = *reinterpret_cast<const uint4*>(st + P::kB + P::kA + rl * 16);
+          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(dst + ((j ^ swz) << 4)) = nf4_lookup8(cw[j], lut);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&wfull[s]);
+      }
+    } else {
+      // -------------------------------------------------- dX dequant
+      const uint32_t half = dt & 1;
+      const int p = dt >> 1;          // block of the stage: 32 rows x 2 column blocks
+      const int nl = p & 31, bs = p >> 5;
+      const int kb = row0 / 64 + bs;
+      const bool kok = kb < kbpr;
+      constexpr int kPD = 6;
+      uint32_t pc[kPD];
+      float ps[kPD];
+      auto fetch = [&](int t, uint32_t& c, float& sv) {
+        const int n = t * 32 + nl;
+        if (t < nmain && kok && n < a.n_out) {
+          const int64_t b = static_cast<int64_t>(n) * kbpr + kb;
+          c = __ldg(a.c8 + b);
+          sv = __ldg(a.s2 + (b >> 8));
+        } else {
+          c = 0;
+          sv = 0.f;
+        }
+      };
+#pragma unroll
+      for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
+      for (int t = 0; t < nmain; ++t) {
+        const uint32_t c8b = pc[0];
+        const float s2v = ps[0];
+#pragma unroll
+        for (int i = 0; i + 1 < kPD; ++i) {
+          pc[i] = pc[i + 1];
+          ps[i] = ps[i + 1];
+        }
+        fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
+        const bool valid = kok && (t * 32 + nl) < a.n_out;
+        const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
+        const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes
+        const uint32_t s = t % P::kStages, u = t / P::kStages;
+        if (!mbar_wait(&full[s], u & 1, wc)) break;
+        uint8_t* st = smem + s * P::kStage;
+        uint8_t* dst = st + P::kB + bs * 4096 + (nl >> 3) * 1024 + (nl & 7) * 128;
+        if (valid) {
+          nf4_half_block_to_swizzled_row(st + P::kB + P::kA + nl * 64 + bs * 32 + 16 * half, lut, dst, nl & 7,
+                                         half);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(dst + (4 * half + j) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&wfull[s]);
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (mbar_wait(accf, 0, wc)) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int orow = row0 + q * 32 + lane;
+      const bool rok = orow < a.rows;
+      const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int cb = 0; cb < 16; ++cb) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tq + cb * 32, v);
+        tmem_ld_wait();
+        const int mb = m0 + cb * 32;
+        const int nv = min(32, a.M - mb);
+        if (rok && nv > 0) {
+          const int64_t ld = a.ld_out;
+          if (a.out_f32) {
+            float* o = reinterpret_cast<float*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nv) *o = __uint_as_float(v[j]);
+              o += ld;
+            }
+          } else {
+            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nv) *o = bf16_bits(__uint_as_float(v[j]));
+              o += ld;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, 512);
+  }
+}
+
+template <bool DX>
+static cudaError_t launch_fused2x_impl(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
+                                       const CUtensorMap& m3, const FusedArgs& a, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fused2x_kernel<DX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Plan2x::kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((a.rows + 127) / 128, (a.M + 511) / 512, 1);
+  fused2x_kernel<DX><<<grid, 192, Plan2x::kSmem, stream>>>(m0, m1, m2, m3, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fused2x(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
+                           const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream) {
+  return dx ? launch_fused2x_impl<true>(tm_b, tm_codes, tm_uc, tm_ext, a, stream)
+            : launch_fused2x_impl<false>(tm_b, tm_codes, tm_uc, tm_ext, a, stream);
+}
+
+template <int BN, bool DX, int DQW>
 static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
                                      const CUtensorMap& m3, const FusedArgs& a, int splits, cudaStream_t stream) {
   using P = FusedPlan<BN>;
   static bool attr_set = false;  // benign race: setting the same value twice is harmless
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fused_kernel<BN, DX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(fused_kernel<BN, DX, DQW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(P::kSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 grid((a.rows + 127) / 128, (a.M + BN - 1) / BN, splits);
-  fused_kernel<BN, DX><<<grid, 192, P::kSmem, stream>>>(m0, m1, m2, m3, a);
+  fused_kernel<BN, DX, DQW><<<grid, 64 + 32 * DQW, P::kSmem, stream>>>(m0, m1, m2, m3, a);
   return cudaGetLastError();
+}
+
+// Dequantiser warps per CTA (4 or 8; QLORA_DEQUANT_WARPS=8 selects 8).  Four
+// is the default: the lookups are bound by the integer pipe's throughput, not
+// by latency, so more warps only add the duplicated table work.
+static int dequant_warps() {
+  static int w = [] {
+    const char* e = getenv("QLORA_DEQUANT_WARPS");
+    return (e && atoi(e) == 8) ? 8 : 4;
+  }();
+  return w;
+}
+
+template <int BN, bool DX>
+static cudaError_t launch_fused_dqw(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
+                                    const CUtensorMap& m3, const FusedArgs& a, int splits, cudaStream_t stream) {
+  return dequant_warps() == 4 ? launch_fused_impl<BN, DX, 4>(m0, m1, m2, m3, a, splits, stream)
+                              : launch_fused_impl<BN, DX, 8>(m0, m1, m2, m3, a, splits, stream);
 }
 
 cudaError_t launch_fused_fwd(int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_codes,
                              const CUtensorMap& tm_uc, const CUtensorMap& tm_bl, const FusedArgs& a,
                              int splits, cudaStream_t stream) {
   switch (bn) {
-    case 32: return launch_fused_impl<32, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
-    case 64: return launch_fused_impl<64, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
-    case 128: return launch_fused_impl<128, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
-    case 256: return launch_fused_impl<256, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
+    case 32: return launch_fused_dqw<32, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
+    case 64: return launch_fused_dqw<64, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
+    case 128: return launch_fused_dqw<128, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
+    case 256: return launch_fused_dqw<256, false>(tm_x, tm_codes, tm_uc, tm_bl, a, splits, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -297,8 +659,8 @@ cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap&
                             const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a,
                             cudaStream_t stream) {
   switch (bn) {
-    case 128: return launch_fused_impl<128, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
-    case 256: return launch_fused_impl<256, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
+    case 128: return launch_fused_dqw<128, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
+    case 256: return launch_fused_dqw<256, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -58,6 +58,14 @@ cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap&
                             const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a,
                             cudaStream_t stream);
 
+// Large-M forward / dX: 128 W-side rows x 512 tokens per CTA, 32-deep stages.
+//   tm_b: X or dY [M, *] box {32, 256} SW64; tm_codes: fwd [N, K/2] box {16, 128},
+//   dX [N, K/2] box {64, 32}; tm_uc: Ucat/dUcat [M, 2r] box {32, 256} SW64;
+//   tm_ext: fwd B [N, r] box {32, 128} SW64, dX A [r, K] box {64, 16} SW128.
+//   a.kt_total counts stages of 32.
+cudaError_t launch_fused2x(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
+                           const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream);
+
 // Skinny LoRA products with split contraction; see skinny.cu for the maps.
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
                           int grid_rows, int splits, cudaStream_t stream);

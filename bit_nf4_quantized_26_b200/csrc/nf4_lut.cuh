@@ -55,11 +55,11 @@ __device__ __forceinline__ Nf4Lut nf4_make_lut(const Nf4Tables& tab, float chat)
   return t;
 }
 
-// Four codes (nibbles 0..3 of c, element i in nibble i) -> four bf16 values,
-// returned as two packed pairs (element 0 in the low half of o01).
-__device__ __forceinline__ void nf4_lookup4(uint32_t c, const Nf4Lut& t, uint32_t& o01, uint32_t& o23) {
-  const uint32_t idx = c & 0x7777u;                                // entry within a half table
-  const uint32_t msk = prmt(0x0000FF00u, 0u, (c >> 3) & 0x1111u);  // 0xFF where code >= 8
+// Four codes -> four bf16 values.  `idx` holds the low three bits of each
+// code in nibbles 0..3 and `msk` is 0xFF in byte i where code i is >= 8; the
+// result is two packed pairs (element 0 in the low half of o01).
+__device__ __forceinline__ void nf4_lookup4(uint32_t idx, uint32_t msk, const Nf4Lut& t, uint32_t& o01,
+                                            uint32_t& o23) {
   const uint32_t la = prmt(t.L[0], t.L[1], idx);
   const uint32_t lb = prmt(t.L[2], t.L[3], idx);
   const uint32_t ha = prmt(t.H[0], t.H[1], idx);
@@ -70,12 +70,57 @@ __device__ __forceinline__ void nf4_lookup4(uint32_t c, const Nf4Lut& t, uint32_
   o23 = prmt(lo, hi, 0x7362u);
 }
 
-// Eight codes (one 32-bit word of packed codes) -> eight bf16 values in a uint4.
+// Eight codes (one 32-bit word of packed codes, element i in nibble i) ->
+// eight bf16 values in a uint4.  The per-nibble index and high-bit masks are
+// formed once for all eight codes.
 __device__ __forceinline__ uint4 nf4_lookup8(uint32_t w, const Nf4Lut& t) {
+  const uint32_t idx = w & 0x77777777u;
+  const uint32_t hib = (w >> 3) & 0x11111111u;
   uint4 o;
-  nf4_lookup4(w, t, o.x, o.y);
-  nf4_lookup4(w >> 16, t, o.z, o.w);
+  nf4_lookup4(idx, prmt(0x0000FF00u, 0u, hib), t, o.x, o.y);
+  nf4_lookup4(idx >> 16, prmt(0x0000FF00u, 0u, hib >> 16), t, o.z, o.w);
   return o;
+}
+
+// Two threads (adjacent lanes, `half` = lane & 1) build one block's table
+// together: each forms four of the eight bf16 pairs and the pairs are swapped
+// with a shuffle.  Every lane of the warp must call this (full-mask shuffle).
+__device__ __forceinline__ Nf4Lut nf4_make_lut_pair(const Nf4Tables& tab, float chat, uint32_t half) {
+  uint32_t mine[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = 8 * static_cast<int>(half) + 2 * j;
+    mine[j] = pack_bf16x2(__fmul_rn(tab.q[e], chat), __fmul_rn(tab.q[e + 1], chat));
+  }
+  uint32_t other[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) other[j] = __shfl_xor_sync(0xFFFFFFFFu, mine[j], 1);
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    P[j] = half ? other[j] : mine[j];
+    P[4 + j] = half ? mine[j] : other[j];
+  }
+  Nf4Lut t;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t.L[k] = prmt(P[2 * k], P[2 * k + 1], 0x6420u);
+    t.H[k] = prmt(P[2 * k], P[2 * k + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Half of a 64-element block (16 bytes of codes at `src`, elements
+// 32*half .. 32*half+31) into the 16-byte chunks 4*half .. 4*half+3 of a
+// 128-byte swizzled shared-memory row (chunk j at position j ^ swz).
+__device__ __forceinline__ void nf4_half_block_to_swizzled_row(const uint8_t* src, const Nf4Lut& t,
+                                                               uint8_t* dst_row, uint32_t swz, uint32_t half) {
+  const uint4 c = *reinterpret_cast<const uint4*>(src);
+  const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (uint32_t j = 0; j < 4; ++j) {
+    *reinterpret_cast<uint4*>(dst_row + (((4 * half + j) ^ swz) << 4)) = nf4_lookup8(cw[j], t);
+  }
 }
 
 // Dequantise one 64-element block (32 bytes of codes at `src`, 16-byte aligned)

@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
 //
 // One thread per half block: 16 bytes of codes in (a coalesced 128-bit load
 // across the warp), 64 bytes of bf16 out (four 128-bit stores).  The 16
-// dequantised values of the block are built once per thread as byte planes
-// and looked up with byte permutes (no per-element multiply).
+// dequantised values of the block are built once per thread pair as byte
+// planes and looked up with byte permutes (no per-element multiply).
 
 constexpr int kDequantThreads = 256;
 
@@ -141,9 +141,11 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const u
   const int64_t b = t >> 1;
   const int h = static_cast<int>(t & 1);
   const int64_t nblocks = (numel + 63) / 64;
-  if (b >= nblocks) return;
-  const float chat = nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8)));
-  const Nf4Lut lut = nf4_make_lut(tab, chat);
+  const bool valid = b < nblocks;
+  const float chat = valid ? nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8))) : 0.0f;
+  // The two threads of a block (adjacent lanes) build its table together.
+  const Nf4Lut lut = nf4_make_lut_pair(tab, chat, static_cast<uint32_t>(h));
+  if (!valid) return;
   const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + b * 32 + h * 16));
   uint4 o[4];
   o[0] = nf4_lookup8(cw.x, lut);

@@ -24,20 +24,24 @@ __device__ __forceinline__ void sk_wait_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Shared-memory ring per mode.  DOWN/DU/DB keep about 97 KB so two CTAs fit
+// on an SM (each still has three to four 24-32 KB stages in flight); DA's
+// 48 KB stages give one CTA per SM.
 template <int MODE>
 struct SkPlan {
   static constexpr uint32_t kA = 16384;
   static constexpr uint32_t kB = MODE == kSkDA ? 32768 : (MODE == kSkDB ? 16384 : 8192);
   static constexpr uint32_t kStage = kA + kB;
-  static constexpr uint32_t kFit = (232448u - 2048u) / kStage;
-  static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
+  static constexpr uint32_t kStages = MODE == kSkDA ? 4 : (MODE == kSkDB ? 3 : 4);
+  static constexpr uint32_t kCtasPerSm = MODE == kSkDA ? 1 : 2;
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
   static constexpr uint32_t kTmemCols = MODE == kSkDA ? 256 : (MODE == kSkDB ? 128 : 64);
+  static_assert(kSmem * kCtasPerSm <= 232448u, "ring too large for the CTAs per SM");
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     skinny_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const SkinnyArgs a) {
   using P = SkPlan<MODE>;
@@ -248,13 +252,28 @@ __device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int r, int j, f
   row[hilo_col(j) + 16] = lo;
 }
 
+// Sum of the S split partials of element i, in split order.  The loads of up
+// to eight partials are issued before the first add so their latencies
+// overlap; the additions stay in the fixed order 0, 1, ..., S-1.
+__device__ __forceinline__ float sum_partials(const float* __restrict__ P, int S, int64_t n, int64_t i) {
+  float acc = 0.f;
+  for (int z0 = 0; z0 < S; z0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = (z0 + k < S) ? __ldg(P + (z0 + k) * n + i) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (z0 + k < S) acc = __fadd_rn(acc, v[k]);
+  }
+  return acc;
+}
+
 __global__ void finish_down_kernel(const float* __restrict__ P, int S, int M, int r, float s, float* __restrict__ U,
                                    uint16_t* __restrict__ ucat) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t n = static_cast<int64_t>(M) * r;
   if (i >= n) return;
-  float acc = 0.f;
-  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  const float acc = sum_partials(P, S, n, i);
   U[i] = acc;
   store_hilo(ucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
 }
@@ -264,8 +283,7 @@ __global__ void finish_du_kernel(const float* __restrict__ P, int S, int M, int 
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t n = static_cast<int64_t>(M) * r;
   if (i >= n) return;
-  float acc = 0.f;
-  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  const float acc = sum_partials(P, S, n, i);
   store_hilo(ducat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
 }
 
@@ -280,8 +298,7 @@ __global__ void finish_sum_kernel(const float* __restrict__ P, int S, int64_t n,
                                   float* __restrict__ out) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
-  float acc = 0.f;
-  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  const float acc = sum_partials(P, S, n, i);
   out[i] = scale == 1.0f ? acc : __fmul_rn(scale, acc);
 }
 
@@ -289,8 +306,7 @@ __global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n,
                                   int out_f32) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
-  float acc = 0.f;
-  for (int z = 0; z < S; ++z) acc = __fadd_rn(acc, P[z * n + i]);
+  const float acc = sum_partials(P, S, n, i);
   if (out_f32) reinterpret_cast<float*>(out)[i] = acc;
   else reinterpret_cast<uint16_t*>(out)[i] = bf16_bits(acc);
 }
