@@ -412,6 +412,29 @@ def run_ours(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """Profiler driver: time one entry point on one shape (no JSON contract).
+
+    --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), --steps calls after 2 warm-up calls.
+    """
+    import torch
+
+    import bit_nf4_quantized_26_b200 as lib
+    import synth
+    kind, M, N, K = args.case.split(":")
+    M, N, K, r = int(M), int(N), int(K), 64
+    d = {k: v.cuda() for k, v in synth.linear_inputs(synth.Linear("case", N, K), M, r, 0).items()}
+    W = lib.quantize_weight(d["W"])
+    Y, U = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.25)
+    for _ in range(2 + args.steps):
+        if kind == "fwd":
+            lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.25, Y=Y, U=U)
+        else:
+            lib.qlora_linear_bwd(d["dY"], d["X"], U, W, d["A"], d["B"], 0.25)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,7 +445,11 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the 65B-shaped forward sweep")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (for profiler captures): no e2e, no NF4 stream test, no CPU baseline")
+    ap.add_argument("--case", default=None, help="profiler driver: fwd:M:N:K or bwd:M:N:K")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -229,6 +229,7 @@ class ProfScope {
 // 148-SM B200), so the workspace query is a pure host function.
 
 constexpr int kSms = 148;
+constexpr int64_t kMaxCluster = 8;  // portable cluster size: splits reduced in-cluster
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -239,6 +240,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int ctas_per_sm, int& splits, int& per) {
   int64_t s = std::max<int64_t>(1, (int64_t(kSms) * ctas_per_sm) / std::max<int64_t>(tiles, 1));
   s = std::min<int64_t>(s, std::max<int64_t>(1, stages / std::max<int64_t>(min_per, 1)));
+  s = std::min<int64_t>(s, kMaxCluster);
   const int64_t p = cdiv(stages, s);
   per = static_cast<int>(p);
   splits = static_cast<int>(cdiv(stages, p));
@@ -249,6 +251,7 @@ struct FwdPlan {
   int bn, s_fwd, per_fwd;
   size_t off_ucat, off_pfwd, total;
 };
+
 
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   FwdPlan p{};
@@ -270,7 +273,7 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
     p.s_fwd = 1;
     p.per_fwd = static_cast<int>(kst);
   }
-  size_t off = align256(static_cast<size_t>(p.s_down) * M * r * 4);
+  size_t off = 0;
   p.off_ucat = off;
   off += align256(static_cast<size_t>(M) * 2 * r * 2);
   p.off_pfwd = off;
@@ -281,7 +284,7 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
 
 struct BwdPlan {
   int s_du, per_du, s_db, per_db, s_da, per_da, bn;
-  size_t off_sucat, off_pdu, off_ducat, off_pdb, off_pda, total;
+  size_t off_sucat, off_ducat, total;
 };
 
 BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
@@ -293,14 +296,8 @@ BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   size_t off = 0;
   p.off_sucat = off;
   off += align256(static_cast<size_t>(M) * 2 * r * 2);
-  p.off_pdu = off;
-  off += align256(static_cast<size_t>(p.s_du) * M * r * 4);
   p.off_ducat = off;
   off += align256(static_cast<size_t>(M) * 2 * r * 2);
-  p.off_pdb = off;
-  off += align256(static_cast<size_t>(p.s_db) * N * r * 4);
-  p.off_pda = off;
-  off += align256(static_cast<size_t>(p.s_da) * r * K * 4);
   p.total = off;
   return p;
 }
@@ -413,31 +410,27 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
   if (qlora_status st = check_device()) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  float* pdown = reinterpret_cast<float*>(wsb);
   uint16_t* ucat = reinterpret_cast<uint16_t*>(wsb + p.off_ucat);
   float* pfwd = reinterpret_cast<float*>(wsb + p.off_pfwd);
 
-  // U = X A^T  (split over K, fixed-order finish), then s*U as bf16 hi/lo.
+  // U = X A^T (contraction split over a cluster), plus the bf16 hi/lo of s*U.
   CUtensorMap mx_down, ma_down;
   if (!map_bf16(&mx_down, X, M, K, 64, 128) || !map_bf16(&ma_down, A, r, K, 64, 64)) return QLORA_ERR_CUDA;
   SkinnyArgs sa{};
-  sa.partial = pdown;
   sa.M = static_cast<int>(M);
   sa.N = static_cast<int>(N);
   sa.K = static_cast<int>(K);
   sa.r = r;
   sa.stages_total = static_cast<int>(K / 64);
   sa.stages_per_split = p.per_down;
+  sa.s = s;
+  sa.out_f32 = U_out;
+  sa.out_cat = ucat;
   sa.status = d_status;
   {
     ProfScope ps(kKDown, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa, static_cast<int>(cdiv(M, 128)),
                                                   p.s_down, cs)))
-      return st;
-  }
-  {
-    ProfScope ps(kKFinishDown, cs);
-    if (qlora_status st = from_cuda(launch_finish_down(pdown, p.s_down, static_cast<int>(M), r, s, U_out, ucat, cs)))
       return st;
   }
 
@@ -515,10 +508,7 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* sucat = reinterpret_cast<uint16_t*>(wsb + p.off_sucat);
-  float* pdu = reinterpret_cast<float*>(wsb + p.off_pdu);
   uint16_t* ducat = reinterpret_cast<uint16_t*>(wsb + p.off_ducat);
-  float* pdb = reinterpret_cast<float*>(wsb + p.off_pdb);
-  float* pda = reinterpret_cast<float*>(wsb + p.off_pda);
   const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
 
   SkinnyArgs sa{};
@@ -533,36 +523,32 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
     if (qlora_status st = from_cuda(launch_prep_su(U, Mi, r, s, sucat, cs))) return st;
   }
 
-  // dU = s dY B  (split over N)
+  // dU = s dY B  (contraction over N split over a cluster) -> bf16 hi/lo
   CUtensorMap mdy128, mbl;
   if (!map_bf16(&mdy128, dY, M, N, 64, 128) || !map_bf16(&mbl, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
-  sa.partial = pdu;
   sa.stages_total = static_cast<int>(N / 64);
   sa.stages_per_split = p.per_du;
+  sa.s = s;
+  sa.out_f32 = nullptr;
+  sa.out_cat = ducat;
   {
     ProfScope ps(kKDU, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)), p.s_du, cs)))
       return st;
   }
-  {
-    ProfScope ps(kKFinishDU, cs);
-    if (qlora_status st = from_cuda(launch_finish_du(pdu, p.s_du, Mi, r, s, ducat, cs))) return st;
-  }
 
-  // dB = dY^T (sU)  (split over M)
+  // dB = dY^T (sU)  (contraction over M split over a cluster)
   CUtensorMap mdy64, msu;
   if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * r, 64, 64)) return QLORA_ERR_CUDA;
-  sa.partial = pdb;
   sa.stages_total = static_cast<int>(cdiv(M, 64));
   sa.stages_per_split = p.per_db;
+  sa.s = 1.0f;
+  sa.out_f32 = dB;
+  sa.out_cat = nullptr;
   {
     ProfScope ps(kKDB, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, cs)))
       return st;
-  }
-  {
-    ProfScope ps(kKFinishDB, cs);
-    if (qlora_status st = from_cuda(launch_finish_sum(pdb, p.s_db, N * r, 1.0f, dB, cs))) return st;
   }
 
   // dX = dY W' + dU A, W' dequantised inside the GEMM.
@@ -615,19 +601,16 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   }
   }
 
-  // dA = dU^T X  (split over M)
+  // dA = dU^T X  (contraction over M split over a cluster)
   CUtensorMap mduc, mx;
   if (!map_bf16(&mduc, ducat, M, 2 * r, 64, 64) || !map_bf16(&mx, X, M, K, 64, 64)) return QLORA_ERR_CUDA;
-  sa.partial = pda;
   sa.stages_total = static_cast<int>(cdiv(M, 64));
   sa.stages_per_split = p.per_da;
-  {
-    ProfScope ps(kKDA, cs);
-    if (qlora_status st = from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 256)), p.s_da, cs)))
-      return st;
-  }
-  ProfScope ps(kKFinishDA, cs);
-  return from_cuda(launch_finish_sum(pda, p.s_da, static_cast<int64_t>(r) * K, 1.0f, dA, cs));
+  sa.s = 1.0f;
+  sa.out_f32 = dA;
+  sa.out_cat = nullptr;
+  ProfScope ps(kKDA, cs);
+  return from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 256)), p.s_da, cs));
 }
 
 }  // extern "C"

@@ -29,13 +29,17 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
+// Ring plan.  For a handful of tokens (BN <= 64) the kernel only streams the
+// weight: two CTAs share an SM (3-4 stages each) so more dequantiser warps
+// hide the lookup latency; larger tiles run one CTA per SM with a deep ring.
 template <int BN>
 struct FusedPlan {
   static constexpr uint32_t kB = BN * 128;  // token tile, 64 bf16 per row
   static constexpr uint32_t kA = 16384;     // W-side tile 128 x 64 bf16
   static constexpr uint32_t kC = 4096;      // packed codes of the stage
   static constexpr uint32_t kStage = kB + kA + kC;
-  static constexpr uint32_t kFit = (232448u - 2048u) / kStage;
+  static constexpr uint32_t kCtasPerSm = BN <= 64 ? 2 : 1;
+  static constexpr uint32_t kFit = (233472u / kCtasPerSm - 1024u - 2048u) / kStage;
   static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
@@ -44,7 +48,7 @@ struct FusedPlan {
 };
 
 template <int BN, bool DX, int DQW>
-__global__ void __launch_bounds__(64 + 32 * DQW, 1)
+__global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     fused_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
                  const FusedArgs a) {
@@ -625,22 +629,25 @@ static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m
   return cudaGetLastError();
 }
 
-// Dequantiser warps per CTA (4 or 8; QLORA_DEQUANT_WARPS=8 selects 8).  Four
-// is the default: the lookups are bound by the integer pipe's throughput, not
-// by latency, so more warps only add the duplicated table work.
-static int dequant_warps() {
-  static int w = [] {
+// Dequantiser warps per CTA.  With 128 or more tokens per tile the MMA work
+// hides the lookups and the integer pipe's throughput is the limit, so four
+// warps (no duplicated table work) are best; with a handful of tokens the
+// kernel is a pure weight stream whose lookups must hide their own latency,
+// so eight.  QLORA_DEQUANT_WARPS=4 or 8 overrides.
+static int dequant_warps(int bn) {
+  static int forced = [] {
     const char* e = getenv("QLORA_DEQUANT_WARPS");
-    return (e && atoi(e) == 8) ? 8 : 4;
+    return e ? atoi(e) : 0;
   }();
-  return w;
+  if (forced == 4 || forced == 8) return forced;
+  return bn <= 64 ? 8 : 4;
 }
 
 template <int BN, bool DX>
 static cudaError_t launch_fused_dqw(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
                                     const CUtensorMap& m3, const FusedArgs& a, int splits, cudaStream_t stream) {
-  return dequant_warps() == 4 ? launch_fused_impl<BN, DX, 4>(m0, m1, m2, m3, a, splits, stream)
-                              : launch_fused_impl<BN, DX, 8>(m0, m1, m2, m3, a, splits, stream);
+  return dequant_warps(BN) == 4 ? launch_fused_impl<BN, DX, 4>(m0, m1, m2, m3, a, splits, stream)
+                                : launch_fused_impl<BN, DX, 8>(m0, m1, m2, m3, a, splits, stream);
 }
 
 cudaError_t launch_fused_fwd(int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_codes,

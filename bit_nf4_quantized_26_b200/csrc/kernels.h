@@ -32,10 +32,12 @@ struct FusedArgs {
 enum SkinnyMode { kSkDown = 0, kSkDU = 1, kSkDB = 2, kSkDA = 3 };
 
 struct SkinnyArgs {
-  float* partial;      // [splits][rows][cols] fp32 partial sums
   int M, N, K, r;
-  int stages_total;    // contraction stages (64 each)
-  int stages_per_split;
+  int stages_total;     // contraction stages (64 each)
+  int stages_per_split; // stages per CTA of a cluster (the cluster spans the splits)
+  float s;              // DOWN: scale of the hi/lo copy of U; DU: the LoRA scale
+  float* out_f32;       // DOWN: U [M, r]; DB: dB [N, r]; DA: dA [r, K]
+  uint16_t* out_cat;    // DOWN: hi/lo of s*U [M, 2r]; DU: hi/lo of dU [M, 2r]
   int32_t* status;
 };
 
@@ -66,16 +68,14 @@ cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap&
 cudaError_t launch_fused2x(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
                            const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream);
 
-// Skinny LoRA products with split contraction; see skinny.cu for the maps.
+// Skinny LoRA products; the contraction is split over a cluster of `splits`
+// (1..8) CTAs along y and reduced in-cluster.  See skinny.cu for the maps.
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
                           int grid_rows, int splits, cudaStream_t stream);
 
-// Elementwise finishers (fixed-order sums over split partials).
-cudaError_t launch_finish_down(const float* P, int S, int M, int r, float s, float* U, uint16_t* ucat,
-                               cudaStream_t stream);
-cudaError_t launch_finish_du(const float* P, int S, int M, int r, float s, uint16_t* ducat, cudaStream_t stream);
+// bf16 hi/lo copy of s*U for the backward's dB operand.
 cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream);
-cudaError_t launch_finish_sum(const float* P, int S, int64_t count, float scale, float* out, cudaStream_t stream);
+// Fixed-order sum of the small-M forward's split-K partials of Y.
 cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32,
                               cudaStream_t stream);
 

@@ -2,17 +2,21 @@
 // encyclopedia entry, tonho.wtf, section "a ideia": the adapters stay in 16 bit
 // and are the only parameters that receive gradients).
 //
-//   mode DOWN:  P[m, j]  = sum_k X[m,k]  A[j,k]      (U = X A^T)
-//   mode DU:    P[m, j]  = sum_n dY[m,n] B[n,j]      (dU = s dY B)
-//   mode DB:    P[n, j]  = sum_m dY[m,n] sU[m,j]     (dB = s dY^T U)
-//   mode DA:    P[j, k]  = sum_m dU[m,j] X[m,k]      (dA = dU^T X)
+//   mode DOWN:  U[m, j]  = sum_k X[m,k]  A[j,k]        -> U (fp32), bf16 hi/lo of s*U
+//   mode DU:    dU[m, j] = s * sum_n dY[m,n] B[n,j]    -> bf16 hi/lo of dU
+//   mode DB:    dB[n, j] = sum_m dY[m,n] sU[m,j]       -> dB (fp32)
+//   mode DA:    dA[j, k] = sum_m dU[m,j] X[m,k]        -> dA (fp32)
 //
-// Each is a tcgen05 GEMM with M = 128 rows and a narrow N, streaming its long
-// operand through a TMA ring; the contraction is split across blockIdx.y
-// slices and the fp32 partials are summed in a fixed order by a finisher, so
-// results are deterministic.  The fp32 operands (sU, dU) enter the tensor core
-// as a bf16 hi/lo pair in the interleaved "hi/lo per 16" column layout:
-// column c holds part (c/16)%2 (0 = hi, 1 = lo) of j = 16*(c/32) + c%16.
+// Each is a tcgen05 GEMM with M = 128 rows and a narrow N that streams its long
+// operand through a TMA ring.  The contraction is split over the S CTAs of a
+// thread-block cluster (S <= 8, along blockIdx.y): every CTA parks its fp32
+// partial tile in its own shared memory, and after a cluster barrier each CTA
+// sums a slice of the tile's rows over all S partials through distributed
+// shared memory, in rank order 0..S-1, and writes the final outputs.  The
+// result is deterministic and needs no partial buffers in global memory and
+// no extra launch.  The fp32 operands (sU, dU) enter the tensor core as a
+// bf16 hi/lo pair in the interleaved "hi/lo per 16" column layout: column c
+// holds part (c/16)%2 (0 = hi, 1 = lo) of j = 16*(c/32) + c%16.
 #include "kernels.h"
 
 namespace qnf4 {
@@ -37,8 +41,26 @@ struct SkPlan {
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
   static constexpr uint32_t kTmemCols = MODE == kSkDA ? 256 : (MODE == kSkDB ? 128 : 64);
+  // Partial tile parked in the (then idle) ring: 128 rows x r (padded to 68
+  // floats per row so the per-row float4 stores spread over the banks), or for
+  // DA r rows x 256 columns (padded to 260).
+  static constexpr int kLdRows = 68;
+  static constexpr int kLdCols = 260;
   static_assert(kSmem * kCtasPerSm <= 232448u, "ring too large for the CTAs per SM");
+  static_assert(128 * kLdRows * 4 <= kStages * kStage, "partial tile must fit in the ring");
+  static_assert(64 * kLdCols * 4 <= kStages * kStage || MODE != kSkDA, "partial tile must fit in the ring");
 };
+
+__device__ __forceinline__ int hilo_col(int j) { return 32 * (j >> 4) + (j & 15); }
+
+// v -> (bf16(v), bf16(v - bf16(v))) at the interleaved hi/lo columns of row m.
+__device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int r, int j, float v) {
+  const uint16_t hi = bf16_bits(v);
+  const uint16_t lo = bf16_bits(__fsub_rn(v, bf16_bits_to_float(hi)));
+  uint16_t* row = cat + static_cast<int64_t>(m) * 2 * r;
+  row[hilo_col(j)] = hi;
+  row[hilo_col(j) + 16] = lo;
+}
 
 template <int MODE>
 __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
@@ -144,43 +166,43 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
       if (aborted) sk_wait_drain(accf, 0);
     }
   } else {
+    // ------------------------------------------------ TMEM -> own partial tile
     const int q = warp & 3;
     const int rl = q * 32 + lane;
+    float* part = reinterpret_cast<float*>(smem);  // ring is idle once accf completes
     if (mbar_wait(accf, 0, wc)) {
       tc_fence_after();
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
       if (MODE == kSkDown || MODE == kSkDU) {
-        const int m = row0 + rl;
-        float* out = a.partial + (static_cast<int64_t>(z) * a.M + m) * a.r;
+        // rows = tokens, columns j < r
         for (int cb = 0; cb < (a.r + 31) / 32; ++cb) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
           tmem_ld_wait();
-          if (m < a.M) {
-            const int nv = min(32, a.r - cb * 32);
-            for (int j = 0; j < nv; j += 4)
-              *reinterpret_cast<float4*>(out + cb * 32 + j) =
-                  make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                              __uint_as_float(v[j + 3]));
-          }
+          float* dst = part + rl * P::kLdRows + cb * 32;
+          const int nv = min(32, a.r - cb * 32);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (j < nv)
+              *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                                __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
         }
       } else if (MODE == kSkDB) {
-        const int n = row0 + rl;
-        float* out = a.partial + (static_cast<int64_t>(z) * a.N + n) * a.r;
+        // rows = output features, columns = hi/lo pairs of j -> combined
         for (int g = 0; g < a.r / 16; ++g) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + g * 32, v);
           tmem_ld_wait();
-          if (n < a.N) {
-            for (int j = 0; j < 16; j += 4)
-              *reinterpret_cast<float4*>(out + g * 16 + j) = make_float4(
-                  __uint_as_float(v[j]) + __uint_as_float(v[j + 16]),
-                  __uint_as_float(v[j + 1]) + __uint_as_float(v[j + 17]),
-                  __uint_as_float(v[j + 2]) + __uint_as_float(v[j + 18]),
-                  __uint_as_float(v[j + 3]) + __uint_as_float(v[j + 19]));
-          }
+          float* dst = part + rl * P::kLdRows + g * 16;
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(
+                __uint_as_float(v[j]) + __uint_as_float(v[j + 16]),
+                __uint_as_float(v[j + 1]) + __uint_as_float(v[j + 17]),
+                __uint_as_float(v[j + 2]) + __uint_as_float(v[j + 18]),
+                __uint_as_float(v[j + 3]) + __uint_as_float(v[j + 19]));
         }
-      } else {  // DA: rows c = 32q + lane; hi row (lane < 16) plus lo row (lane + 16)
+      } else {  // DA: TMEM rows c = 32q + lane; hi row (lane < 16) plus lo row (lane + 16)
         const int j = 16 * q + lane;
         const bool jok = lane < 16 && j < a.r;
         for (int cb = 0; cb < 8; ++cb) {
@@ -189,21 +211,66 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
           tmem_ld_wait();
           float sum[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float lo = __shfl_down_sync(0xFFFFFFFFu, __uint_as_float(v[i]), 16);
-            sum[i] = __uint_as_float(v[i]) + lo;
-          }
-          const int k = row0 + cb * 32;
-          if (jok && k < a.K) {
-            float* out = a.partial + (static_cast<int64_t>(z) * a.r + j) * a.K + k;
-            const int nv = min(32, a.K - k);
-            for (int i = 0; i < nv; i += 4)
-              *reinterpret_cast<float4*>(out + i) = make_float4(sum[i], sum[i + 1], sum[i + 2], sum[i + 3]);
+          for (int i = 0; i < 32; ++i)
+            sum[i] = __uint_as_float(v[i]) + __shfl_down_sync(0xFFFFFFFFu, __uint_as_float(v[i]), 16);
+          if (jok) {
+            float* dst = part + j * P::kLdCols + cb * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) = make_float4(sum[i], sum[i + 1], sum[i + 2], sum[i + 3]);
           }
         }
       }
     }
   }
+
+  // -------------------------------------------- cluster-wide fixed-order sum
+  __syncwarp();
+  cluster_sync_all();
+  {
+    const float* part = reinterpret_cast<const float*>(smem);
+    const uint32_t S = gridDim.y;  // the cluster spans the split dimension
+    const uint32_t rank = cluster_ctarank();
+    const bool by_rows = (MODE != kSkDA);
+    const int R = by_rows ? 128 : a.r;                 // rows of the partial tile
+    const int C = by_rows ? a.r : 256;                 // columns
+    const int ld = by_rows ? P::kLdRows : P::kLdCols;  // floats per smem row
+    const int rows_per = (R + static_cast<int>(S) - 1) / static_cast<int>(S);
+    const int r0 = static_cast<int>(rank) * rows_per;
+    const int r1 = min(R, r0 + rows_per);
+    const int c4 = C / 4;
+    for (int e = threadIdx.x; e < (r1 - r0) * c4; e += blockDim.x) {
+      const int row = r0 + e / c4;
+      const int col = (e % c4) * 4;
+      const float* loc = part + row * ld + col;
+      float4 acc = dsmem_ld_f4(dsmem_addr(loc, 0));
+      for (uint32_t z = 1; z < S; ++z) {
+        const float4 v = dsmem_ld_f4(dsmem_addr(loc, z));
+        acc.x = __fadd_rn(acc.x, v.x);
+        acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z);
+        acc.w = __fadd_rn(acc.w, v.w);
+      }
+      const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+      if (MODE == kSkDown || MODE == kSkDU) {
+        const int m = row0 + row;
+        if (m < a.M) {
+          if (MODE == kSkDown)
+            *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(m) * a.r + col) = acc;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) store_hilo(a.out_cat, m, a.r, col + i, __fmul_rn(a.s, vals[i]));
+        }
+      } else if (MODE == kSkDB) {
+        const int n = row0 + row;
+        if (n < a.N) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(n) * a.r + col) = acc;
+      } else {
+        const int k = row0 + col;
+        if (k < a.K) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(row) * a.K + k) = acc;
+      }
+    }
+  }
+  __syncwarp();
+  cluster_sync_all();  // peers may still be reading this CTA's partial tile
 
   tc_fence_before();
   __syncthreads();
@@ -224,8 +291,20 @@ static cudaError_t launch_skinny_impl(const CUtensorMap& tmA, const CUtensorMap&
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  skinny_kernel<MODE><<<dim3(grid_rows, splits), 192, P::kSmem, stream>>>(tmA, tmB, a);
-  return cudaGetLastError();
+  if (splits < 1 || splits > 8) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_rows, splits, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = P::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, skinny_kernel<MODE>, tmA, tmB, a);
 }
 
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
@@ -240,17 +319,6 @@ cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& t
 }
 
 // ------------------------------------------------------------------ finishers
-
-__device__ __forceinline__ int hilo_col(int j) { return 32 * (j >> 4) + (j & 15); }
-
-// v -> (bf16(v), bf16(v - bf16(v))) at the interleaved hi/lo columns of row m.
-__device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int r, int j, float v) {
-  const uint16_t hi = bf16_bits(v);
-  const uint16_t lo = bf16_bits(__fsub_rn(v, bf16_bits_to_float(hi)));
-  uint16_t* row = cat + static_cast<int64_t>(m) * 2 * r;
-  row[hilo_col(j)] = hi;
-  row[hilo_col(j) + 16] = lo;
-}
 
 // Sum of the S split partials of element i, in split order.  The loads of up
 // to eight partials are issued before the first add so their latencies
@@ -268,38 +336,11 @@ __device__ __forceinline__ float sum_partials(const float* __restrict__ P, int S
   return acc;
 }
 
-__global__ void finish_down_kernel(const float* __restrict__ P, int S, int M, int r, float s, float* __restrict__ U,
-                                   uint16_t* __restrict__ ucat) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(M) * r;
-  if (i >= n) return;
-  const float acc = sum_partials(P, S, n, i);
-  U[i] = acc;
-  store_hilo(ucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
-}
-
-__global__ void finish_du_kernel(const float* __restrict__ P, int S, int M, int r, float s,
-                                 uint16_t* __restrict__ ducat) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(M) * r;
-  if (i >= n) return;
-  const float acc = sum_partials(P, S, n, i);
-  store_hilo(ducat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, acc));
-}
-
 __global__ void prep_su_kernel(const float* __restrict__ U, int M, int r, float s, uint16_t* __restrict__ sucat) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t n = static_cast<int64_t>(M) * r;
   if (i >= n) return;
   store_hilo(sucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, U[i]));
-}
-
-__global__ void finish_sum_kernel(const float* __restrict__ P, int S, int64_t n, float scale,
-                                  float* __restrict__ out) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const float acc = sum_partials(P, S, n, i);
-  out[i] = scale == 1.0f ? acc : __fmul_rn(scale, acc);
 }
 
 __global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n, void* __restrict__ out,
@@ -313,24 +354,9 @@ __global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n,
 
 static inline unsigned blocks_for(int64_t n) { return static_cast<unsigned>((n + 255) / 256); }
 
-cudaError_t launch_finish_down(const float* P, int S, int M, int r, float s, float* U, uint16_t* ucat,
-                               cudaStream_t stream) {
-  const int64_t n = static_cast<int64_t>(M) * r;
-  finish_down_kernel<<<blocks_for(n), 256, 0, stream>>>(P, S, M, r, s, U, ucat);
-  return cudaGetLastError();
-}
-cudaError_t launch_finish_du(const float* P, int S, int M, int r, float s, uint16_t* ducat, cudaStream_t stream) {
-  const int64_t n = static_cast<int64_t>(M) * r;
-  finish_du_kernel<<<blocks_for(n), 256, 0, stream>>>(P, S, M, r, s, ducat);
-  return cudaGetLastError();
-}
 cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream) {
   const int64_t n = static_cast<int64_t>(M) * r;
   prep_su_kernel<<<blocks_for(n), 256, 0, stream>>>(U, M, r, s, sucat);
-  return cudaGetLastError();
-}
-cudaError_t launch_finish_sum(const float* P, int S, int64_t count, float scale, float* out, cudaStream_t stream) {
-  finish_sum_kernel<<<blocks_for(count), 256, 0, stream>>>(P, S, count, scale, out);
   return cudaGetLastError();
 }
 cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32, cudaStream_t stream) {
