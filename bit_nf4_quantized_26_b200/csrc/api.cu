@@ -2,6 +2,7 @@
 // workspace planning, TMA descriptor creation and kernel launches.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -127,8 +128,18 @@ bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32
   return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, 0);
 }
 
-// Token count above which the 512-token kernel runs.
+// Token count above which the 512-token kernels run.
 constexpr int64_t kWideM = 256;
+
+// CTA-pair (cta_group::2) kernels for large M when the W-side extent is a
+// multiple of 256; QLORA_PAIR=0 selects the single-CTA 512-token kernel.
+bool use_pair(int64_t rows) {
+  static const bool enabled = [] {
+    const char* e = getenv("QLORA_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return enabled && rows % 256 == 0;
+}
 
 // ------------------------------------------------------------ checks
 
@@ -436,9 +447,11 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
 
   // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
   if (M > kWideM) {
+    const bool pair = use_pair(N);
+    const uint32_t tok_box = pair ? 128 : 256;
     CUtensorMap wx, wc, wu, wb;
-    if (!map_bf16(&wx, X, M, K, 32, 256, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
-        !map_bf16(&wu, ucat, M, 2 * r, 32, 256, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
+    if (!map_bf16(&wx, X, M, K, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
+        !map_bf16(&wu, ucat, M, 2 * r, 32, tok_box, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
       return QLORA_ERR_CUDA;
     FusedArgs fa{};
     fa.c8 = W.c8;
@@ -456,7 +469,8 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
     fa.status = d_status;
     fa.tab = tables();
     ProfScope ps(kKFusedFwd, cs);
-    return from_cuda(launch_fused2x(false, wx, wc, wu, wb, fa, cs));
+    return from_cuda(pair ? launch_fused_pair(false, wx, wc, wu, wb, fa, cs)
+                          : launch_fused2x(false, wx, wc, wu, wb, fa, cs));
   }
   CUtensorMap mx, mc, mu, mb;
   if (!map_bf16(&mx, X, M, K, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 32, 128) ||
@@ -553,9 +567,11 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
 
   // dX = dY W' + dU A, W' dequantised inside the GEMM.
   if (M > kWideM) {
+    const bool pair = use_pair(K);
+    const uint32_t tok_box = pair ? 128 : 256;
     CUtensorMap wdy, wc, wdu, wal;
-    if (!map_bf16(&wdy, dY, M, N, 32, 256, 64) || !map_u8(&wc, W.codes, N, K / 2, 64, 32) ||
-        !map_bf16(&wdu, ducat, M, 2 * r, 32, 256, 64) || !map_bf16(&wal, A, r, K, 64, 16, 128))
+    if (!map_bf16(&wdy, dY, M, N, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 64, 32) ||
+        !map_bf16(&wdu, ducat, M, 2 * r, 32, tok_box, 64) || !map_bf16(&wal, A, r, K, 64, 16, 128))
       return QLORA_ERR_CUDA;
     FusedArgs fa{};
     fa.c8 = W.c8;
@@ -573,7 +589,9 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
     fa.status = d_status;
     fa.tab = tables();
     ProfScope ps(kKFusedDX, cs);
-    if (qlora_status st = from_cuda(launch_fused2x(true, wdy, wc, wdu, wal, fa, cs))) return st;
+    if (qlora_status st = from_cuda(pair ? launch_fused_pair(true, wdy, wc, wdu, wal, fa, cs)
+                                         : launch_fused2x(true, wdy, wc, wdu, wal, fa, cs)))
+      return st;
   } else {
   CUtensorMap mdy, mc, mdu, mal;
   if (!map_bf16(&mdy, dY, M, N, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 64, 64) ||

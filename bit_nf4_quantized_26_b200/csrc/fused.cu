@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&wfull[s], 32 * DQW);
+      mbar_init(&wfull[s], DQW);  // one elected arrival per dequantiser warp
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       int64_t bdummy;
       const bool valid = block_of(t, bdummy);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
-      if (!mbar_wait(&full[s], u & 1, wc)) break;
+      if (!mbar_wait_all(&full[s], u & 1, wc)) break;
       uint8_t* st = smem + s * P::kStage;
       const uint8_t* src;
       uint8_t* dst;
@@ -246,14 +246,15 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
             *reinterpret_cast<uint4*>(dst + (4 * half + j) * 16) = make_uint4(0, 0, 0, 0);
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&wfull[s]);
+      fence_proxy_async_smem();  // this lane's tile writes -> async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wfull[s]);
     }
 
     // ------------------------------------------------------------ epilogue
     // Warp w reads TMEM lane quadrant w % 4; with 8 dequant warps the two
     // warps of a quadrant split the BN accumulator columns in halves.
-    if (mbar_wait(accf, 0, wc)) {
+    if (mbar_wait_warp(accf, 0, wc)) {
       tc_fence_after();
       const int q = warp & 3;
       const int erow = q * 32 + lane;
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&wfull[s], 128);
+      mbar_init(&wfull[s], 4);  // one elected arrival per dequantiser warp
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -480,7 +481,7 @@ __global__ void __launch_bounds__(192, 1)
           lut = nf4_make_lut(a.tab, chat);
         }
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) break;
+        if (!mbar_wait_all(&full[s], u & 1, wc)) break;
         uint8_t* st = smem + s * P::kStage;
         uint8_t* dst = st + P::kB + rl * 64;
         if (valid) {
@@ -493,8 +494,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&wfull[s]);
+        fence_proxy_async_smem();  // this lane's tile writes -> async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wfull[s]);
       }
     } else {
       // -------------------------------------------------- dX dequant
@@ -532,7 +534,7 @@ __global__ void __launch_bounds__(192, 1)
         const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
         const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) break;
+        if (!mbar_wait_all(&full[s], u & 1, wc)) break;
         uint8_t* st = smem + s * P::kStage;
         uint8_t* dst = st + P::kB + bs * 4096 + (nl >> 3) * 1024 + (nl & 7) * 128;
         if (valid) {
@@ -543,13 +545,14 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < 4; ++j)
             *reinterpret_cast<uint4*>(dst + (4 * half + j) * 16) = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&wfull[s]);
+        fence_proxy_async_smem();  // this lane's tile writes -> async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wfull[s]);
       }
     }
 
     // ------------------------------------------------------------ epilogue
-    if (mbar_wait(accf, 0, wc)) {
+    if (mbar_wait_warp(accf, 0, wc)) {
       tc_fence_after();
       const int q = warp & 3;
       const int orow = row0 + q * 32 + lane;

@@ -68,6 +68,13 @@ cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap&
 cudaError_t launch_fused2x(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
                            const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream);
 
+// Same products on CTA pairs (tcgen05 cta_group::2): 256 W-side rows x 512
+// tokens per cluster of two CTAs, 8-stage rings.  Needs rows % 256 == 0.
+//   tm_b / tm_uc: boxes {32, 128} SW64; other maps as for launch_fused2x.
+cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes,
+                              const CUtensorMap& tm_uc, const CUtensorMap& tm_ext, const FusedArgs& a,
+                              cudaStream_t stream);
+
 // Skinny LoRA products; the contraction is split over a cluster of `splits`
 // (1..8) CTAs along y and reduced in-cluster.  See skinny.cu for the maps.
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,

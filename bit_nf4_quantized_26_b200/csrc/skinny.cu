@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     const int q = warp & 3;
     const int rl = q * 32 + lane;
     float* part = reinterpret_cast<float*>(smem);  // ring is idle once accf completes
-    if (mbar_wait(accf, 0, wc)) {
+    if (mbar_wait_warp(accf, 0, wc)) {
       tc_fence_after();
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
       if (MODE == kSkDown || MODE == kSkDU) {

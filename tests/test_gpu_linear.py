@@ -79,6 +79,7 @@ def test_c1_full_f32_outputs():
     (1, 192, 256, 16), (16, 256, 192, 32), (63, 320, 448, 48), (65, 128, 128, 64),
     (300, 192, 320, 64), (128, 64, 64, 16), (257, 384, 576, 64), (33, 64, 1024, 32),
     (700, 320, 448, 48), (1000, 192, 576, 16), (513, 128, 128, 64), (2000, 384, 192, 32),
+    (700, 256, 512, 48), (1300, 512, 256, 16), (600, 768, 1024, 64),
 ])
 def test_ragged_shapes(M, N, K, r):
     _check_full(M, N, K, r, 16.0 / r, M + N + K, out_dtype=1)
