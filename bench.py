@@ -33,9 +33,10 @@ METRIC = "QLoRA linear fwd+bwd TFLOP/s (% bf16 peak); NF4 quant/dequant HBM GB/s
 WORKLOAD = "c2"
 WORKLOAD_NAME = "LLaMA-7B attention projection: W 4096x4096 NF4/64 + FP8/256, 4x1024 tokens, r=64, alpha=16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-# Per-launch DRAM traffic (read + write bytes) of the dominant kernels from an
-# ncu capture of the same workload; None until captured for the current code.
-NCU_TRAFFIC_BYTES = {"fused_fwd": None, "fused_dx": None}
+# Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# tensor-core kernels of this workload, from one ncu capture of the CTA-pair
+# kernels (profiles/fused_pair_c2.md); set back to None when those kernels change.
+NCU_TRAFFIC_BYTES = {"fused_fwd": 43.952896e6 + 4.615936e6, "fused_dx": 43.993600e6 + 3.332864e6}
 
 
 def flops_fwd_bwd(M, N, K, r):
