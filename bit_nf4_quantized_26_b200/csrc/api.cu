@@ -128,6 +128,18 @@ bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32
   return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, 0);
 }
 
+}  // namespace
+
+bool qnf4::pdl_enabled() {
+  static const bool enabled = [] {
+    const char* e = getenv("QLORA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return enabled;
+}
+
+namespace {
+
 // Token count above which the 512-token kernels run.
 constexpr int64_t kWideM = 256;
 
@@ -302,7 +314,7 @@ BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   BwdPlan p{};
   split_plan(cdiv(M, 128), N / 64, 4, 2, p.s_du, p.per_du);
   split_plan(cdiv(N, 128), cdiv(M, 64), 4, 2, p.s_db, p.per_db);
-  split_plan(cdiv(K, 256), cdiv(M, 64), 4, 1, p.s_da, p.per_da);
+  split_plan(cdiv(K, 128), cdiv(M, 64), 4, 2, p.s_da, p.per_da);
   p.bn = M > 128 ? 256 : 128;
   size_t off = 0;
   p.off_sucat = off;
@@ -532,12 +544,8 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   sa.r = r;
   sa.status = d_status;
 
-  {
-    ProfScope ps(kKPrepSU, cs);
-    if (qlora_status st = from_cuda(launch_prep_su(U, Mi, r, s, sucat, cs))) return st;
-  }
-
-  // dU = s dY B  (contraction over N split over a cluster) -> bf16 hi/lo
+  // dU = s dY B  (contraction over N split over a cluster) -> bf16 hi/lo,
+  // and the bf16 hi/lo of s*U for dB from the saved U.
   CUtensorMap mdy128, mbl;
   if (!map_bf16(&mdy128, dY, M, N, 64, 128) || !map_bf16(&mbl, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
   sa.stages_total = static_cast<int>(N / 64);
@@ -545,6 +553,8 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   sa.s = s;
   sa.out_f32 = nullptr;
   sa.out_cat = ducat;
+  sa.in_u = U;
+  sa.out_cat2 = sucat;
   {
     ProfScope ps(kKDU, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)), p.s_du, cs)))
@@ -559,6 +569,8 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   sa.s = 1.0f;
   sa.out_f32 = dB;
   sa.out_cat = nullptr;
+  sa.in_u = nullptr;
+  sa.out_cat2 = nullptr;
   {
     ProfScope ps(kKDB, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, cs)))
@@ -628,7 +640,7 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   sa.out_f32 = dA;
   sa.out_cat = nullptr;
   ProfScope ps(kKDA, cs);
-  return from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 256)), p.s_da, cs));
+  return from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 128)), p.s_da, cs));
 }
 
 }  // extern "C"

@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
+  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
+  grid_dependents_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -378,6 +380,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
+  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
+  grid_dependents_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -606,8 +610,7 @@ static cudaError_t launch_fused2x_impl(const CUtensorMap& m0, const CUtensorMap&
     attr_set = true;
   }
   dim3 grid((a.rows + 127) / 128, (a.M + 511) / 512, 1);
-  fused2x_kernel<DX><<<grid, 192, Plan2x::kSmem, stream>>>(m0, m1, m2, m3, a);
-  return cudaGetLastError();
+  return launch_kernel(fused2x_kernel<DX>, grid, dim3(192), Plan2x::kSmem, stream, dim3(1, 1, 1), m0, m1, m2, m3, a);
 }
 
 cudaError_t launch_fused2x(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
@@ -628,8 +631,8 @@ static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m
     attr_set = true;
   }
   dim3 grid((a.rows + 127) / 128, (a.M + BN - 1) / BN, splits);
-  fused_kernel<BN, DX, DQW><<<grid, 64 + 32 * DQW, P::kSmem, stream>>>(m0, m1, m2, m3, a);
-  return cudaGetLastError();
+  return launch_kernel(fused_kernel<BN, DX, DQW>, grid, dim3(64 + 32 * DQW), P::kSmem, stream, dim3(1, 1, 1), m0, m1,
+                       m2, m3, a);
 }
 
 // Dequantiser warps per CTA.  With 128 or more tokens per tile the MMA work

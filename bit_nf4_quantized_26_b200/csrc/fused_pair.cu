@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
+  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
+  grid_dependents_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -335,19 +337,8 @@ static cudaError_t launch_pair_impl(const CUtensorMap& m0, const CUtensorMap& m1
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * ((a.rows + 255) / 256), (a.M + 511) / 512, 1);
-  cfg.blockDim = dim3(192, 1, 1);
-  cfg.dynamicSmemBytes = PlanPair::kSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fused_pair_kernel<DX>, m0, m1, m2, m3, a);
+  return launch_kernel(fused_pair_kernel<DX>, dim3(2 * ((a.rows + 255) / 256), (a.M + 511) / 512, 1), dim3(192),
+                       PlanPair::kSmem, stream, dim3(2, 1, 1), m0, m1, m2, m3, a);
 }
 
 cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMap& tm_codes,

@@ -4,10 +4,43 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <utility>
 
 #include "nf4_lut.cuh"
 
 namespace qnf4 {
+
+// Whether launches use programmatic dependent launch (QLORA_PDL=0 disables).
+bool pdl_enabled();
+
+// cudaLaunchKernelEx with programmatic stream serialisation (when enabled)
+// and an optional thread-block cluster shape.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 dim3 cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster.x * cluster.y * cluster.z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster.x;
+    attr[n].val.clusterDim.y = cluster.y;
+    attr[n].val.clusterDim.z = cluster.z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Arguments shared by the fused dequantise-in-GEMM kernels.  The W side of the
 // product (dequantised NF4 rows: output features in the forward, input
@@ -38,6 +71,8 @@ struct SkinnyArgs {
   float s;              // DOWN: scale of the hi/lo copy of U; DU: the LoRA scale
   float* out_f32;       // DOWN: U [M, r]; DB: dB [N, r]; DA: dA [r, K]
   uint16_t* out_cat;    // DOWN: hi/lo of s*U [M, 2r]; DU: hi/lo of dU [M, 2r]
+  const float* in_u;    // DU: the saved U [M, r]
+  uint16_t* out_cat2;   // DU: hi/lo of s*U [M, 2r] (the dB operand)
   int32_t* status;
 };
 
@@ -80,8 +115,6 @@ cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMa
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
                           int grid_rows, int splits, cudaStream_t stream);
 
-// bf16 hi/lo copy of s*U for the backward's dB operand.
-cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream);
 // Fixed-order sum of the small-M forward's split-K partials of Y.
 cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32,
                               cudaStream_t stream);

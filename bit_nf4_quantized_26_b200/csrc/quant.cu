@@ -63,6 +63,8 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, sub = lane & 7;
   if (tid < 64) lut[tid] = make_float2(tab.thr[tid], __int_as_float(tab.base[tid]));
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   const int64_t nblocks = (numel + 63) / 64;
   const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * 256;
@@ -137,6 +139,8 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const u
                                                                           const float* __restrict__ s2,
                                                                           int64_t numel, uint16_t* __restrict__ out,
                                                                           Nf4Tables tab) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDequantThreads + threadIdx.x;
   const int64_t b = t >> 1;
   const int h = static_cast<int>(t & 1);
@@ -169,18 +173,16 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const u
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
                                 int32_t* status, const Nf4Tables& tab, cudaStream_t stream) {
   const int64_t ngroups = (numel + 16383) / 16384;
-  nf4_quantize_kernel<<<static_cast<unsigned>(ngroups), kQuantThreads, 0, stream>>>(w, numel, codes, c8, s2,
-                                                                                    status, tab);
-  return cudaGetLastError();
+  return launch_kernel(nf4_quantize_kernel, dim3(static_cast<unsigned>(ngroups)), dim3(kQuantThreads), 0, stream,
+                       dim3(1, 1, 1), w, numel, codes, c8, s2, status, tab);
 }
 
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
                                   uint16_t* out, const Nf4Tables& tab, cudaStream_t stream) {
   const int64_t nhalf = ((numel + 63) / 64) * 2;
   const int64_t grid = (nhalf + kDequantThreads - 1) / kDequantThreads;
-  nf4_dequantize_kernel<<<static_cast<unsigned>(grid), kDequantThreads, 0, stream>>>(codes, c8, s2, numel, out,
-                                                                                      tab);
-  return cudaGetLastError();
+  return launch_kernel(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(kDequantThreads), 0, stream,
+                       dim3(1, 1, 1), codes, c8, s2, numel, out, tab);
 }
 
 }  // namespace qnf4

@@ -3,7 +3,7 @@
 // and are the only parameters that receive gradients).
 //
 //   mode DOWN:  U[m, j]  = sum_k X[m,k]  A[j,k]        -> U (fp32), bf16 hi/lo of s*U
-//   mode DU:    dU[m, j] = s * sum_n dY[m,n] B[n,j]    -> bf16 hi/lo of dU
+//   mode DU:    dU[m, j] = s * sum_n dY[m,n] B[n,j]    -> bf16 hi/lo of dU (and of s*U)
 //   mode DB:    dB[n, j] = sum_m dY[m,n] sU[m,j]       -> dB (fp32)
 //   mode DA:    dA[j, k] = sum_m dU[m,j] X[m,k]        -> dA (fp32)
 //
@@ -28,24 +28,23 @@ __device__ __forceinline__ void sk_wait_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Shared-memory ring per mode.  DOWN/DU/DB keep about 97 KB so two CTAs fit
-// on an SM (each still has three to four 24-32 KB stages in flight); DA's
-// 48 KB stages give one CTA per SM.
+// Shared-memory ring per mode: about 97 KB, so two CTAs fit on an SM (each
+// with three or four 24-32 KB stages in flight).
 template <int MODE>
 struct SkPlan {
   static constexpr uint32_t kA = 16384;
-  static constexpr uint32_t kB = MODE == kSkDA ? 32768 : (MODE == kSkDB ? 16384 : 8192);
+  static constexpr uint32_t kB = (MODE == kSkDA || MODE == kSkDB) ? 16384 : 8192;
   static constexpr uint32_t kStage = kA + kB;
-  static constexpr uint32_t kStages = MODE == kSkDA ? 4 : (MODE == kSkDB ? 3 : 4);
-  static constexpr uint32_t kCtasPerSm = MODE == kSkDA ? 1 : 2;
+  static constexpr uint32_t kStages = (MODE == kSkDA || MODE == kSkDB) ? 3 : 4;
+  static constexpr uint32_t kCtasPerSm = 2;
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
-  static constexpr uint32_t kTmemCols = MODE == kSkDA ? 256 : (MODE == kSkDB ? 128 : 64);
+  static constexpr uint32_t kTmemCols = (MODE == kSkDA || MODE == kSkDB) ? 128 : 64;
   // Partial tile parked in the (then idle) ring: 128 rows x r (padded to 68
   // floats per row so the per-row float4 stores spread over the banks), or for
-  // DA r rows x 256 columns (padded to 260).
+  // DA r rows x 128 columns (padded to 132).
   static constexpr int kLdRows = 68;
-  static constexpr int kLdCols = 260;
+  static constexpr int kLdCols = 132;
   static_assert(kSmem * kCtasPerSm <= 232448u, "ring too large for the CTAs per SM");
   static_assert(128 * kLdRows * 4 <= kStages * kStage, "partial tile must fit in the ring");
   static_assert(64 * kLdCols * 4 <= kStages * kStage || MODE != kSkDA, "partial tile must fit in the ring");
@@ -77,8 +76,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Tile origin: DOWN/DU rows are tokens, DB rows are output features, DA's
-  // 128 rows are the hi/lo columns of dU and blockIdx.x walks K in 256s.
-  const int row0 = blockIdx.x * (MODE == kSkDA ? 256 : 128);
+  // 128 rows are the hi/lo columns of dU and blockIdx.x walks K in 128s.
+  const int row0 = blockIdx.x * 128;
   const int z = blockIdx.y;
   const int st0 = z * a.stages_per_split;
   const int T = min(a.stages_total, st0 + a.stages_per_split) - st0;
@@ -106,6 +105,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
+  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
+  grid_dependents_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
           if (nc == 128) tma_load_2d(sb + 8192, &tmB, &full[s], 64, kt * 64);
         } else {  // DA
           int nb = 0;
-          for (int i = 0; i < 4; ++i) nb += (row0 + 64 * i < a.K) ? 1 : 0;
+          for (int i = 0; i < 2; ++i) nb += (row0 + 64 * i < a.K) ? 1 : 0;
           mbar_arrive_expect_tx(&full[s], 8192u * ((nc / 64) + nb));
           tma_load_2d(sa, &tmA, &full[s], 0, kt * 64);
           if (nc == 128) tma_load_2d(sa + 8192, &tmA, &full[s], 64, kt * 64);
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     if (lane == 0) {
       const bool a_mn = (MODE == kSkDB || MODE == kSkDA);
       const bool b_mn = (MODE != kSkDown);
-      const int n = MODE == kSkDA ? 256 : (MODE == kSkDB ? nc : 64);
+      const int n = MODE == kSkDA ? 128 : (MODE == kSkDB ? nc : 64);
       const uint32_t idesc = idesc_bf16_f32(128, n, a_mn ? 1 : 0, b_mn ? 1 : 0);
       const uint32_t a_step = a_mn ? (2048u >> 4) : (32u >> 4);
       const uint32_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
       } else {  // DA: TMEM rows c = 32q + lane; hi row (lane < 16) plus lo row (lane + 16)
         const int j = 16 * q + lane;
         const bool jok = lane < 16 && j < a.r;
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
           tmem_ld_wait();
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     const uint32_t rank = cluster_ctarank();
     const bool by_rows = (MODE != kSkDA);
     const int R = by_rows ? 128 : a.r;                 // rows of the partial tile
-    const int C = by_rows ? a.r : 256;                 // columns
+    const int C = by_rows ? a.r : 128;                 // columns
     const int ld = by_rows ? P::kLdRows : P::kLdCols;  // floats per smem row
     const int rows_per = (R + static_cast<int>(S) - 1) / static_cast<int>(S);
     const int r0 = static_cast<int>(rank) * rows_per;
@@ -259,6 +260,13 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
             *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(m) * a.r + col) = acc;
 #pragma unroll
           for (int i = 0; i < 4; ++i) store_hilo(a.out_cat, m, a.r, col + i, __fmul_rn(a.s, vals[i]));
+          if (MODE == kSkDU) {
+            // The same rows of the saved U, as the bf16 hi/lo of s*U for dB.
+            const float4 uv = __ldg(reinterpret_cast<const float4*>(a.in_u + static_cast<int64_t>(m) * a.r + col));
+            const float us[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) store_hilo(a.out_cat2, m, a.r, col + i, __fmul_rn(a.s, us[i]));
+          }
         }
       } else if (MODE == kSkDB) {
         const int n = row0 + row;
@@ -292,19 +300,8 @@ static cudaError_t launch_skinny_impl(const CUtensorMap& tmA, const CUtensorMap&
     attr_set = true;
   }
   if (splits < 1 || splits > 8) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid_rows, splits, 1);
-  cfg.blockDim = dim3(192, 1, 1);
-  cfg.dynamicSmemBytes = P::kSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, skinny_kernel<MODE>, tmA, tmB, a);
+  return launch_kernel(skinny_kernel<MODE>, dim3(grid_rows, splits, 1), dim3(192), P::kSmem, stream,
+                       dim3(1, static_cast<unsigned>(splits), 1), tmA, tmB, a);
 }
 
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
@@ -336,16 +333,11 @@ __device__ __forceinline__ float sum_partials(const float* __restrict__ P, int S
   return acc;
 }
 
-__global__ void prep_su_kernel(const float* __restrict__ U, int M, int r, float s, uint16_t* __restrict__ sucat) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t n = static_cast<int64_t>(M) * r;
-  if (i >= n) return;
-  store_hilo(sucat, static_cast<int>(i / r), r, static_cast<int>(i % r), __fmul_rn(s, U[i]));
-}
-
 __global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n, void* __restrict__ out,
                                   int out_f32) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  grid_dependency_wait();
+  grid_dependents_launch();
   if (i >= n) return;
   const float acc = sum_partials(P, S, n, i);
   if (out_f32) reinterpret_cast<float*>(out)[i] = acc;
@@ -354,14 +346,9 @@ __global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n,
 
 static inline unsigned blocks_for(int64_t n) { return static_cast<unsigned>((n + 255) / 256); }
 
-cudaError_t launch_prep_su(const float* U, int M, int r, float s, uint16_t* sucat, cudaStream_t stream) {
-  const int64_t n = static_cast<int64_t>(M) * r;
-  prep_su_kernel<<<blocks_for(n), 256, 0, stream>>>(U, M, r, s, sucat);
-  return cudaGetLastError();
-}
 cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32, cudaStream_t stream) {
-  finish_out_kernel<<<blocks_for(count), 256, 0, stream>>>(P, S, count, out, out_f32);
-  return cudaGetLastError();
+  return launch_kernel(finish_out_kernel, dim3(blocks_for(count)), dim3(256), 0, stream, dim3(1, 1, 1), P, S, count,
+                       out, out_f32);
 }
 
 }  // namespace qnf4

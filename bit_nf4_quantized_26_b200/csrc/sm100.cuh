@@ -97,6 +97,19 @@ __device__ __forceinline__ bool mbar_wait_all(uint64_t* bar, uint32_t parity, co
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// ----------------------------------------- programmatic dependent launch
+//
+// Kernels are launched with programmatic stream serialisation: the next
+// kernel's CTAs may start while this one finishes.  Each kernel therefore
+// sets up (barriers, TMEM, descriptor prefetch) first, then waits for the
+// preceding grid to complete and its writes to be visible before it touches
+// global memory, and only then lets its own dependents launch.  Outside such
+// a launch both instructions return at once.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x,
