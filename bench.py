@@ -36,7 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # tensor-core kernels of this workload, from one ncu capture of the CTA-pair
 # kernels (profiles/fused_pair_c2.md); set back to None when those kernels change.
-NCU_TRAFFIC_BYTES = {"fused_fwd": 43.952896e6 + 4.615936e6, "fused_dx": 43.993600e6 + 3.332864e6}
+NCU_TRAFFIC_BYTES = {}
 
 
 def flops_fwd_bwd(M, N, K, r):
@@ -188,12 +188,21 @@ def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
                 e1.synchronize()
                 ts.append(e0.elapsed_time(e1))
             ms = float(np.mean(ts))
+            # one more call with per-kernel event brackets (not part of ms)
+            flush.zero_()
+            lib.profile_enable(True)
+            lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
+            torch.cuda.synchronize()
+            lib.profile_enable(False)
+            kern = {}
+            for name, kms in lib.profile_collect():
+                kern[name] = round(kern.get(name, 0.0) + kms, 5)
             byts = 0.51587 * N * K + 2 * M * K + 2 * M * N + 2 * r * (K + N)
             fl = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
             out[f"{lin.name}_{N}x{K}_M{M}"] = {
                 "ms": round(ms, 5), "tflops": round(fl / ms / 1e9, 2), "gbs": round(byts / ms / 1e6, 1),
                 "hbm_frac": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
-                "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+                "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "kernels_ms": kern}
             del X, Y, U, ws
         del W, A, B
     return out

@@ -124,8 +124,9 @@ bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint
                   swizzle_bytes);
 }
 
-bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows) {
-  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, 0);
+bool map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_cols, uint32_t box_rows,
+            int swizzle_bytes = 0) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, cols, rows, cols, box_cols, box_rows, swizzle_bytes);
 }
 
 }  // namespace
@@ -192,12 +193,12 @@ qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLO
 // ------------------------------------------------------------ kernel timing
 
 enum KernelId {
-  kKQuantize = 0, kKDequantize, kKDown, kKFinishDown, kKFusedFwd, kKFinishFwd, kKPrepSU, kKDU, kKFinishDU,
-  kKDB, kKFinishDB, kKFusedDX, kKDA, kKFinishDA, kKCount
+  kKQuantize = 0, kKDequantize, kKDown, kKFusedFwd, kKFinishFwd, kKLowFwd, kKLowFinish, kKDU, kKDB, kKFusedDX,
+  kKDA, kKCount
 };
 const char* const kKernelNames[kKCount] = {
-    "nf4_quantize", "nf4_dequantize", "lora_down", "finish_down", "fused_fwd", "finish_fwd", "prep_su",
-    "lora_du", "finish_du", "lora_db", "finish_db", "fused_dx", "lora_da", "finish_da"};
+    "nf4_quantize", "nf4_dequantize", "lora_down", "fused_fwd", "finish_fwd", "lowm_fwd", "lowm_finish",
+    "lora_du", "lora_db", "fused_dx", "lora_da"};
 
 struct ProfRecord {
   int id;
@@ -272,11 +273,30 @@ void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int ctas_per_sm,
 struct FwdPlan {
   int s_down, per_down;
   int bn, s_fwd, per_fwd;
+  bool low;                  // few-token path (lowm.cu)
+  int low_tiles, low_atiles, low_kc, low_ctas;
   size_t off_ucat, off_pfwd, total;
 };
 
+// Few tokens: persistent CTAs (two per SM, and at least one per row tile so
+// that no CTA's range spans more than two tiles) over (tiles + atiles) * kc
+// units.
+FwdPlan plan_fwd_low(int64_t N, int64_t K, int32_t r) {
+  FwdPlan p{};
+  p.low = true;
+  p.low_tiles = static_cast<int>(cdiv(N, kLowmRows));
+  p.low_atiles = static_cast<int>(cdiv(r, kLowmARows));
+  p.low_kc = static_cast<int>(cdiv(K / 64, 4));
+  const int64_t all_tiles = p.low_tiles + p.low_atiles;
+  const int64_t units = all_tiles * p.low_kc;
+  p.low_ctas = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(2 * kSms, all_tiles)));
+  p.off_pfwd = 0;
+  p.total = align256(static_cast<size_t>(p.low_ctas) * 2 * kLowmRows * kLowmMpad * 4);
+  return p;
+}
 
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M <= kLowmMaxM) return plan_fwd_low(N, K, r);
   FwdPlan p{};
   const int64_t kst = K / 64;
   split_plan(cdiv(M, 128), kst, 4, 2, p.s_down, p.per_down);
@@ -435,6 +455,41 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* ucat = reinterpret_cast<uint16_t*>(wsb + p.off_ucat);
   float* pfwd = reinterpret_cast<float*>(wsb + p.off_pfwd);
+
+  if (p.low) {
+    LowmArgs la{};
+    la.codes = W.codes;
+    la.c8 = W.c8;
+    la.s2 = W.s2;
+    la.X = X;
+    la.A = A;
+    la.B = B;
+    la.part = pfwd;
+    la.Y = Y;
+    la.y_f32 = y_dtype == QLORA_DTYPE_F32;
+    la.U = U_out;
+    la.s = s;
+    la.M = static_cast<int>(M);
+    la.N = static_cast<int>(N);
+    la.K = static_cast<int>(K);
+    la.r = r;
+    la.tiles = p.low_tiles;
+    la.atiles = p.low_atiles;
+    la.kc = p.low_kc;
+    la.ctas = p.low_ctas;
+    la.status = d_status;
+    la.tab = tables();
+    CUtensorMap lc, la_map, lx;
+    if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, r, K, 64, kLowmARows, 128) ||
+        !map_bf16(&lx, X, M, K, 64, M <= 8 ? 8 : 16, 128))
+      return QLORA_ERR_CUDA;
+    {
+      ProfScope ps(kKLowFwd, cs);
+      if (qlora_status st = from_cuda(launch_lowm_fwd(lc, la_map, lx, la, cs))) return st;
+    }
+    ProfScope ps(kKLowFinish, cs);
+    return from_cuda(launch_lowm_finish(la, cs));
+  }
 
   // U = X A^T (contraction split over a cluster), plus the bf16 hi/lo of s*U.
   CUtensorMap mx_down, ma_down;

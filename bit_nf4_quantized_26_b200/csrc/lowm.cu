@@ -1,0 +1,419 @@
+// lowm.cu — QLoRA linear forward for a few tokens (M <= 16):
+//   Y = X W'^T + s (X A^T) B^T,  W' = NF4-dequantised frozen weight
+// ("QLoRA" encyclopedia entry, tonho.wtf, section "como funciona": the
+// frozen weight is stored in NF4 and turned back into BFloat16 only where it
+// is used; the adapters stay 16-bit).
+//
+// At M <= 16 the product does at most 32 flops per byte of NF4 codes, so the
+// weight stream and the nibble-to-bf16 lookups bound it, not the tensor
+// pipe.  This kernel therefore keeps the dequantised weight in registers:
+// every lane turns its own codes into bf16 pairs with byte-permute lookups
+// and hands them straight to register-operand MMAs (m16n8k16, fp32
+// accumulate).  The weight never goes back to shared memory.
+//
+// Work unit: 128 rows of W (one 16-row slice per warp) x 256 input features
+// (four 64-element blocks; lane t of each quad owns block t, so each lane
+// builds one lookup table per row and block).  The contraction slots of each
+// MMA step j take, per lane, the 8 features of chunk (j ^ c_t) of that lane's
+// own block, c_t = 5t mod 8; the token fragments read X at the same features,
+// so the permutation cancels.  The lane-dependent chunk order makes every
+// shared-memory read conflict-free: the 8 lanes of each quarter warp (two
+// rows g, four blocks t) hit 8 different 16-byte bank groups.
+//
+// Rows of A (the LoRA down-projection, bf16) form ceil(r/32) more row tiles
+// of 32 rows (two warps) whose operands are copied as they are instead of
+// dequantised, so U = X A^T comes out of the same pass at little cost.
+//
+// Lane 0 of warp 0 streams each unit's codes (one 128 x 128-byte TMA box; for
+// an A tile four 32 x 64-feature boxes) and its X slice (four 64-feature
+// boxes; rows past M and features past K arrive as zeros) into a four-stage
+// shared-memory ring, two units ahead of the unit being computed.  No warp is
+// set aside for the copies, so every warp has the full register budget.
+//
+// The units (row tile major, K chunk minor) are cut into equal contiguous
+// ranges, one per persistent CTA.  A range spans at most two row tiles (the
+// CTA count is at least the tile count); the CTA writes one fp32 partial per
+// tile it touches.  The finisher adds a tile's partials in CTA order (a fixed
+// order: results are deterministic), adds s U B^T in fp32 and rounds once.
+#include "kernels.h"
+
+namespace qnf4 {
+
+namespace {
+
+constexpr int kLowmWarps = kLowmThreads / 32;
+constexpr int kLowmStages = 4;
+constexpr int kLowmAhead = 2;                     // units in flight ahead of the one computed
+constexpr uint32_t kLowmCodes = kLowmRows * 128;  // 16 KB: 128 rows x 256 codes, or 32 A rows x 256 bf16
+constexpr uint32_t kLowmABox = kLowmARows * 128;  // {64 features, 32 rows} bf16
+
+template <int NT>
+struct LowmPlan {
+  static constexpr uint32_t kXBox = 8 * NT * 128;  // {64 features, 8 NT tokens} bf16
+  static constexpr uint32_t kStage = kLowmCodes + 4 * kXBox;
+  static constexpr uint32_t kBarOff = kLowmStages * kStage;
+  static constexpr uint32_t kSmem = kBarOff + 2 * kLowmStages * 8 + 16 + 1024;
+};
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+__device__ __forceinline__ void lowm_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
+  }
+}
+
+__device__ __forceinline__ int64_t unit_start(int64_t c, int64_t units, int ctas) { return c * units / ctas; }
+
+// CTA whose range holds unit u: the largest c with floor(c * L / P) <= u.
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int ctas) {
+  return static_cast<int>(((u + 1) * ctas - 1) / units);
+}
+
+__device__ __forceinline__ int64_t lowm_units(const LowmArgs& a) {
+  return static_cast<int64_t>(a.tiles + a.atiles) * a.kc;
+}
+
+// Whether this warp has rows in `tile`: all 16 rows of its slice exist (N and
+// r are multiples of 16).  A tiles use warps 0 and 1 only.
+__device__ __forceinline__ bool warp_rows_valid(const LowmArgs& a, int tile, int warp) {
+  if (tile < a.tiles) return tile * kLowmRows + warp * 16 + 16 <= a.N;
+  return warp < 2 && (tile - a.tiles) * kLowmARows + warp * 16 + 16 <= a.r;
+}
+
+// Block constants of rows g and g + 8 of this warp's slice, block t of the
+// unit's chunk (zero where the block does not exist: the table is then 0).
+struct UnitConsts {
+  uint32_t ca, cb;
+  float sa, sb;
+};
+
+__device__ __forceinline__ void load_consts(const LowmArgs& a, int tile, int kci, int warp, int g, int t,
+                                            UnitConsts& c) {
+  const int blk = kci * 4 + t;
+  const int kb = a.K >> 6;
+  c.ca = c.cb = 0;
+  c.sa = c.sb = 0.0f;
+  if (tile >= a.tiles || blk >= kb || !warp_rows_valid(a, tile, warp)) return;
+  const int64_t ia = (static_cast<int64_t>(tile) * kLowmRows + warp * 16 + g) * kb + blk, ib = ia + 8 * kb;
+  c.ca = __ldg(a.c8 + ia);
+  c.cb = __ldg(a.c8 + ib);
+  c.sa = __ldg(a.s2 + (ia >> 8));
+  c.sb = __ldg(a.s2 + (ib >> 8));
+}
+
+// Lane 0 of warp 0: issue the copies of unit `i` of this CTA's range into
+// stage i % kLowmStages once the eight warps have released its previous use.
+template <int NT>
+__device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_a,
+                                           const CUtensorMap* tm_x, const LowmArgs& a, uint8_t* smem,
+                                           uint64_t* full, uint64_t* empty, int i, int tile, int kci,
+                                           const WaitCtx& wc) {
+  using P = LowmPlan<NT>;
+  const int s = i % kLowmStages;
+  if (i >= kLowmStages && !mbar_wait(&empty[s], ((i / kLowmStages) & 1) ^ 1, wc)) return false;
+  uint8_t* st = smem + s * P::kStage;
+  mbar_arrive_expect_tx(&full[s], kLowmCodes + 4 * P::kXBox);
+  if (tile < a.tiles) {
+    tma_load_2d(st, tm_codes, &full[s], kci * 128, tile * kLowmRows);
+  } else {
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      tma_load_2d(st + b * kLowmABox, tm_a, &full[s], kci * 256 + b * 64, (tile - a.tiles) * kLowmARows);
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) tma_load_2d(st + kLowmCodes + b * P::kXBox, tm_x, &full[s], kci * 256 + b * 64, 0);
+  return true;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kLowmThreads, 2)
+    lowm_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_x, const LowmArgs a) {
+  using P = LowmPlan<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
+  uint64_t* empty = full + kLowmStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kLowmStages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool issuer = threadIdx.x == 0;
+
+  const int64_t units = lowm_units(a);
+  const int64_t u_beg = unit_start(blockIdx.x, units, a.ctas);
+  const int count = static_cast<int>(unit_start(blockIdx.x + 1, units, a.ctas) - u_beg);
+  const int tile0 = static_cast<int>(u_beg / a.kc);
+  const int kci0 = static_cast<int>(u_beg - static_cast<int64_t>(tile0) * a.kc);
+
+  if (issuer) {
+    for (int s = 0; s < kLowmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kLowmWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_x);
+  }
+  __syncthreads();
+  const WaitCtx wc{abort_flag, a.status};
+  grid_dependency_wait();
+  grid_dependents_launch();
+  if (count <= 0) return;
+
+  // Copy issue state (lane 0 of warp 0 only).
+  int issued = 0, itile = tile0, ikci = kci0;
+  bool ok = true;
+  auto issue_next = [&]() {
+    ok = lowm_issue<NT>(&tm_codes, &tm_a, &tm_x, a, smem, full, empty, issued, itile, ikci, wc);
+    if (ok) {
+      ++issued;
+      if (++ikci == a.kc) {
+        ikci = 0;
+        ++itile;
+      }
+    }
+  };
+  if (issuer) {
+    while (ok && issued < count && issued < kLowmAhead) issue_next();
+  }
+
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t ct = (5u * static_cast<uint32_t>(t)) & 7u;
+  // Byte offsets, within a 128-byte swizzled row of phase g, of codes word
+  // (j ^ ct) of block t (XOR j << 2 for step j), and of X / A chunk (j ^ ct)
+  // (XOR j << 4 for step j).
+  const uint32_t code_off = ((static_cast<uint32_t>(2 * t) ^ static_cast<uint32_t>(g)) << 4) ^ (ct << 2);
+  const uint32_t chunk_off = (ct ^ static_cast<uint32_t>(g)) << 4;
+
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+
+  int tile = tile0, kci = kci0;
+  UnitConsts cur;
+  load_consts(a, tile, kci, warp, g, t, cur);
+  for (int i = 0; i < count; ++i) {
+    int ntile = tile, nkci = kci + 1;
+    if (nkci == a.kc) {
+      nkci = 0;
+      ++ntile;
+    }
+    const bool more = i + 1 < count;
+    if (issuer && ok && issued < count) issue_next();
+    UnitConsts nxt = {0u, 0u, 0.0f, 0.0f};
+    if (more) load_consts(a, ntile, nkci, warp, g, t, nxt);
+    const int s = i % kLowmStages;
+    if (!mbar_wait_all(&full[s], (i / kLowmStages) & 1, wc)) break;
+    const uint8_t* st = smem + s * P::kStage;
+    // X box of this lane's block; token row 8n + g has phase g.
+    const uint8_t* xs = st + kLowmCodes + t * P::kXBox + g * 128;
+    if (warp_rows_valid(a, tile, warp)) {
+      if (tile < a.tiles) {
+        const Nf4Lut la = nf4_make_lut(a.tab, nf4_block_scale(cur.ca, cur.sa));
+        const Nf4Lut lb = nf4_make_lut(a.tab, nf4_block_scale(cur.cb, cur.sb));
+        // rows warp*16 + g and + 8, both of phase g
+        const uint8_t* ra = st + (warp * 16 + g) * 128;
+        uint32_t wa[8], wb[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t o = code_off ^ (static_cast<uint32_t>(j) << 2);
+          wa[j] = lds32(ra + o);
+          wb[j] = lds32(ra + 1024 + o);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 oa = nf4_lookup8(wa[j], la);
+          const uint4 ob = nf4_lookup8(wb[j], lb);
+          const uint32_t xo = chunk_off ^ (static_cast<uint32_t>(j) << 4);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xv = lds128(xs + n * 1024 + xo);
+            mma_16816(acc[n], oa.x, ob.x, oa.y, ob.y, xv.x, xv.y);
+            mma_16816(acc[n], oa.z, ob.z, oa.w, ob.w, xv.z, xv.w);
+          }
+        }
+      } else {
+        // Rows of A (bf16, box t holds block t's 64 features of 32 rows).
+        const uint8_t* ra = st + t * kLowmABox + (warp * 16 + g) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t xo = chunk_off ^ (static_cast<uint32_t>(j) << 4);
+          const uint4 oa = lds128(ra + xo);
+          const uint4 ob = lds128(ra + 1024 + xo);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xv = lds128(xs + n * 1024 + xo);
+            mma_16816(acc[n], oa.x, ob.x, oa.y, ob.y, xv.x, xv.y);
+            mma_16816(acc[n], oa.z, ob.z, oa.w, ob.w, xv.z, xv.w);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    // Last unit of this tile in the range: write the partial, restart.
+    if (!more || ntile != tile) {
+      const int slot = tile == tile0 ? 0 : 1;
+      float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * kLowmRows + warp * 16 + g) * kLowmMpad +
+                   2 * t;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(acc[n][0], acc[n][1]);
+        *reinterpret_cast<float2*>(dst + 8 * kLowmMpad + 8 * n) = make_float2(acc[n][2], acc[n][3]);
+        acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+      }
+    }
+    cur = nxt;
+    tile = ntile;
+    kci = nkci;
+  }
+  // After a timeout, let copies still in flight land before the CTA exits
+  // (after a normal run every stage's last phase has completed already).
+  if (issuer) {
+    for (int i = max(0, issued - kLowmStages); i < issued; ++i)
+      lowm_drain(&full[i % kLowmStages], (i / kLowmStages) & 1);
+  }
+}
+
+// Finisher layout: 256 threads = 64 rows x 4 token quads; CTA b covers rows
+// [64 b, 64 b + 64) of the output (half of row tile b / 2).
+constexpr int kFinRows = 64;
+
+// Sum over the CTAs that touched `tile`, in CTA order, of the partial of
+// `row` for tokens 4 q .. 4 q + 3.  Loads are issued four contributors at a
+// time so their latencies overlap; the additions keep the CTA order.
+__device__ __forceinline__ float4 sum_tile_partials(const LowmArgs& a, int tile, int row, int q) {
+  const int64_t units = lowm_units(a);
+  const int c0 = cta_of_unit(static_cast<int64_t>(tile) * a.kc, units, a.ctas);
+  const int c1 = cta_of_unit(static_cast<int64_t>(tile + 1) * a.kc - 1, units, a.ctas);
+  float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int cb = c0; cb <= c1; cb += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = cb + j;
+      v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (c <= c1) {
+        const int first = static_cast<int>(unit_start(c, units, a.ctas) / a.kc);
+        v[j] = *reinterpret_cast<const float4*>(
+            a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * kLowmMpad + 4 * q);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (cb + j <= c1) {
+        y.x += v[j].x;
+        y.y += v[j].y;
+        y.z += v[j].z;
+        y.w += v[j].w;
+      }
+    }
+  }
+  return y;
+}
+
+// Y[m, n] = sum of the row tile's partials + s * sum_j U[m, j] B[n, j], with
+// U = the A tiles' partials summed (every CTA forms U; CTA 0 stores it).  The
+// row of B is read before the wait for the main kernel (B is not one of its
+// outputs).
+__global__ void __launch_bounds__(256) lowm_finish_kernel(const LowmArgs a) {
+  __shared__ float su[kLowmMpad][64];
+  const int tid = threadIdx.x;
+  const int rl = tid & (kFinRows - 1), q = tid >> 6;
+  const int n = blockIdx.x * kFinRows + rl;
+  const bool active = n < a.N && 4 * q < a.M;
+  uint4 bv[8];
+  const uint4* br = reinterpret_cast<const uint4*>(a.B + static_cast<int64_t>(n < a.N ? n : 0) * a.r);
+#pragma unroll
+  for (int j8 = 0; j8 < 8; ++j8) bv[j8] = j8 < a.r / 8 ? __ldg(br + j8) : make_uint4(0u, 0u, 0u, 0u);
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (active) y = sum_tile_partials(a, blockIdx.x >> 1, (blockIdx.x & 1) * kFinRows + rl, q);
+  // U: thread (j = tid & 63, quad q) sums row j of the A tiles for its tokens.
+  {
+    const int j = tid & 63;
+    if (j < a.r && 4 * q < a.M) {
+      const float4 u = sum_tile_partials(a, a.tiles + j / kLowmARows, j % kLowmARows, q);
+      const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = 4 * q + e;
+        if (m < a.M) {
+          su[m][j] = uv[e];
+          if (blockIdx.x == 0) a.U[static_cast<int64_t>(m) * a.r + j] = uv[e];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (!active) return;
+  float lo[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int j8 = 0; j8 < 8; ++j8) {
+    if (j8 < a.r / 8) {
+      const uint32_t w[4] = {bv[j8].x, bv[j8].y, bv[j8].z, bv[j8].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float b = __uint_as_float(e & 1 ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          if (4 * q + mm < a.M) lo[mm] = fmaf(su[4 * q + mm][8 * j8 + e], b, lo[mm]);
+        }
+      }
+    }
+  }
+  const float yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int mm = 0; mm < 4; ++mm) {
+    const int m = 4 * q + mm;
+    if (m < a.M) {
+      const float v = yv[mm] + a.s * lo[mm];
+      const int64_t o = static_cast<int64_t>(m) * a.N + n;
+      if (a.y_f32) reinterpret_cast<float*>(a.Y)[o] = v;
+      else reinterpret_cast<uint16_t*>(a.Y)[o] = bf16_bits(v);
+    }
+  }
+}
+
+template <int NT>
+static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
+                                    const LowmArgs& a, cudaStream_t stream) {
+  static bool attr_set = false;  // benign race: setting the same value twice is harmless
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(lowm_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(LowmPlan<NT>::kSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  return launch_kernel(lowm_fwd_kernel<NT>, dim3(a.ctas), dim3(kLowmThreads), LowmPlan<NT>::kSmem, stream,
+                       dim3(1, 1, 1), tm_codes, tm_a, tm_x, a);
+}
+
+}  // namespace
+
+cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
+                            const LowmArgs& a, cudaStream_t stream) {
+  return a.M <= 8 ? launch_lowm_impl<1>(tm_codes, tm_a, tm_x, a, stream)
+                  : launch_lowm_impl<2>(tm_codes, tm_a, tm_x, a, stream);
+}
+
+cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>((a.N + kFinRows - 1) / kFinRows);
+  return launch_kernel(lowm_finish_kernel, dim3(grid), dim3(256), 0, stream, dim3(1, 1, 1), a);
+}
+
+}  // namespace qnf4

@@ -71,14 +71,16 @@ __device__ __forceinline__ void nf4_lookup4(uint32_t idx, uint32_t msk, const Nf
 }
 
 // Eight codes (one 32-bit word of packed codes, element i in nibble i) ->
-// eight bf16 values in a uint4.  The per-nibble index and high-bit masks are
-// formed once for all eight codes.
+// eight bf16 values in a uint4.  The high-bit masks come from the byte
+// permute's sign-replicate mode: the top bit of code 2j is the top bit of
+// byte j of (w << 4), that of code 2j+1 the top bit of byte j of w, so one
+// permute of (w << 4, w) spreads four of them into byte masks.
 __device__ __forceinline__ uint4 nf4_lookup8(uint32_t w, const Nf4Lut& t) {
   const uint32_t idx = w & 0x77777777u;
-  const uint32_t hib = (w >> 3) & 0x11111111u;
+  const uint32_t ws = w << 4;
   uint4 o;
-  nf4_lookup4(idx, prmt(0x0000FF00u, 0u, hib), t, o.x, o.y);
-  nf4_lookup4(idx >> 16, prmt(0x0000FF00u, 0u, hib >> 16), t, o.z, o.w);
+  nf4_lookup4(idx, prmt(ws, w, 0xD9C8u), t, o.x, o.y);
+  nf4_lookup4(idx >> 16, prmt(ws, w, 0xFBEAu), t, o.z, o.w);
   return o;
 }
 

@@ -86,6 +86,30 @@ def test_ragged_shapes(M, N, K, r):
     _check_full(M, N, K, r, 16.0 / r, M + N + K, out_dtype=0)
 
 
+@pytest.mark.parametrize("M,N,K,r", [
+    (1, 64, 64, 16), (3, 320, 832, 48), (8, 448, 1344, 64), (9, 128, 64, 16),
+    (12, 1088, 2112, 32), (16, 960, 4160, 64), (5, 4096, 256, 16), (7, 2048, 8192, 64),
+    (11, 1024, 16384, 48), (16, 4096, 4096, 32),
+])
+def test_few_tokens(M, N, K, r):
+    """M <= 16 forward path: row tiles with a half-empty last tile (N % 128 =
+    64), K chunks with 1..3 of their 4 blocks present, 1..19 units per CTA,
+    ranges that start and end inside a tile, r = 16..64 rows of A."""
+    _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=1)
+    _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=0)
+
+
+def test_few_tokens_forward_is_deterministic():
+    lib = _lib()
+    d = {k: v.cuda() for k, v in _inputs(13, 2048, 8192, 64, 12).items()}
+    W = lib.quantize_weight(d["W"])
+    y1, u1 = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.25)
+    y2, u2 = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.25)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(u1.view(torch.int32), u2.view(torch.int32))
+
+
 def test_lora_path_alone_w_zero():
     """W = 0: Y, dX come from the adapters alone (all codes 7, constants 0)."""
     _check_full(96, 256, 384, 64, 0.25, 7, out_dtype=1, w_zero=True)
