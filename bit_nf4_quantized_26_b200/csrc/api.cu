@@ -247,6 +247,75 @@ class ProfScope {
   bool active_ = false;
 };
 
+// ------------------------------------------------------------ side stream
+//
+// The backward's dB and dA products depend on dU (and dY, X) but not on the
+// dX GEMM, so they run on a second stream of the same device while dX runs:
+// they are HBM-bound and fill the SMs that the dX GEMM's last wave of tiles
+// leaves idle.  The fork and join are event edges on the caller's stream, so
+// ordering for the caller (and stream capture) is unchanged.  QLORA_FORK=0
+// keeps everything on the caller's stream.
+
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+bool fork_enabled() {
+  static const bool enabled = [] {
+    const char* e = getenv("QLORA_FORK");
+    return !(e && e[0] == '0');
+  }();
+  return enabled;
+}
+
+// The current device's side stream, created on first use; `lk` holds the
+// lock (one fork/join sequence at a time).  nullptr: no fork.
+SideStream* side_stream(std::unique_lock<std::mutex>& lk) {
+  if (!fork_enabled()) return nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  lk = std::unique_lock<std::mutex>(g_side_mu);
+  SideStream& ss = g_side[dev];
+  if (ss.failed) return nullptr;
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      ss.failed = true;
+      return nullptr;
+    }
+  }
+  return &ss;
+}
+
+// Fork on construction (side waits for everything issued on `main` so far),
+// join on destruction (`main` waits for everything issued on the side).
+class Fork {
+ public:
+  explicit Fork(cudaStream_t main) : main_(main), side_(main) {
+    ss_ = side_stream(lk_);
+    if (ss_ && cudaEventRecord(ss_->fork, main_) == cudaSuccess &&
+        cudaStreamWaitEvent(ss_->s, ss_->fork, 0) == cudaSuccess) {
+      side_ = ss_->s;
+    } else {
+      ss_ = nullptr;
+    }
+  }
+  ~Fork() {
+    if (ss_ && cudaEventRecord(ss_->join, side_) == cudaSuccess) cudaStreamWaitEvent(main_, ss_->join, 0);
+  }
+  cudaStream_t side() const { return side_; }
+
+ private:
+  std::unique_lock<std::mutex> lk_;
+  cudaStream_t main_, side_;
+  SideStream* ss_ = nullptr;
+};
+
 // ------------------------------------------------------------ planning
 //
 // Split counts depend only on the shape (aim: about two CTAs per SM of a
@@ -616,21 +685,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
       return st;
   }
 
-  // dB = dY^T (sU)  (contraction over M split over a cluster)
-  CUtensorMap mdy64, msu;
-  if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * r, 64, 64)) return QLORA_ERR_CUDA;
-  sa.stages_total = static_cast<int>(cdiv(M, 64));
-  sa.stages_per_split = p.per_db;
-  sa.s = 1.0f;
-  sa.out_f32 = dB;
-  sa.out_cat = nullptr;
-  sa.in_u = nullptr;
-  sa.out_cat2 = nullptr;
-  {
-    ProfScope ps(kKDB, cs);
-    if (qlora_status st = from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, cs)))
-      return st;
-  }
+  // dB and dA go to the side stream (they need dU, not dX) and are issued
+  // after dX, so dX's tiles take the SMs first and dB / dA fill the ones its
+  // last wave leaves idle; the join at the end of this scope makes the
+  // caller's stream wait for them.
+  Fork fork(cs);
+  const cudaStream_t side = fork.side();
 
   // dX = dY W' + dU A, W' dequantised inside the GEMM.
   if (M > kWideM) {
@@ -686,16 +746,39 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   }
   }
 
+  // dB = dY^T (sU)  (contraction over M split over a cluster)
+  CUtensorMap mdy64, msu;
+  if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * r, 64, 64)) return QLORA_ERR_CUDA;
+  sa.stages_total = static_cast<int>(cdiv(M, 64));
+  sa.stages_per_split = p.per_db;
+  sa.s = 1.0f;
+  sa.out_f32 = dB;
+  sa.out_cat = nullptr;
+  sa.in_u = nullptr;
+  sa.out_cat2 = nullptr;
+  {
+    ProfScope ps(kKDB, side);
+    if (qlora_status st =
+            from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, side)))
+      return st;
+  }
+
   // dA = dU^T X  (contraction over M split over a cluster)
   CUtensorMap mduc, mx;
   if (!map_bf16(&mduc, ducat, M, 2 * r, 64, 64) || !map_bf16(&mx, X, M, K, 64, 64)) return QLORA_ERR_CUDA;
-  sa.stages_total = static_cast<int>(cdiv(M, 64));
-  sa.stages_per_split = p.per_da;
-  sa.s = 1.0f;
-  sa.out_f32 = dA;
-  sa.out_cat = nullptr;
-  ProfScope ps(kKDA, cs);
-  return from_cuda(launch_skinny(kSkDA, mduc, mx, sa, static_cast<int>(cdiv(K, 128)), p.s_da, cs));
+  {
+    SkinnyArgs da = sa;
+    da.stages_total = static_cast<int>(cdiv(M, 64));
+    da.stages_per_split = p.per_da;
+    da.s = 1.0f;
+    da.out_f32 = dA;
+    da.out_cat = nullptr;
+    ProfScope ps(kKDA, side);
+    if (qlora_status st = from_cuda(launch_skinny(kSkDA, mduc, mx, da, static_cast<int>(cdiv(K, 128)), p.s_da, side)))
+      return st;
+  }
+
+  return QLORA_OK;
 }
 
 }  // extern "C"

@@ -212,17 +212,20 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     }
     const bool more = i + 1 < count;
     if (issuer && ok && issued < count) issue_next();
-    UnitConsts nxt = {0u, 0u, 0.0f, 0.0f};
-    if (more) load_consts(a, ntile, nkci, warp, g, t, nxt);
     const int s = i % kLowmStages;
     if (!mbar_wait_all(&full[s], (i / kLowmStages) & 1, wc)) break;
     const uint8_t* st = smem + s * P::kStage;
     // X box of this lane's block; token row 8n + g has phase g.
     const uint8_t* xs = st + kLowmCodes + t * P::kXBox + g * 128;
+    const bool nf4_unit = tile < a.tiles && warp_rows_valid(a, tile, warp);
+    if (!nf4_unit && more) load_consts(a, ntile, nkci, warp, g, t, cur);
     if (warp_rows_valid(a, tile, warp)) {
       if (tile < a.tiles) {
         const Nf4Lut la = nf4_make_lut(a.tab, nf4_block_scale(cur.ca, cur.sa));
         const Nf4Lut lb = nf4_make_lut(a.tab, nf4_block_scale(cur.cb, cur.sb));
+        // The next unit's constants load into `cur` (dead from here on) and
+        // have a whole unit of work to arrive.
+        if (more) load_consts(a, ntile, nkci, warp, g, t, cur);
         // rows warp*16 + g and + 8, both of phase g
         const uint8_t* ra = st + (warp * 16 + g) * 128;
         uint32_t wa[8], wb[8];
@@ -275,7 +278,6 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
         acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
       }
     }
-    cur = nxt;
     tile = ntile;
     kci = nkci;
   }
