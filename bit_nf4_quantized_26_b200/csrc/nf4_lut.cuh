@@ -139,15 +139,4 @@ __device__ __forceinline__ void nf4_block_to_swizzled_row(const uint8_t* src, co
   }
 }
 
-// Nearest-level code of a normalised value through the bucket table in shared
-// memory (lut[b] = (thr, base as int bits)).  The bucket is
-// b = RNE(16 x + 16), read from the low bits of a float whose ulp is 1
-// (1.5 * 2^23 + 16 is exact in fp32; the fma rounds once).
-__device__ __forceinline__ uint32_t nf4_code_of(float x, const float2* lut) {
-  const float t = fmaf(x, 16.0f, 12582928.0f);
-  const uint32_t b = __float_as_uint(t) & 63u;
-  const float2 e = lut[b];
-  return static_cast<uint32_t>(__float_as_int(e.y)) + (x > e.x ? 1u : 0u);
-}
-
 }  // namespace qnf4

@@ -12,10 +12,15 @@ namespace qnf4 {
 // elements = 32 KB of bf16 input.  Eight threads share a block (8 elements,
 // 16 bytes each), so a warp reads 512 contiguous bytes per pass and writes
 // 128 contiguous bytes of codes; 8 passes cover the group.  All 8 loads of a
-// thread are issued before any arithmetic.  The block absmax is a max over
-// the bf16 magnitude bits (non-negative floats order like unsigned ints)
-// reduced across the 8 lanes with shuffles; the code search uses a bucket
-// table in shared memory (one fma, one load, one compare per element).
+// thread are issued before any arithmetic; five CTAs per SM keep 160 KB of
+// loads in flight.  The block absmax is a max over the bf16 magnitude bits
+// (non-negative floats order like unsigned ints) reduced across the 8 lanes
+// with shuffles.  Per pair of elements the scaling and the bucket fma are one
+// packed two-lane fp32 instruction each; the bucket table is split into
+// float thresholds and byte bases in shared memory (bank conflicts only
+// between buckets 0 and 32); codes are packed with integer multiply-adds on
+// the FMA pipe.  The kernel is issue-bound: 19-21 instructions per element,
+// ~3.5 of 4 per cycle per SM.
 
 constexpr int kQuantThreads = 256;
 
@@ -26,12 +31,43 @@ __device__ __forceinline__ uint32_t max_abs_bits(uint4 v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
-__device__ __forceinline__ uint32_t code_pair(uint32_t word, float rc, const float2* lut, uint32_t shift) {
-  const float a = __uint_as_float(word << 16);
-  const float b = __uint_as_float(word & 0xFFFF0000u);
-  const uint32_t ca = nf4_code_of(__fmul_rn(a, rc), lut);
-  const uint32_t cb = nf4_code_of(__fmul_rn(b, rc), lut);
-  return (ca | (cb << 4)) << shift;
+// Nearest-level code of x: bucket b = RNE(16 x + 16) is the low 6 bits of t
+// (t = fma(x, 16, 1.5 * 2^23 + 16), exact offset, one rounding), then
+// base[b] + (x > thr[b]).
+__device__ __forceinline__ uint32_t quant_code(float x, float t, const float* thr, const uint8_t* base) {
+  const uint32_t b = __float_as_uint(t) & 63u;
+  return static_cast<uint32_t>(base[b]) + (x > thr[b] ? 1u : 0u);
+}
+
+// x = RN32(e * rc) and t = RN32(16 x + C) for both elements of a bf16 pair,
+// with packed two-lane fp32 instructions (each lane rounds as the scalar op).
+__device__ __forceinline__ void scale_pair(uint32_t word, uint64_t rc2, float& x0, float& x1, float& t0,
+                                           float& t1) {
+  uint64_t e2, x2, t2;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(e2) : "r"(word << 16), "r"(word & 0xFFFF0000u));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(x2) : "l"(e2), "l"(rc2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(t2)
+      : "l"(x2), "l"(0x4180000041800000ull), "l"(0x4B4000104B400010ull));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(x2));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t2));
+}
+
+// Packed codes of the 8 elements of v (element i in nibble i); the nibbles
+// are placed with integer multiply-adds, which run on the FMA pipe.
+__device__ __forceinline__ uint32_t codes8(uint4 v, float rc, const float* thr, const uint8_t* base) {
+  uint64_t rc2;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float x0, x1, t0, t1;
+    scale_pair(w[i], rc2, x0, x1, t0, t1);
+    out = quant_code(x0, t0, thr, base) * (1u << (8 * i)) + out;
+    out = quant_code(x1, t1, thr, base) * (1u << (8 * i + 4)) + out;  // disjoint nibbles: + == |
+  }
+  return out;
 }
 
 // Codes of 8 elements where 1/c is not finite (c = 0, or c so small that the
@@ -51,18 +87,22 @@ __device__ __forceinline__ uint32_t codes_degenerate(uint4 v) {
   return out;
 }
 
-__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint16_t* __restrict__ w,
-                                                                      int64_t numel, uint8_t* __restrict__ codes,
-                                                                      uint8_t* __restrict__ c8,
-                                                                      float* __restrict__ s2, int32_t* status,
-                                                                      Nf4Tables tab) {
-  __shared__ float2 lut[64];
+__global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const uint16_t* __restrict__ w,
+                                                                         int64_t numel, uint8_t* __restrict__ codes,
+                                                                         uint8_t* __restrict__ c8,
+                                                                         float* __restrict__ s2, int32_t* status,
+                                                                         Nf4Tables tab) {
+  __shared__ float thr[64];
+  __shared__ uint8_t base[64];
   __shared__ uint32_t cblk[256];
   __shared__ uint32_t wmax[kQuantThreads / 32];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, sub = lane & 7;
-  if (tid < 64) lut[tid] = make_float2(tab.thr[tid], __int_as_float(tab.base[tid]));
+  if (tid < 64) {
+    thr[tid] = tab.thr[tid];
+    base[tid] = static_cast<uint8_t>(tab.base[tid]);
+  }
   grid_dependency_wait();
   grid_dependents_launch();
 
@@ -99,8 +139,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const uint1
     const float rc = __frcp_rn(c);
     uint32_t out;
     if (rc < __int_as_float(0x7F800000)) {
-      out = code_pair(v[p].x, rc, lut, 0) | code_pair(v[p].y, rc, lut, 8) | code_pair(v[p].z, rc, lut, 16) |
-            code_pair(v[p].w, rc, lut, 24);
+      out = codes8(v[p], rc, thr, base);
     } else {
       out = codes_degenerate(v[p]);
     }
