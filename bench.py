@@ -35,8 +35,8 @@ WORKLOAD_NAME = "LLaMA-7B attention projection: W 4096x4096 NF4/64 + FP8/256, 4x
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # tensor-core kernels of this workload, from one ncu capture of the CTA-pair
-# kernels (profiles/fused_pair_c2.md); set back to None when those kernels change.
-NCU_TRAFFIC_BYTES = {}
+# kernels (profiles/fused_pair_c2.md); emptied whenever those kernels change.
+NCU_TRAFFIC_BYTES = {"fused_fwd": 43.863552e6 + 3.565568e6, "fused_dx": 43.956992e6 + 3.669504e6}
 
 
 def flops_fwd_bwd(M, N, K, r):
@@ -441,12 +441,22 @@ def run_ours(args, rank, world):
 def run_case(args):
     """Profiler driver: time one entry point on one shape (no JSON contract).
 
-    --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), --steps calls after 2 warm-up calls.
+    --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), or quant:N:K (NF4 quantisation of
+    an N x K weight), --steps calls after 2 warm-up calls.
     """
     import torch
 
     import bit_nf4_quantized_26_b200 as lib
     import synth
+    if args.case.startswith("quant:"):
+        _, N, K = args.case.split(":")
+        w = synth.weight_bf16(int(N), int(K), seed=1, device="cuda")
+        W = lib.quantize_weight(w)
+        for _ in range(2 + args.steps):
+            lib.nf4_quantize(w.view(-1), W.codes, W.c8, W.s2)
+        torch.cuda.synchronize()
+        print(json.dumps({"case": args.case, "ok": True}))
+        return
     kind, M, N, K = args.case.split(":")
     M, N, K, r = int(M), int(N), int(K), 64
     d = {k: v.cuda() for k, v in synth.linear_inputs(synth.Linear("case", N, K), M, r, 0).items()}
@@ -471,7 +481,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the 65B-shaped forward sweep")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (for profiler captures): no e2e, no NF4 stream test, no CPU baseline")
-    ap.add_argument("--case", default=None, help="profiler driver: fwd:M:N:K or bwd:M:N:K")
+    ap.add_argument("--case", default=None, help="profiler driver: fwd:M:N:K, bwd:M:N:K or quant:N:K")
     args = ap.parse_args()
     if args.case:
         run_case(args)

@@ -97,11 +97,16 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
-  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
-  grid_dependents_launch();
+  // Programmatic dependent launch: of this kernel's inputs, only the hi/lo
+  // of sU / dU (read by the extension stages) comes from the kernel launched
+  // just before it; the rest comes from earlier kernels, complete when that
+  // kernel let this one launch.  The producer waits just before the first
+  // extension load; every other role passes the wait after its main loop,
+  // before triggering the next kernel.
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    bool waited = false;
     if (lane == 0) {
       int issued = 0;
       for (int t = 0; t < T; ++t) {
@@ -115,6 +120,11 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
           if (!DX) tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], kt * 32, row0);
           else tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], row0 / 2, kt * 64);
         } else {
+          if (!waited) {
+            grid_dependency_wait();  // sU / dU of the preceding kernel are complete and visible
+            grid_dependents_launch();
+            waited = true;
+          }
           const int e = t - nmain;
           if (!DX) {
             mbar_arrive_expect_tx(&full[s], P::kB + 16384);
@@ -133,6 +143,10 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       // Do not leave the CTA while a copy into its shared memory is in flight.
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
         mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+    }
+    if (!waited) {  // lanes 1..31, a split without extension stages, or a producer that gave up
+      grid_dependency_wait();
+      grid_dependents_launch();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -165,6 +179,8 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       umma_commit(accf);
       if (aborted) mbar_wait_drain(accf, 0);
     }
+    grid_dependency_wait();
+    grid_dependents_launch();
   } else {
     // ------------------------------------------------------------ dequantisers
     // DQW == 4: thread dt owns tile row dt (one whole NF4 block per stage).
@@ -252,6 +268,9 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       __syncwarp();
       if (lane == 0) mbar_arrive(&wfull[s]);
     }
+
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     // ------------------------------------------------------------ epilogue
     // Warp w reads TMEM lane quadrant w % 4; with 8 dequant warps the two
@@ -380,10 +399,15 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
-  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
-  grid_dependents_launch();
+  // Programmatic dependent launch: of this kernel's inputs, only the hi/lo
+  // of sU / dU (read by the extension stages) comes from the kernel launched
+  // just before it; the rest comes from earlier kernels, complete when that
+  // kernel let this one launch.  The producer waits just before the first
+  // extension load; every other role passes the wait after its main loop,
+  // before triggering the next kernel.
 
   if (warp == 0) {
+    bool waited = false;
     if (lane == 0) {
       int issued = 0;
       const bool a2 = !DX || row0 + 64 < a.rows;  // dX ext: second 64-column half inside K
@@ -398,6 +422,11 @@ __global__ void __launch_bounds__(192, 1)
           if (!DX) tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], t * 16, row0);
           else tma_load_2d(st + P::kB + P::kA, &tm_codes, &full[s], row0 / 2, t * 32);
         } else {
+          if (!waited) {
+            grid_dependency_wait();  // sU / dU of the preceding kernel are complete and visible
+            grid_dependents_launch();
+            waited = true;
+          }
           const int e = t - nmain;
           if (!DX) {
             mbar_arrive_expect_tx(&full[s], P::kB + P::kA);
@@ -414,6 +443,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
         mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+    }
+    if (!waited) {  // lanes 1..31, or a producer that gave up
+      grid_dependency_wait();
+      grid_dependents_launch();
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -448,6 +481,8 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(accf);
       if (aborted) mbar_wait_drain(accf, 0);
     }
+    grid_dependency_wait();
+    grid_dependents_launch();
   } else {
     const int dt = threadIdx.x - 64;  // 0..127
     const int64_t kbpr = a.k_in / 64;
@@ -554,6 +589,9 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&wfull[s]);
       }
     }
+
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     // ------------------------------------------------------------ epilogue
     if (mbar_wait_warp(accf, 0, wc)) {

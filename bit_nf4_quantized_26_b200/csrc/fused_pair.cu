@@ -99,11 +99,18 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status};
-  grid_dependency_wait();  // inputs of earlier kernels are complete and visible
-  grid_dependents_launch();
+  // Programmatic dependent launch: the only input produced by the kernel
+  // launched just before this one is the bf16 hi/lo of sU / dU, read by the
+  // extension stages at the end of the contraction; X or dY, the codes and
+  // the block constants come from earlier kernels, which had completed when
+  // that kernel let this one launch (every kernel here waits before it
+  // triggers).  So the producer waits for the preceding grid just before the
+  // first extension load, and every other role passes the wait (a no-op by
+  // then) after its main loop, before triggering the next kernel.
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    bool waited = false;
     if (lane == 0) {
       int issued = 0;
       // Extension bytes of one CTA: token/U halves plus the LoRA tile.
@@ -121,6 +128,11 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_2d_pair(st, &tm_b, full0, t * 32, mt);
           tma_load_2d_pair(st + P::kBq, &tm_b, full0, t * 32, mt + 256);
         } else {
+          if (t == nmain) {
+            grid_dependency_wait();  // sU / dU of the preceding kernel are complete and visible
+            grid_dependents_launch();
+            waited = true;
+          }
           const int e = t - nmain;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (P::kB + ext_a));
           tma_load_2d_pair(st, &tm_uc, full0, 32 * e, mt);
@@ -140,6 +152,10 @@ __global__ void __launch_bounds__(192, 1)
         if (t < nmain) wait_drain(&cfull[t % P::kStages], (t / P::kStages) & 1);
         if (rank == 0) wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
       }
+    }
+    if (!waited) {  // lanes 1..31, or a producer that gave up early
+      grid_dependency_wait();
+      grid_dependents_launch();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA (leader)
@@ -175,6 +191,8 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit_pair(accf, 0x3);
       if (aborted) wait_drain(accf, 0);
     }
+    grid_dependency_wait();
+    grid_dependents_launch();
   } else {
     const int dt = threadIdx.x - 64;  // 0..127
     const int64_t kbpr = a.k_in / 64;
@@ -281,6 +299,9 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive_remote(dsmem_addr(&wfull[s], 0));
       }
     }
+
+    grid_dependency_wait();
+    grid_dependents_launch();
 
     // ------------------------------------------------------------ epilogue
     if (mbar_wait_warp(accf, 0, wc)) {
