@@ -499,9 +499,14 @@ qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float
   if (numel == 0) return QLORA_OK;
   if (!w_bf16 || !codes || !c8 || !s2) return QLORA_ERR_NULL;
   if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(c8) || !aligned16(s2)) return QLORA_ERR_ALIGN;
+  if (numel >= (int64_t(1) << 37)) return QLORA_ERR_SHAPE;  // the output tensor map holds < 2^31 rows of 64
   if (qlora_status st = check_device()) return st;
+  const int64_t nfull = numel / 64;
+  CUtensorMap tm_out;
+  if (nfull > 0 && !map_bf16(&tm_out, w_bf16, nfull, 64, 64, 32, 128)) return QLORA_ERR_CUDA;
   ProfScope ps(kKDequantize, static_cast<cudaStream_t>(stream));
-  return from_cuda(launch_nf4_dequantize(codes, c8, s2, numel, w_bf16, tables(), static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_nf4_dequantize(codes, c8, s2, numel, w_bf16, nfull > 0 ? &tm_out : nullptr, tables(),
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,

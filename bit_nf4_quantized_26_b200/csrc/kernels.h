@@ -78,8 +78,10 @@ struct SkinnyArgs {
 
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
                                 int32_t* status, const Nf4Tables& tab, cudaStream_t stream);
+//   tm_out: out viewed as [numel / 64, 64] bf16, box {64, 32} SW128 (null when numel < 64).
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
-                                  uint16_t* out, const Nf4Tables& tab, cudaStream_t stream);
+                                  uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
+                                  cudaStream_t stream);
 
 // Forward: Y[m, n] (+)= sum_k X[m,k] W'[n,k]  (+ LoRA extension in split 0).
 //   tm_x: X [M,K] box {64, BN} SW128; tm_codes: codes [N, K/2] box {32, 128};

@@ -166,44 +166,57 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const ui
 
 // ---------------------------------------------------------------- dequantize
 //
-// One thread per half block: 16 bytes of codes in (a coalesced 128-bit load
-// across the warp), 64 bytes of bf16 out (four 128-bit stores).  The 16
-// dequantised values of the block are built once per thread pair as byte
-// planes and looked up with byte permutes (no per-element multiply).
+// One thread per 64-element block (its 32 bytes of codes in two 128-bit
+// loads, a warp reading 1 KB contiguous; its table built once).  The 128
+// bytes of bf16 it produces go to shared memory in the 128-byte-swizzled
+// layout (row = block; conflict-free), and one lane per warp writes the
+// warp's 32 rows (4 KB contiguous in HBM) with a single TMA store, so the
+// global writes are whole lines.  A CTA covers one double-quantisation group,
+// so all its blocks share one s2.  A trailing partial block (numel % 64) is
+// written element by element.
 
 constexpr int kDequantThreads = 256;
 
-__global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
+__global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const __grid_constant__ CUtensorMap tm_out,
+                                                                          int has_map,
+                                                                          const uint8_t* __restrict__ codes,
                                                                           const uint8_t* __restrict__ c8,
                                                                           const float* __restrict__ s2,
                                                                           int64_t numel, uint16_t* __restrict__ out,
                                                                           Nf4Tables tab) {
+  __shared__ __align__(1024) uint8_t stage[kDequantThreads * 128];
   grid_dependency_wait();
   grid_dependents_launch();
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDequantThreads + threadIdx.x;
-  const int64_t b = t >> 1;
-  const int h = static_cast<int>(t & 1);
-  const int64_t nblocks = (numel + 63) / 64;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * kDequantThreads + tid;
+  const int64_t nblocks = (numel + 63) / 64, nfull = numel / 64;
   const bool valid = b < nblocks;
   const float chat = valid ? nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8))) : 0.0f;
-  // The two threads of a block (adjacent lanes) build its table together.
-  const Nf4Lut lut = nf4_make_lut_pair(tab, chat, static_cast<uint32_t>(h));
-  if (!valid) return;
-  const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + b * 32 + h * 16));
-  uint4 o[4];
-  o[0] = nf4_lookup8(cw.x, lut);
-  o[1] = nf4_lookup8(cw.y, lut);
-  o[2] = nf4_lookup8(cw.z, lut);
-  o[3] = nf4_lookup8(cw.w, lut);
-  const int64_t e0 = b * 64 + h * 32;
-  if (e0 + 32 <= numel) {
-    uint4* dst = reinterpret_cast<uint4*>(out + e0);
+  const Nf4Lut lut = nf4_make_lut(tab, chat);
+  uint4 c0 = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u), c1 = c0;  // code 7 = +0
+  if (valid) {
+    c0 = __ldg(reinterpret_cast<const uint4*>(codes + b * 32));
+    c1 = __ldg(reinterpret_cast<const uint4*>(codes + b * 32 + 16));
+  }
+  const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  uint8_t* row = stage + tid * 128;
+  const uint32_t sw = static_cast<uint32_t>(tid) & 7u;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = o[i];
-  } else {
-    const uint16_t* vals = reinterpret_cast<const uint16_t*>(o);
-    for (int i = 0; i < 32; ++i)
-      if (e0 + i < numel) out[e0 + i] = vals[i];
+  for (uint32_t j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(row + ((j ^ sw) << 4)) = nf4_lookup8(cw[j], lut);
+  if (b == nfull && valid) {
+    // partial last block: elements [b*64, numel)
+    for (int e = 0; e < static_cast<int>(numel - b * 64); ++e) {
+      const int j = e >> 3;
+      out[b * 64 + e] = *reinterpret_cast<const uint16_t*>(row + ((j ^ sw) << 4) + (e & 7) * 2);
+    }
+  }
+  fence_proxy_async_smem();  // this lane's rows -> async proxy
+  __syncwarp();
+  const int64_t wrow = static_cast<int64_t>(blockIdx.x) * kDequantThreads + warp * 32;
+  if (lane == 0 && has_map && wrow < nfull) {
+    tma_store_2d(&tm_out, stage + warp * 32 * 128, 0, static_cast<int>(wrow));  // rows >= nfull are clipped
+    bulk_commit_group();
+    bulk_wait_group_read0();  // shared memory stays valid until the store has read it
   }
 }
 
@@ -217,11 +230,13 @@ cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes
 }
 
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
-                                  uint16_t* out, const Nf4Tables& tab, cudaStream_t stream) {
-  const int64_t nhalf = ((numel + 63) / 64) * 2;
-  const int64_t grid = (nhalf + kDequantThreads - 1) / kDequantThreads;
+                                  uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
+                                  cudaStream_t stream) {
+  const int64_t nblocks = (numel + 63) / 64;
+  const int64_t grid = (nblocks + kDequantThreads - 1) / kDequantThreads;
+  CUtensorMap none{};
   return launch_kernel(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(kDequantThreads), 0, stream,
-                       dim3(1, 1, 1), codes, c8, s2, numel, out, tab);
+                       dim3(1, 1, 1), tm_out ? *tm_out : none, tm_out ? 1 : 0, codes, c8, s2, numel, out, tab);
 }
 
 }  // namespace qnf4

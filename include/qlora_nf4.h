@@ -119,7 +119,8 @@ QLORA_API qlora_status nf4_quantize(const uint16_t* w_bf16, int64_t numel, uint8
  * nf4_dequantize — bf16 weights from NF4 storage ("a ideia": dequantised to
  * BFloat16 at use).  w' = bf16(RN32(q[code] * RN32(e4m3(c8) * s2))), two
  * separate roundings.  Writes exactly numel bf16 values.  numel == 0 is a
- * no-op.
+ * no-op; numel >= 2^37 returns QLORA_ERR_SHAPE (the output is written
+ * through a 2-D tensor map of numel/64 rows).  All pointers 16-byte aligned.
  */
 QLORA_API qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2,
                             int64_t numel, uint16_t* w_bf16, void* stream);

@@ -85,8 +85,11 @@ def test_quantize_65b_shape_sampled_groups():
         assert s2_h[g].view(np.uint32) == s[0].view(np.uint32), g
 
 
-@pytest.mark.parametrize("numel", [64 * 256 * 8, 5000, 16384 * 3 + 100])
+@pytest.mark.parametrize("numel", [64 * 256 * 8, 5000, 16384 * 3 + 100, 1, 5, 63, 64, 65, 127, 64 * 32 + 3,
+                                   64 * 33, 16384 * 2 + 64 * 33 + 7])
 def test_dequantize_bit_exact(numel):
+    """Sizes: no full block (no tensor-map store), a partial last block, warps
+    whose 32-row store box runs past the last full row."""
     lib = _lib()
     w = synth.normal_bf16((numel,), 0.02, seed=numel + 1)
     ref_codes, ref_c8, ref_s2 = nf4.quantize(bits(w))
