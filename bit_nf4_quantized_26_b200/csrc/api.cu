@@ -343,16 +343,17 @@ struct FwdPlan {
   int s_down, per_down;
   int bn, s_fwd, per_fwd;
   bool low;                  // few-token path (lowm.cu)
-  int low_tiles, low_atiles, low_kc, low_ctas;
+  int low_tiles, low_atiles, low_kc, low_ctas, low_mpad;
   size_t off_ucat, off_pfwd, total;
 };
 
 // Few tokens: persistent CTAs (two per SM, and at least one per row tile so
 // that no CTA's range spans more than two tiles) over (tiles + atiles) * kc
 // units.
-FwdPlan plan_fwd_low(int64_t N, int64_t K, int32_t r) {
+FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r) {
   FwdPlan p{};
   p.low = true;
+  p.low_mpad = M <= 8 ? 8 : (M <= 16 ? 16 : 32);
   p.low_tiles = static_cast<int>(cdiv(N, kLowmRows));
   p.low_atiles = static_cast<int>(cdiv(r, kLowmARows));
   p.low_kc = static_cast<int>(cdiv(K / 64, 4));
@@ -360,12 +361,12 @@ FwdPlan plan_fwd_low(int64_t N, int64_t K, int32_t r) {
   const int64_t units = all_tiles * p.low_kc;
   p.low_ctas = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(2 * kSms, all_tiles)));
   p.off_pfwd = 0;
-  p.total = align256(static_cast<size_t>(p.low_ctas) * 2 * kLowmRows * kLowmMpad * 4);
+  p.total = align256(static_cast<size_t>(p.low_ctas) * 2 * kLowmRows * p.low_mpad * 4);
   return p;
 }
 
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
-  if (M <= kLowmMaxM) return plan_fwd_low(N, K, r);
+  if (M <= kLowmMaxM) return plan_fwd_low(M, N, K, r);
   FwdPlan p{};
   const int64_t kst = K / 64;
   split_plan(cdiv(M, 128), kst, 4, 2, p.s_down, p.per_down);
@@ -551,11 +552,12 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
     la.atiles = p.low_atiles;
     la.kc = p.low_kc;
     la.ctas = p.low_ctas;
+    la.mpad = p.low_mpad;
     la.status = d_status;
     la.tab = tables();
     CUtensorMap lc, la_map, lx;
     if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, r, K, 64, kLowmARows, 128) ||
-        !map_bf16(&lx, X, M, K, 64, M <= 8 ? 8 : 16, 128))
+        !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
       return QLORA_ERR_CUDA;
     {
       ProfScope ps(kKLowFwd, cs);

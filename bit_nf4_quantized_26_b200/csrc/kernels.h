@@ -117,15 +117,15 @@ cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMa
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
                           int grid_rows, int splits, cudaStream_t stream);
 
-// Few-token forward (M <= 16): register-operand MMAs on in-register
+// Few-token forward (M <= 32): register-operand MMAs on in-register
 // dequantised tiles, persistent CTAs over (128-row tile, 256-wide K chunk)
 // units; row tiles tiles .. tiles + atiles - 1 hold the rows of A, 32 each.
 // See lowm.cu.
 constexpr int kLowmThreads = 256;
 constexpr int kLowmRows = 128;
 constexpr int kLowmARows = 32;
-constexpr int kLowmMpad = 16;
-constexpr int kLowmMaxM = 16;
+constexpr int kLowmMpad = 32;  // largest partial row stride (tokens, padded to 8)
+constexpr int kLowmMaxM = 32;
 
 struct LowmArgs {
   const uint8_t* codes;  // [N, K/2]
@@ -134,7 +134,7 @@ struct LowmArgs {
   const uint16_t* X;     // [M, K] bf16
   const uint16_t* A;     // [r, K] bf16
   const uint16_t* B;     // [N, r] bf16
-  float* part;           // [ctas][2][128][16] fp32 partials
+  float* part;           // [ctas][2][128][mpad] fp32 partials
   void* Y;               // [M, N]
   int y_f32;
   float* U;              // [M, r] fp32
@@ -144,13 +144,13 @@ struct LowmArgs {
   int atiles;            // r / 32 rounded up
   int kc;                // ceil(K / 256)
   int ctas;              // CTAs of the main kernel (>= tiles + atiles)
+  int mpad;              // tokens per partial row: 8 * n8 token tiles (8, 16 or 32)
   int32_t* status;
   Nf4Tables tab;
 };
 
 //   tm_codes: codes [N, K/2] u8 box {128, 128} SW128; tm_a: A [r, K] bf16
-//   box {64, 32} SW128; tm_x: X [M, K] bf16 box {64, 8} (M <= 8) or {64, 16}
-//   SW128.
+//   box {64, 32} SW128; tm_x: X [M, K] bf16 box {64, mpad} SW128.
 cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
                             const LowmArgs& a, cudaStream_t stream);
 cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream);

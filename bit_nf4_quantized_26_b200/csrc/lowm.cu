@@ -1,10 +1,10 @@
-// lowm.cu — QLoRA linear forward for a few tokens (M <= 16):
+// lowm.cu — QLoRA linear forward for a few tokens (M <= 32):
 //   Y = X W'^T + s (X A^T) B^T,  W' = NF4-dequantised frozen weight
 // ("QLoRA" encyclopedia entry, tonho.wtf, section "como funciona": the
 // frozen weight is stored in NF4 and turned back into BFloat16 only where it
 // is used; the adapters stay 16-bit).
 //
-// At M <= 16 the product does at most 32 flops per byte of NF4 codes, so the
+// At M <= 32 the product does at most 64 flops per byte of NF4 codes, so the
 // weight stream and the nibble-to-bf16 lookups bound it, not the tensor
 // pipe.  This kernel therefore keeps the dequantised weight in registers:
 // every lane turns its own codes into bf16 pairs with byte-permute lookups
@@ -26,8 +26,9 @@
 //
 // Lane 0 of warp 0 streams each unit's codes (one 128 x 128-byte TMA box; for
 // an A tile four 32 x 64-feature boxes) and its X slice (four 64-feature
-// boxes; rows past M and features past K arrive as zeros) into a four-stage
-// shared-memory ring, two units ahead of the unit being computed.  No warp is
+// boxes; rows past M and features past K arrive as zeros) into a shared-memory
+// ring (four stages, three for 32 tokens), two units ahead of the unit being
+// computed.  No warp is
 // set aside for the copies, so every warp has the full register budget.
 //
 // The units (row tile major, K chunk minor) are cut into equal contiguous
@@ -42,7 +43,6 @@ namespace qnf4 {
 namespace {
 
 constexpr int kLowmWarps = kLowmThreads / 32;
-constexpr int kLowmStages = 4;
 constexpr int kLowmAhead = 2;                     // units in flight ahead of the one computed
 constexpr uint32_t kLowmCodes = kLowmRows * 128;  // 16 KB: 128 rows x 256 codes, or 32 A rows x 256 bf16
 constexpr uint32_t kLowmABox = kLowmARows * 128;  // {64 features, 32 rows} bf16
@@ -51,8 +51,10 @@ template <int NT>
 struct LowmPlan {
   static constexpr uint32_t kXBox = 8 * NT * 128;  // {64 features, 8 NT tokens} bf16
   static constexpr uint32_t kStage = kLowmCodes + 4 * kXBox;
-  static constexpr uint32_t kBarOff = kLowmStages * kStage;
-  static constexpr uint32_t kSmem = kBarOff + 2 * kLowmStages * 8 + 16 + 1024;
+  static constexpr int kStages = NT <= 2 ? 4 : 3;  // two CTAs per SM either way
+  static constexpr uint32_t kBarOff = kStages * kStage;
+  static constexpr uint32_t kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
+  static_assert(kStages > kLowmAhead, "ring must hold the units in flight plus the one computed");
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -113,15 +115,15 @@ __device__ __forceinline__ void load_consts(const LowmArgs& a, int tile, int kci
 }
 
 // Lane 0 of warp 0: issue the copies of unit `i` of this CTA's range into
-// stage i % kLowmStages once the eight warps have released its previous use.
+// stage i % kStages once the eight warps have released its previous use.
 template <int NT>
 __device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_a,
                                            const CUtensorMap* tm_x, const LowmArgs& a, uint8_t* smem,
                                            uint64_t* full, uint64_t* empty, int i, int tile, int kci,
                                            const WaitCtx& wc) {
   using P = LowmPlan<NT>;
-  const int s = i % kLowmStages;
-  if (i >= kLowmStages && !mbar_wait(&empty[s], ((i / kLowmStages) & 1) ^ 1, wc)) return false;
+  const int s = i % P::kStages;
+  if (i >= P::kStages && !mbar_wait(&empty[s], ((i / P::kStages) & 1) ^ 1, wc)) return false;
   uint8_t* st = smem + s * P::kStage;
   mbar_arrive_expect_tx(&full[s], kLowmCodes + 4 * P::kXBox);
   if (tile < a.tiles) {
@@ -144,8 +146,8 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
-  uint64_t* empty = full + kLowmStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kLowmStages);
+  uint64_t* empty = full + P::kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + P::kStages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool issuer = threadIdx.x == 0;
 
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   const int kci0 = static_cast<int>(u_beg - static_cast<int64_t>(tile0) * a.kc);
 
   if (issuer) {
-    for (int s = 0; s < kLowmStages; ++s) {
+    for (int s = 0; s < P::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kLowmWarps);
     }
@@ -212,8 +214,8 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     }
     const bool more = i + 1 < count;
     if (issuer && ok && issued < count) issue_next();
-    const int s = i % kLowmStages;
-    if (!mbar_wait_all(&full[s], (i / kLowmStages) & 1, wc)) break;
+    const int s = i % P::kStages;
+    if (!mbar_wait_all(&full[s], (i / P::kStages) & 1, wc)) break;
     const uint8_t* st = smem + s * P::kStage;
     // X box of this lane's block; token row 8n + g has phase g.
     const uint8_t* xs = st + kLowmCodes + t * P::kXBox + g * 128;
@@ -269,12 +271,13 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     // Last unit of this tile in the range: write the partial, restart.
     if (!more || ntile != tile) {
       const int slot = tile == tile0 ? 0 : 1;
-      float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * kLowmRows + warp * 16 + g) * kLowmMpad +
+      constexpr int kMpad = 8 * NT;  // == a.mpad
+      float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * kLowmRows + warp * 16 + g) * kMpad +
                    2 * t;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(acc[n][0], acc[n][1]);
-        *reinterpret_cast<float2*>(dst + 8 * kLowmMpad + 8 * n) = make_float2(acc[n][2], acc[n][3]);
+        *reinterpret_cast<float2*>(dst + 8 * kMpad + 8 * n) = make_float2(acc[n][2], acc[n][3]);
         acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
       }
     }
@@ -284,13 +287,13 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   // After a timeout, let copies still in flight land before the CTA exits
   // (after a normal run every stage's last phase has completed already).
   if (issuer) {
-    for (int i = max(0, issued - kLowmStages); i < issued; ++i)
-      lowm_drain(&full[i % kLowmStages], (i / kLowmStages) & 1);
+    for (int i = max(0, issued - P::kStages); i < issued; ++i)
+      lowm_drain(&full[i % P::kStages], (i / P::kStages) & 1);
   }
 }
 
-// Finisher layout: 256 threads = 64 rows x 4 token quads; CTA b covers rows
-// [64 b, 64 b + 64) of the output (half of row tile b / 2).
+// Finisher layout: 64 rows x mpad/4 token quads (128, 256 or 512 threads);
+// CTA b covers rows [64 b, 64 b + 64) of the output (half of row tile b / 2).
 constexpr int kFinRows = 64;
 
 // Sum over the CTAs that touched `tile`, in CTA order, of the partial of
@@ -310,7 +313,7 @@ __device__ __forceinline__ float4 sum_tile_partials(const LowmArgs& a, int tile,
       if (c <= c1) {
         const int first = static_cast<int>(unit_start(c, units, a.ctas) / a.kc);
         v[j] = *reinterpret_cast<const float4*>(
-            a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * kLowmMpad + 4 * q);
+            a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * a.mpad + 4 * q);
       }
     }
 #pragma unroll
@@ -330,7 +333,7 @@ __device__ __forceinline__ float4 sum_tile_partials(const LowmArgs& a, int tile,
 // U = the A tiles' partials summed (every CTA forms U; CTA 0 stores it).  The
 // row of B is read before the wait for the main kernel (B is not one of its
 // outputs).
-__global__ void __launch_bounds__(256) lowm_finish_kernel(const LowmArgs a) {
+__global__ void __launch_bounds__(512) lowm_finish_kernel(const LowmArgs a) {
   __shared__ float su[kLowmMpad][64];
   const int tid = threadIdx.x;
   const int rl = tid & (kFinRows - 1), q = tid >> 6;
@@ -409,13 +412,17 @@ static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorM
 
 cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
                             const LowmArgs& a, cudaStream_t stream) {
-  return a.M <= 8 ? launch_lowm_impl<1>(tm_codes, tm_a, tm_x, a, stream)
-                  : launch_lowm_impl<2>(tm_codes, tm_a, tm_x, a, stream);
+  switch (a.mpad) {
+    case 8: return launch_lowm_impl<1>(tm_codes, tm_a, tm_x, a, stream);
+    case 16: return launch_lowm_impl<2>(tm_codes, tm_a, tm_x, a, stream);
+    case 32: return launch_lowm_impl<4>(tm_codes, tm_a, tm_x, a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>((a.N + kFinRows - 1) / kFinRows);
-  return launch_kernel(lowm_finish_kernel, dim3(grid), dim3(256), 0, stream, dim3(1, 1, 1), a);
+  return launch_kernel(lowm_finish_kernel, dim3(grid), dim3(kFinRows * (a.mpad / 4)), 0, stream, dim3(1, 1, 1), a);
 }
 
 }  // namespace qnf4

@@ -89,12 +89,14 @@ def test_ragged_shapes(M, N, K, r):
 @pytest.mark.parametrize("M,N,K,r", [
     (1, 64, 64, 16), (3, 320, 832, 48), (8, 448, 1344, 64), (9, 128, 64, 16),
     (12, 1088, 2112, 32), (16, 960, 4160, 64), (5, 4096, 256, 16), (7, 2048, 8192, 64),
-    (11, 1024, 16384, 48), (16, 4096, 4096, 32),
+    (11, 1024, 16384, 48), (16, 4096, 4096, 32), (17, 320, 832, 48), (24, 1088, 2112, 64),
+    (32, 960, 4160, 16), (29, 2048, 8192, 32),
 ])
 def test_few_tokens(M, N, K, r):
-    """M <= 16 forward path: row tiles with a half-empty last tile (N % 128 =
+    """M <= 32 forward path: row tiles with a half-empty last tile (N % 128 =
     64), K chunks with 1..3 of their 4 blocks present, 1..19 units per CTA,
-    ranges that start and end inside a tile, r = 16..64 rows of A."""
+    ranges that start and end inside a tile, r = 16..64 rows of A, 1, 2 and 4
+    token tiles of 8."""
     _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=1)
     _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=0)
 
@@ -185,7 +187,7 @@ def test_c3_mlp_with_outliers(N, K):
     _check_sampled(N, K, 8192, 64, 0.25, 3, outliers=True, nrows=48)
 
 
-@pytest.mark.parametrize("M", [1, 16, 128, 2048])
+@pytest.mark.parametrize("M", [1, 16, 32, 128, 2048])
 @pytest.mark.parametrize("N,K", [(22016, 8192), (8192, 22016)])
 def test_c5_forward_sweep(N, K, M):
     _check_sampled(N, K, M, 64, 0.25, 5, nrows=32, bwd=False)
