@@ -208,6 +208,73 @@ def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
     return out
 
 
+def c1_graph_timing(lib, synth, torch, dev, reps=200):
+    """c1 step (quantize + fwd + bwd, 512x512, 64 tokens, r=16) eager vs one CUDA graph.
+
+    The step is launch-bound at this size; the graph holds the library's
+    kernels (programmatic launches and the side-stream fork/join included).
+    Outputs of a replay are compared bit for bit with an eager step.
+    """
+    wl = synth.WORKLOADS["c1"]
+    lin = wl.linears[0]
+    M, N, K, r, s = wl.m_tokens, lin.n_out, lin.k_in, wl.r, wl.s
+    g = {k: v.to(dev) for k, v in synth.linear_inputs(lin, M, r, 0).items()}
+    nc, nb, ns = lib.nf4_sizes(N * K)
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+    c8 = torch.empty(nb, dtype=torch.uint8, device=dev)
+    s2 = torch.empty(ns, dtype=torch.float32, device=dev)
+    W = lib.NF4Weight(codes, c8, s2, N, K)
+    out = {"Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+           "U": torch.empty((M, r), dtype=torch.float32, device=dev),
+           "dX": torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+           "dA": torch.empty((r, K), dtype=torch.float32, device=dev),
+           "dB": torch.empty((N, r), dtype=torch.float32, device=dev)}
+    ws_f = torch.empty(max(lib.qlora_fwd_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(lib.qlora_bwd_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        lib.nf4_quantize(g["W"].reshape(-1), codes, c8, s2)
+        lib.qlora_linear_fwd(g["X"], W, g["A"], g["B"], s, Y=out["Y"], U=out["U"], ws=ws_f)
+        lib.qlora_linear_bwd(g["dY"], g["X"], out["U"], W, g["A"], g["B"], s, dX=out["dX"], dA=out["dA"],
+                             dB=out["dB"], ws=ws_b)
+
+    cs = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(cs):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+    ref = {k: v.clone() for k, v in out.items()}
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cs):
+        step()
+    for v in out.values():
+        v.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    equal = all(torch.equal(out[k].view(torch.int16) if out[k].dtype == torch.bfloat16 else out[k].view(torch.int32),
+                            ref[k].view(torch.int16) if ref[k].dtype == torch.bfloat16 else ref[k].view(torch.int32))
+                for k in out)
+
+    def timed(fn):
+        with torch.cuda.stream(cs):
+            for _ in range(10):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(cs)
+            for _ in range(reps):
+                fn()
+            e1.record(cs)
+        e1.synchronize()
+        return 1000.0 * e0.elapsed_time(e1) / reps
+
+    eager_us = timed(step)
+    graph_us = timed(graph.replay)
+    del graph
+    return {"eager_us_per_step": round(eager_us, 2), "graph_us_per_step": round(graph_us, 2),
+            "replay_bit_equal": bool(equal), "steps": reps,
+            "workload": "512x512 NF4, 64 tokens, r=16: quantize + fwd + bwd back to back (L2-resident)"}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -371,6 +438,7 @@ def run_ours(args, rank, world):
 
     # ------------------------------------------- 65B-shaped forward sweep
     c5 = c5_forward_sweep(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
+    c1g = c1_graph_timing(lib, synth, torch, dev) if (rank == 0 and not args.no_sweep) else None
 
     # ------------------------------------------------------------- e2e
     host = {k: torch.empty_like(g[k], device="cpu").pin_memory() for k in ("W", "X", "dY")}
@@ -432,6 +500,7 @@ def run_ours(args, rank, world):
                         for n, k in sorted(kern.items(), key=lambda x: -x[1]["ms_total"])},
             "nf4_quantize_gbs": quant_gbs, "nf4_dequantize_gbs": dequant_gbs,
             "c5_forward": c5,
+            "c1_graph": c1g,
             "nf4_hbm_frac": {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
                              "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
         }
