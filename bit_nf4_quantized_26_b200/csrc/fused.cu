@@ -38,7 +38,7 @@ struct FusedPlan {
   static constexpr uint32_t kA = 16384;     // W-side tile 128 x 64 bf16
   static constexpr uint32_t kC = 4096;      // packed codes of the stage
   static constexpr uint32_t kStage = kB + kA + kC;
-  static constexpr uint32_t kCtasPerSm = BN <= 64 ? 2 : 1;
+  static constexpr uint32_t kCtasPerSm = BN <= 128 ? 2 : 1;
   static constexpr uint32_t kFit = (233472u / kCtasPerSm - 1024u - 2048u) / kStage;
   static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
   static constexpr uint32_t kBarOff = kStages * kStage;
