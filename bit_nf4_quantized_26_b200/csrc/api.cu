@@ -318,8 +318,8 @@ class Fork {
 
 // ------------------------------------------------------------ planning
 //
-// Split counts depend only on the shape (aim: about two CTAs per SM of a
-// 148-SM B200), so the workspace query is a pure host function.
+// Split counts depend only on the shape (sized against the 148 SMs of a
+// B200), so the workspace query is a pure host function.
 
 constexpr int kSms = 148;
 constexpr int64_t kMaxCluster = 8;  // portable cluster size: splits reduced in-cluster
@@ -328,10 +328,10 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Number of slices for `stages` contraction steps over `tiles` output tiles so
-// that tiles * slices fits in one wave of `ctas_per_sm` CTAs per SM, with at
-// least `min_per` steps per slice; every slice is non-empty.
-void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int ctas_per_sm, int& splits, int& per) {
-  int64_t s = std::max<int64_t>(1, (int64_t(kSms) * ctas_per_sm) / std::max<int64_t>(tiles, 1));
+// that tiles * slices stays within `cta_budget` CTAs, with at least `min_per`
+// steps per slice; every slice is non-empty.
+void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int64_t cta_budget, int& splits, int& per) {
+  int64_t s = std::max<int64_t>(1, cta_budget / std::max<int64_t>(tiles, 1));
   s = std::min<int64_t>(s, std::max<int64_t>(1, stages / std::max<int64_t>(min_per, 1)));
   s = std::min<int64_t>(s, kMaxCluster);
   const int64_t p = cdiv(stages, s);
@@ -369,7 +369,15 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (M <= kLowmMaxM) return plan_fwd_low(M, N, K, r);
   FwdPlan p{};
   const int64_t kst = K / 64;
-  split_plan(cdiv(M, 128), kst, 4, 2, p.s_down, p.per_down);
+  split_plan(cdiv(M, 128), kst, 4, 2 * kSms, p.s_down, p.per_down);
+  if (M > kWideM) {
+    // The wide GEMM needs U only in its last stages and does not wait for it
+    // before then, so U = X A^T runs beside the GEMM's main loop: one CTA per
+    // 128-token tile over the whole contraction (about half as long as a GEMM
+    // tile's main loop) holds few SMs and leaves the rest to the GEMM.
+    p.s_down = 1;
+    p.per_down = static_cast<int>(kst);
+  }
   p.bn = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
   if (M <= 256) {
@@ -402,9 +410,15 @@ struct BwdPlan {
 
 BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   BwdPlan p{};
-  split_plan(cdiv(M, 128), N / 64, 4, 2, p.s_du, p.per_du);
-  split_plan(cdiv(N, 128), cdiv(M, 64), 4, 2, p.s_db, p.per_db);
-  split_plan(cdiv(K, 128), cdiv(M, 64), 4, 2, p.s_da, p.per_da);
+  split_plan(cdiv(M, 128), N / 64, 4, 2 * kSms, p.s_du, p.per_du);
+  if (M > kWideM) {  // dU runs beside the wide dX GEMM's main loop (as U beside Y)
+    p.s_du = 1;
+    p.per_du = static_cast<int>(N / 64);
+  }
+  // dB and dA run on the side stream beside dX: few CTAs with long
+  // contractions take fewer SM-cycles from it than many short ones.
+  split_plan(cdiv(N, 128), cdiv(M, 64), 4, kSms / 2, p.s_db, p.per_db);
+  split_plan(cdiv(K, 128), cdiv(M, 64), 4, kSms / 2, p.s_da, p.per_da);
   p.bn = M > 128 ? 256 : 128;
   size_t off = 0;
   p.off_sucat = off;

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
         mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
     }
+    __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
     if (!waited) {  // lanes 1..31, a split without extension stages, or a producer that gave up
       grid_dependency_wait();
       grid_dependents_launch();
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       umma_commit(accf);
       if (aborted) mbar_wait_drain(accf, 0);
     }
+    __syncwarp();
     grid_dependency_wait();
     grid_dependents_launch();
   } else {
@@ -444,6 +446,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
         mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
     }
+    __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
     if (!waited) {  // lanes 1..31, or a producer that gave up
       grid_dependency_wait();
       grid_dependents_launch();
@@ -481,6 +484,7 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(accf);
       if (aborted) mbar_wait_drain(accf, 0);
     }
+    __syncwarp();
     grid_dependency_wait();
     grid_dependents_launch();
   } else {

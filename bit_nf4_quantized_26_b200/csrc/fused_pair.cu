@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(192, 1)
         if (rank == 0) wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
       }
     }
+    __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
     if (!waited) {  // lanes 1..31, or a producer that gave up early
       grid_dependency_wait();
       grid_dependents_launch();
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit_pair(accf, 0x3);
       if (aborted) wait_drain(accf, 0);
     }
+    __syncwarp();
     grid_dependency_wait();
     grid_dependents_launch();
   } else {

@@ -230,8 +230,12 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   cluster_sync_all();
   {
     const float* part = reinterpret_cast<const float*>(smem);
-    const uint32_t S = gridDim.y;  // the cluster spans the split dimension
-    const uint32_t rank = cluster_ctarank();
+    const uint32_t S = gridDim.y;      // splits; a cluster of S > 1 spans the split dimension
+    const uint32_t rank = blockIdx.y;  // this CTA's slice of the tile's rows
+    // Cluster rank of the CTA holding split z: z itself, or with S = 1 (a
+    // cluster of two row tiles, or none) this CTA.
+    const uint32_t self = cluster_ctarank();
+    auto holder = [&](uint32_t z) { return S == 1 ? self : z; };
     const bool by_rows = (MODE != kSkDA);
     const int R = by_rows ? 128 : a.r;                 // rows of the partial tile
     const int C = by_rows ? a.r : 128;                 // columns
@@ -244,9 +248,9 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
       const int row = r0 + e / c4;
       const int col = (e % c4) * 4;
       const float* loc = part + row * ld + col;
-      float4 acc = dsmem_ld_f4(dsmem_addr(loc, 0));
+      float4 acc = dsmem_ld_f4(dsmem_addr(loc, holder(0)));
       for (uint32_t z = 1; z < S; ++z) {
-        const float4 v = dsmem_ld_f4(dsmem_addr(loc, z));
+        const float4 v = dsmem_ld_f4(dsmem_addr(loc, holder(z)));
         acc.x = __fadd_rn(acc.x, v.x);
         acc.y = __fadd_rn(acc.y, v.y);
         acc.z = __fadd_rn(acc.z, v.z);
@@ -300,8 +304,12 @@ static cudaError_t launch_skinny_impl(const CUtensorMap& tmA, const CUtensorMap&
     attr_set = true;
   }
   if (splits < 1 || splits > 8) return cudaErrorInvalidValue;
-  return launch_kernel(skinny_kernel<MODE>, dim3(grid_rows, splits, 1), dim3(192), P::kSmem, stream,
-                       dim3(1, static_cast<unsigned>(splits), 1), tmA, tmB, a);
+  // Unsplit products run beside a CTA-pair GEMM: launched as clusters of two
+  // row tiles they sit on both SMs of a TPC, rather than on one SM of many
+  // TPCs, each of which could then hold no GEMM pair.
+  const dim3 cluster = (splits == 1 && grid_rows % 2 == 0) ? dim3(2, 1, 1) : dim3(1, static_cast<unsigned>(splits), 1);
+  return launch_kernel(skinny_kernel<MODE>, dim3(grid_rows, splits, 1), dim3(192), P::kSmem, stream, cluster, tmA,
+                       tmB, a);
 }
 
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
