@@ -18,7 +18,10 @@ Sources (web pages; cited by title and section):
   adapters in 16 bit receive the only gradients.
 * "Tutorial fine-tuning LLM LoRA/QLoRA 2026" (nexusinovation), section
   "LoRA: O Padrão Ouro de Eficiência": W' = W + alpha*A*B, and the
-  ``LoraConfig``/``BitsAndBytesConfig`` knobs in "Mão na Massa".
+  ``LoraConfig``/``BitsAndBytesConfig`` knobs and the ``paged_adamw_8bit``
+  trainer in "Mão na Massa".
+* "QLoRA" encyclopedia entry, section "como funciona", third piece: optimizer
+  states paged between GPU and CPU memory (unified memory).
 
 Modules:
 
@@ -27,10 +30,13 @@ Modules:
   dequantisation (encodings: the GPU must match these bit for bit).
 * :mod:`oracle.linear` — forward / backward of the adapter-augmented linear in
   fp64 (the GPU must match within a relative Frobenius error).
+* :mod:`oracle.optim` — the adapter optimizer step, AdamW with 8-bit blockwise
+  FP8 states (every operation one fp32 rounding: the GPU must match bit for
+  bit).
 
 Parity status per function is listed in each module header.  Every function
 here is pinned by ``tests/test_oracle_*.py`` to facts the pages or
 mathematics fix; functions whose pin is partial say so.
 """
 
-from . import numerics, nf4, linear  # noqa: F401
+from . import numerics, nf4, linear, optim  # noqa: F401
