@@ -436,6 +436,9 @@ def run_ours(args, rank, world):
     dequant_gbs = bytes_nf4 / (statistics.median(dqt) * 1e-3) / 1e9
     del big, bcodes, bc8, bs2, bout
 
+    # ------------------------------------------- adapter optimizer step
+    adamw = adamw8_timing(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
+
     # ------------------------------------------- 65B-shaped forward sweep
     c5 = c5_forward_sweep(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
     c1g = c1_graph_timing(lib, synth, torch, dev) if (rank == 0 and not args.no_sweep) else None
@@ -501,10 +504,48 @@ def run_ours(args, rank, world):
             "nf4_quantize_gbs": quant_gbs, "nf4_dequantize_gbs": dequant_gbs,
             "c5_forward": c5,
             "c1_graph": c1g,
+            "adamw8": adamw,
             "nf4_hbm_frac": {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
                              "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
         }
         print(json.dumps(line), flush=True)
+
+
+def adamw8_timing(lib, synth, torch, dev, flush, peaks, layers=10, reps=10):
+    """AdamW with 8-bit states over the r=64 adapters of ``layers`` 65B-shaped
+    layers (about 100M parameters, 1.2 GB streamed per step: larger than L2),
+    states in device memory and in paged (managed, device-resident) memory.
+    Algorithmic bytes per parameter: bf16 p read + write, fp32 gradient, two
+    state bytes read + write, two fp32 scales per 256 read + write."""
+    import statistics
+    r = 64
+    per_layer = sum(r * (lin.n_out + lin.k_in) for lin in synth.c5_layer_linears())
+    n = per_layer * layers
+    gen = torch.Generator(device=dev).manual_seed(5)
+    p = (torch.randn(n, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    grad = torch.randn(n, generator=gen, device=dev) * 1e-3
+    bytes_per = 2 + 2 + 4 + 2 + 2 + 16 / 256
+    out = {"params": n, "layers": layers, "bytes_per_param": bytes_per}
+    for paged in (False, True):
+        st = lib.AdamW8State(n, paged=paged)
+        st.prefetch(to_host=False)
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            lib.qlora_adamw8_step(p, grad, st, lr=2e-4, step=i + 1)
+            e1.record()
+            e1.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        gbs = n * bytes_per / (ms * 1e-3) / 1e9
+        key = "paged" if paged else "device"
+        out[key] = {"us": ms * 1e3, "gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"]}
+        st.close()
+    del p, grad
+    return out
 
 
 def run_case(args):

@@ -1,4 +1,5 @@
-"""Python binding of ``libqlora_nf4.so`` (the C ABI in ``include/qlora_nf4.h``).
+"""Python binding of ``libqlora_nf4.so`` (the C ABI in ``include/qlora_nf4.h`` and
+``include/qlora_optim.h``).
 
 Argument marshalling only: every step of the computation runs in the
 library's CUDA kernels.  PyTorch provides device memory and the current
@@ -11,6 +12,7 @@ Functions keep the C names:
 * :func:`qlora_linear_fwd` / :func:`qlora_linear_bwd`
 * :func:`qlora_fwd_workspace_size` / :func:`qlora_bwd_workspace_size`
 * :func:`nf4_levels`, :func:`qlora_strerror`
+* :func:`qlora_adamw8_step` with :class:`AdamW8State` (``include/qlora_optim.h``)
 """
 
 import ctypes
@@ -234,3 +236,102 @@ def profile_collect(capacity=1 << 16):
 def raw():
     """The loaded ``ctypes.CDLL`` (for callers that pass raw pointers)."""
     return _lib
+
+
+# ------------------------------------------------------------ optimizer step
+# (include/qlora_optim.h: AdamW with 8-bit states in paged memory)
+
+_F = ctypes.c_float
+_lib.qlora_adamw8_step.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _F, _F, _F, _F, _F, _I64, _P, _P]
+_lib.qlora_adamw8_step.restype = ctypes.c_int
+_lib.qlora_paged_alloc.argtypes = [ctypes.POINTER(ctypes.c_void_p), _SZ]
+_lib.qlora_paged_alloc.restype = ctypes.c_int
+_lib.qlora_paged_prefetch.argtypes = [_P, _SZ, _I32, _P]
+_lib.qlora_paged_prefetch.restype = ctypes.c_int
+_lib.qlora_paged_free.argtypes = [_P]
+_lib.qlora_paged_free.restype = ctypes.c_int
+
+EXPORTED = EXPORTED + ("qlora_adamw8_step", "qlora_paged_alloc", "qlora_paged_prefetch", "qlora_paged_free")
+
+STATE_BLOCK = 256  # parameters per fp32 state scale
+
+
+def _al(b):
+    return (b + 255) & ~255
+
+
+class AdamW8State:
+    """8-bit AdamW state of an ``n``-parameter tensor: E4M3 codes of m and of
+    sqrt(v) (one byte each per parameter) and one fp32 scale per 256
+    parameters for each.  ``paged=True`` puts all four arrays in one CUDA
+    managed allocation (``qlora_paged_alloc``: resident in HBM, evicted to
+    host RAM under memory pressure, migrated back when touched); otherwise
+    they live in a torch device tensor.  A fresh state is all zeros."""
+
+    def __init__(self, n, paged=True, device=None):
+        self.n = int(n)
+        self.nb = -(-self.n // STATE_BLOCK)
+        self._offs = (0, _al(self.n), 2 * _al(self.n), 2 * _al(self.n) + _al(4 * self.nb))
+        self.bytes = self._offs[3] + _al(4 * self.nb)
+        self.paged = paged
+        self._buf = None
+        self._base = None
+        if paged:
+            ptr = ctypes.c_void_p()
+            _check(_lib.qlora_paged_alloc(ctypes.byref(ptr), self.bytes), "qlora_paged_alloc")
+            self._base = ptr.value
+        else:
+            self._buf = torch.zeros(self.bytes, dtype=torch.uint8, device=device or "cuda")
+            self._base = self._buf.data_ptr()
+
+    def pointers(self):
+        """Device-usable addresses of (m8, u8, m_scale, u_scale)."""
+        return tuple(self._base + o for o in self._offs)
+
+    def prefetch(self, to_host=False, stream=None):
+        """Migrate a paged state to the device (or to host RAM) on ``stream``."""
+        if self.paged:
+            _check(_lib.qlora_paged_prefetch(ctypes.c_void_p(self._base), self.bytes, 1 if to_host else 0,
+                                             _stream(stream)), "qlora_paged_prefetch")
+
+    def host_arrays(self):
+        """Copies of (m8, u8, m_scale, u_scale) as numpy arrays (synchronises)."""
+        import numpy as np
+        torch.cuda.synchronize()
+        if self.paged:
+            def grab(off, n, ct, dt):
+                return np.ctypeslib.as_array((ct * n).from_address(self._base + off)).astype(dt, copy=True)
+            return (grab(self._offs[0], self.n, ctypes.c_uint8, np.uint8),
+                    grab(self._offs[1], self.n, ctypes.c_uint8, np.uint8),
+                    grab(self._offs[2], self.nb, ctypes.c_float, np.float32),
+                    grab(self._offs[3], self.nb, ctypes.c_float, np.float32))
+        b = self._buf.cpu().numpy()
+        o = self._offs
+        return (b[o[0]:o[0] + self.n].copy(), b[o[1]:o[1] + self.n].copy(),
+                b[o[2]:o[2] + 4 * self.nb].view(np.float32).copy(), b[o[3]:o[3] + 4 * self.nb].view(np.float32).copy())
+
+    def close(self):
+        if self.paged and self._base is not None:
+            torch.cuda.synchronize()
+            _check(_lib.qlora_paged_free(ctypes.c_void_p(self._base)), "qlora_paged_free")
+        self._base = None
+        self._buf = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def qlora_adamw8_step(p, grad, state, lr, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1,
+                      status=None, stream=None):
+    """One AdamW step in place on the bf16 parameter tensor ``p`` with fp32
+    gradient ``grad`` and the 8-bit :class:`AdamW8State` ``state``."""
+    assert p.dtype == torch.bfloat16 and grad.dtype == torch.float32
+    assert p.is_contiguous() and grad.is_contiguous() and p.numel() == grad.numel() == state.n
+    m8, u8, ms, us = state.pointers()
+    _check(_lib.qlora_adamw8_step(_ptr(p), _ptr(grad), ctypes.c_void_p(m8), ctypes.c_void_p(u8),
+                                  ctypes.c_void_p(ms), ctypes.c_void_p(us), state.n, lr, beta1, beta2, eps,
+                                  weight_decay, int(step), _ptr(status), _stream(stream)), "qlora_adamw8_step")
+    return p

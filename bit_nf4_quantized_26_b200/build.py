@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqlora_nf4.so")
-SOURCES = ["api.cu", "quant.cu", "fused.cu", "fused_pair.cu", "skinny.cu", "lowm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "fused.cu", "fused_pair.cu", "skinny.cu", "lowm.cu", "noalloc.cu", "optim.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
@@ -33,7 +33,7 @@ def _stale(obj, src):
     if not os.path.exists(obj):
         return True
     deps = [src] + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    deps.append(os.path.join(ROOT, "include", "qlora_nf4.h"))
+    deps += [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
     t = os.path.getmtime(obj)
     return any(os.path.getmtime(d) > t for d in deps)
 

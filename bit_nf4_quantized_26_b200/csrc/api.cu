@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "kernels.h"
+#include "../../include/qlora_optim.h"
 
 using namespace qnf4;
 
@@ -194,11 +195,11 @@ qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLO
 
 enum KernelId {
   kKQuantize = 0, kKDequantize, kKDown, kKFusedFwd, kKFinishFwd, kKLowFwd, kKLowFinish, kKDU, kKDB, kKFusedDX,
-  kKDA, kKCount
+  kKDA, kKAdamW8, kKCount
 };
 const char* const kKernelNames[kKCount] = {
     "nf4_quantize", "nf4_dequantize", "lora_down", "fused_fwd", "finish_fwd", "lowm_fwd", "lowm_finish",
-    "lora_du", "lora_db", "fused_dx", "lora_da"};
+    "lora_du", "lora_db", "fused_dx", "lora_da", "adamw8"};
 
 struct ProfRecord {
   int id;
@@ -800,6 +801,76 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   }
 
   return QLORA_OK;
+}
+
+// ------------------------------------------------------------------ optimizer
+
+qlora_status qlora_adamw8_step(uint16_t* p, const float* grad, uint8_t* m8, uint8_t* u8, float* m_scale,
+                               float* u_scale, int64_t n, float lr, float beta1, float beta2, float eps,
+                               float weight_decay, int64_t step, int32_t* d_status, void* stream) {
+  if (n < 0 || n >= (int64_t(1) << 40) || step < 1) return QLORA_ERR_SHAPE;
+  if (!std::isfinite(lr) || !std::isfinite(eps) || !std::isfinite(weight_decay) || eps < 0.0f ||
+      !(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f))
+    return QLORA_ERR_SHAPE;
+  if (n == 0) return QLORA_OK;
+  if (!p || !grad || !m8 || !u8 || !m_scale || !u_scale) return QLORA_ERR_NULL;
+  if (!aligned16(p) || !aligned16(grad) || !aligned16(m8) || !aligned16(u8) || !aligned16(m_scale) ||
+      !aligned16(u_scale) || (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  AdamW8Args a{};
+  a.p = p;
+  a.g = grad;
+  a.m8 = m8;
+  a.u8 = u8;
+  a.m_scale = m_scale;
+  a.u_scale = u_scale;
+  a.n = n;
+  a.lr = lr;
+  a.b1 = beta1;
+  a.b2 = beta2;
+  a.omb1 = 1.0f - beta1;  // one fp32 subtraction (exact for beta in [0.5, 1))
+  a.omb2 = 1.0f - beta2;
+  a.eps = eps;
+  a.wd = weight_decay;
+  // Bias corrections in fp64 from the fp32 betas, rounded once to fp32.
+  const double t = static_cast<double>(step);
+  a.bc1 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(beta1), t)));
+  a.bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), t)));
+  a.status = d_status;
+  ProfScope ps(kKAdamW8, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_adamw8(a, static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_paged_alloc(void** ptr, size_t bytes) {
+  if (!ptr) return QLORA_ERR_NULL;
+  *ptr = nullptr;
+  if (bytes == 0) return QLORA_ERR_SHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  void* q = nullptr;
+  if (cudaMallocManaged(&q, bytes, cudaMemAttachGlobal) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemAdvise(q, bytes, cudaMemAdviseSetPreferredLocation, dev) != cudaSuccess ||
+      cudaMemset(q, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(q);
+    return QLORA_ERR_CUDA;
+  }
+  *ptr = q;
+  return QLORA_OK;
+}
+
+qlora_status qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_host, void* stream) {
+  if (!ptr) return QLORA_ERR_NULL;
+  if (bytes == 0) return QLORA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  return from_cuda(cudaMemPrefetchAsync(ptr, bytes, to_host ? cudaCpuDeviceId : dev,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_paged_free(void* ptr) {
+  if (!ptr) return QLORA_OK;
+  return from_cuda(cudaFree(ptr));
 }
 
 }  // extern "C"

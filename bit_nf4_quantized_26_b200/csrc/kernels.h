@@ -76,6 +76,20 @@ struct SkinnyArgs {
   int32_t* status;
 };
 
+// AdamW step with 8-bit states (optim.cu).
+struct AdamW8Args {
+  uint16_t* p;       // [n] bf16 parameters, in place
+  const float* g;    // [n] fp32 gradients
+  uint8_t* m8;       // [n] E4M3 codes of m
+  uint8_t* u8;       // [n] E4M3 codes of sqrt(v)
+  float* m_scale;    // [ceil(n/256)]
+  float* u_scale;    // [ceil(n/256)]
+  int64_t n;
+  float lr, b1, b2, omb1, omb2, eps, wd, bc1, bc2;
+  int32_t* status;
+};
+cudaError_t launch_adamw8(const AdamW8Args& a, cudaStream_t stream);
+
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
                                 int32_t* status, const Nf4Tables& tab, cudaStream_t stream);
 //   tm_out: out viewed as [numel / 64, 64] bf16, box {64, 32} SW128 (null when numel < 64).

@@ -15,19 +15,19 @@ import bit_nf4_quantized_26_b200 as q
 from oracle import nf4
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("qlora_nf4.h", "qlora_optim.h")]
 
 OK, NULL, SHAPE, ALIGN, WS, CUDA, ARCH, DTYPE = 0, 1, 2, 3, 4, 7, 8, 9
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
 
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 12
+    assert len(names) == 16
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -122,3 +122,29 @@ def test_valid_arguments_without_device_fail_cleanly():
     error status (never crashes, never falls back)."""
     assert _fwd() in (CUDA, ARCH)
     assert q.raw().nf4_quantize(FAKE, 64, FAKE, FAKE, FAKE, None, None) in (CUDA, ARCH)
+
+
+def test_adamw8_rejects_bad_arguments_before_touching_a_device():
+    """Sizes, step and hyper-parameters are checked first, then pointers and
+    alignment; none of these reach the device."""
+    f = q._lib.qlora_adamw8_step
+    P = ctypes.c_void_p
+    good = [P(256)] * 6
+    def call(ptrs=good, n=10, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1):
+        return f(*ptrs, n, lr, b1, b2, eps, wd, step, None, None)
+    assert call(n=-1) == SHAPE
+    assert call(n=1 << 40) == SHAPE
+    assert call(step=0) == SHAPE
+    assert call(b1=1.0) == SHAPE and call(b2=-0.1) == SHAPE and call(b1=float("nan")) == SHAPE
+    assert call(eps=-1e-8) == SHAPE and call(lr=float("inf")) == SHAPE and call(wd=float("nan")) == SHAPE
+    assert call(n=0) == OK
+    assert call(ptrs=[None] + good[1:]) == NULL
+    assert call(ptrs=good[:3] + [None] + good[4:]) == NULL
+    assert call(ptrs=[P(256 + 8)] + good[1:]) == ALIGN
+    assert call(ptrs=good[:5] + [P(256 + 4)]) == ALIGN
+
+
+def test_paged_calls_reject_null_pointers():
+    assert q._lib.qlora_paged_alloc(None, 16) == NULL
+    assert q._lib.qlora_paged_prefetch(None, 16, 0, None) == NULL
+    assert q._lib.qlora_paged_free(None) == OK
