@@ -551,13 +551,37 @@ def adamw8_timing(lib, synth, torch, dev, flush, peaks, layers=10, reps=10):
 def run_case(args):
     """Profiler driver: time one entry point on one shape (no JSON contract).
 
-    --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), or quant:N:K (NF4 quantisation of
-    an N x K weight), --steps calls after 2 warm-up calls.
+    --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), quant:N:K / dequant:N:K (NF4
+    quantisation / dequantisation of an N x K weight), or adamw8:n (one 8-bit AdamW
+    step over n parameters), --steps calls after 2 warm-up calls.
     """
     import torch
 
     import bit_nf4_quantized_26_b200 as lib
     import synth
+    if args.case.startswith("adamw8:"):
+        n = int(args.case.split(":")[1])
+        gen = torch.Generator(device="cuda").manual_seed(5)
+        p = (torch.randn(n, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        g = torch.randn(n, generator=gen, device="cuda") * 1e-3
+        st = lib.AdamW8State(n, paged=False)
+        for i in range(2 + args.steps):
+            lib.qlora_adamw8_step(p, g, st, lr=2e-4, step=i + 1)
+        torch.cuda.synchronize()
+        st.close()
+        print(json.dumps({"case": args.case, "ok": True}))
+        return
+    if args.case.startswith("dequant:"):
+        _, N, K = args.case.split(":")
+        w = synth.weight_bf16(int(N), int(K), seed=1, device="cuda")
+        W = lib.quantize_weight(w)
+        out = torch.empty(w.numel(), dtype=torch.bfloat16, device="cuda")
+        del w
+        for _ in range(2 + args.steps):
+            lib.nf4_dequantize(W.codes, W.c8, W.s2, out.numel(), out=out)
+        torch.cuda.synchronize()
+        print(json.dumps({"case": args.case, "ok": True}))
+        return
     if args.case.startswith("quant:"):
         _, N, K = args.case.split(":")
         w = synth.weight_bf16(int(N), int(K), seed=1, device="cuda")
@@ -591,7 +615,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the 65B-shaped forward sweep")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (for profiler captures): no e2e, no NF4 stream test, no CPU baseline")
-    ap.add_argument("--case", default=None, help="profiler driver: fwd:M:N:K, bwd:M:N:K or quant:N:K")
+    ap.add_argument("--case", default=None,
+                    help="profiler driver: fwd:M:N:K, bwd:M:N:K, quant:N:K, dequant:N:K or adamw8:n")
     args = ap.parse_args()
     if args.case:
         run_case(args)
