@@ -36,7 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # tensor-core kernels of this workload, from one ncu capture of the CTA-pair
 # kernels (profiles/fused_pair_c2.md); emptied whenever those kernels change.
-NCU_TRAFFIC_BYTES = {"fused_fwd": 43.901696e6 + 3.418624e6, "fused_dx": 43.927808e6 + 3.746048e6}
+NCU_TRAFFIC_BYTES = {"fused_fwd": 43.871232e6 + 3.50336e6, "fused_dx": 43.949312e6 + 2.96576e6}
 
 
 def flops_fwd_bwd(M, N, K, r):
