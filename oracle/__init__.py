@@ -33,10 +33,12 @@ Modules:
 * :mod:`oracle.optim` — the adapter optimizer step, AdamW with 8-bit blockwise
   FP8 states (every operation one fp32 rounding: the GPU must match bit for
   bit).
+* :mod:`oracle.dropout` — LoRA dropout on the adapter input with a
+  Philox-4x32-10 mask (no CUDA path yet).
 
 Parity status per function is listed in each module header.  Every function
 here is pinned by ``tests/test_oracle_*.py`` to facts the pages or
 mathematics fix; functions whose pin is partial say so.
 """
 
-from . import numerics, nf4, linear, optim  # noqa: F401
+from . import numerics, nf4, linear, optim, dropout  # noqa: F401
