@@ -335,3 +335,67 @@ def qlora_adamw8_step(p, grad, state, lr, beta1=0.9, beta2=0.999, eps=1e-8, weig
                                   ctypes.c_void_p(ms), ctypes.c_void_p(us), state.n, lr, beta1, beta2, eps,
                                   weight_decay, int(step), _ptr(status), _stream(stream)), "qlora_adamw8_step")
     return p
+
+
+# ------------------------------------------------------------ LoRA dropout
+# (include/qlora_nf4.h: dropout on the adapter input, Philox-4x32-10 mask)
+
+_U64 = ctypes.c_uint64
+_lib.qlora_bwd_dropout_workspace_size.argtypes = [_I64, _I64, _I64, _I32]
+_lib.qlora_bwd_dropout_workspace_size.restype = _SZ
+_lib.qlora_linear_fwd_dropout.argtypes = [_P, _I64, _NF4Weight, _P, _P, _I32, ctypes.c_float, ctypes.c_float, _U64,
+                                          _P, _P, _I32, _P, _P, _SZ, _P, _P]
+_lib.qlora_linear_fwd_dropout.restype = ctypes.c_int
+_lib.qlora_linear_bwd_dropout.argtypes = [_P, _P, _P, _I64, _NF4Weight, _P, _P, _I32, ctypes.c_float, ctypes.c_float,
+                                          _U64, _P, _I32, _P, _P, _P, _SZ, _P, _P]
+_lib.qlora_linear_bwd_dropout.restype = ctypes.c_int
+
+EXPORTED = EXPORTED + ("qlora_bwd_dropout_workspace_size", "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout")
+
+
+def qlora_bwd_dropout_workspace_size(M, N, K, r):
+    return int(_lib.qlora_bwd_dropout_workspace_size(M, N, K, r))
+
+
+def qlora_linear_fwd_dropout(X, W, A, B, s, p, seed, y_dtype=DTYPE_BF16, Y=None, U=None, X_drop=None, ws=None,
+                             status=None, stream=None):
+    """Forward with dropout (probability ``p``, Philox ``seed``) on the adapter
+    input; returns ``(Y, U, X_drop)`` (keep X_drop for the backward)."""
+    M = X.shape[0]
+    N, K, r = int(W.n_out), int(W.k_in), A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32 if y_dtype == DTYPE_F32 else torch.bfloat16, device=dev)
+    if U is None:
+        U = torch.empty((M, r), dtype=torch.float32, device=dev)
+    if X_drop is None:
+        X_drop = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = torch.empty(max(qlora_fwd_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.qlora_linear_fwd_dropout(_ptr(X), M, _weight(W), _ptr(A), _ptr(B), r, float(s), float(p), int(seed),
+                                         _ptr(X_drop), _ptr(Y), y_dtype, _ptr(U), _ptr(ws), ws.numel(), _ptr(status),
+                                         _stream(stream)),
+           "qlora_linear_fwd_dropout")
+    return Y, U, X_drop
+
+
+def qlora_linear_bwd_dropout(dY, X_drop, U, W, A, B, s, p, seed, dx_dtype=DTYPE_BF16, dX=None, dA=None, dB=None,
+                             ws=None, status=None, stream=None):
+    """Backward of :func:`qlora_linear_fwd_dropout` (same ``p`` and ``seed``);
+    returns ``(dX, dA, dB)``."""
+    M = X_drop.shape[0]
+    N, K, r = int(W.n_out), int(W.k_in), A.shape[0]
+    dev = X_drop.device
+    if dX is None:
+        dX = torch.empty((M, K), dtype=torch.float32 if dx_dtype == DTYPE_F32 else torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(max(qlora_bwd_dropout_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.qlora_linear_bwd_dropout(_ptr(dY), _ptr(X_drop), _ptr(U), M, _weight(W), _ptr(A), _ptr(B), r,
+                                         float(s), float(p), int(seed), _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB),
+                                         _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
+           "qlora_linear_bwd_dropout")
+    return dX, dA, dB

@@ -195,11 +195,11 @@ qlora_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLO
 
 enum KernelId {
   kKQuantize = 0, kKDequantize, kKDown, kKFusedFwd, kKFinishFwd, kKLowFwd, kKLowFinish, kKDU, kKDB, kKFusedDX,
-  kKDA, kKAdamW8, kKCount
+  kKDA, kKAdamW8, kKDropout, kKDropoutDx, kKCount
 };
 const char* const kKernelNames[kKCount] = {
     "nf4_quantize", "nf4_dequantize", "lora_down", "fused_fwd", "finish_fwd", "lowm_fwd", "lowm_finish",
-    "lora_du", "lora_db", "fused_dx", "lora_da", "adamw8"};
+    "lora_du", "lora_db", "fused_dx", "lora_da", "adamw8", "dropout", "dropout_dx"};
 
 struct ProfRecord {
   int id;
@@ -525,15 +525,17 @@ qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float
                                          static_cast<cudaStream_t>(stream)));
 }
 
-qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
-                              int32_t r, float s, void* Y, int32_t y_dtype, float* U_out, void* ws,
-                              size_t ws_bytes, int32_t* d_status, void* stream) {
+// The forward; Xa is the adapter's input: X itself, or X after dropout.
+static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64_t M, nf4_weight W,
+                                    const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y,
+                                    int32_t y_dtype, float* U_out, void* ws, size_t ws_bytes, int32_t* d_status,
+                                    void* stream) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
-  if (!X || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;
+  if (!X || !Xa || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;
   if (qlora_status st = check_weight_ptrs(W)) return st;
-  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(U_out) ||
+  if (!aligned16(X) || !aligned16(Xa) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(U_out) ||
       (d_status && !aligned16(d_status)))
     return QLORA_ERR_ALIGN;
   const int64_t N = W.n_out, K = W.k_in;
@@ -570,21 +572,22 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
     la.mpad = p.low_mpad;
     la.status = d_status;
     la.tab = tables();
-    CUtensorMap lc, la_map, lx;
+    CUtensorMap lc, la_map, lx, lxa;
     if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, r, K, 64, kLowmARows, 128) ||
-        !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
+        !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128) ||
+        !map_bf16(&lxa, Xa, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
       return QLORA_ERR_CUDA;
     {
       ProfScope ps(kKLowFwd, cs);
-      if (qlora_status st = from_cuda(launch_lowm_fwd(lc, la_map, lx, la, cs))) return st;
+      if (qlora_status st = from_cuda(launch_lowm_fwd(lc, la_map, lx, lxa, la, cs))) return st;
     }
     ProfScope ps(kKLowFinish, cs);
     return from_cuda(launch_lowm_finish(la, cs));
   }
 
-  // U = X A^T (contraction split over a cluster), plus the bf16 hi/lo of s*U.
+  // U = Xa A^T (contraction split over a cluster), plus the bf16 hi/lo of s*U.
   CUtensorMap mx_down, ma_down;
-  if (!map_bf16(&mx_down, X, M, K, 64, 128) || !map_bf16(&ma_down, A, r, K, 64, 64)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mx_down, Xa, M, K, 64, 128) || !map_bf16(&ma_down, A, r, K, 64, 64)) return QLORA_ERR_CUDA;
   SkinnyArgs sa{};
   sa.M = static_cast<int>(M);
   sa.N = static_cast<int>(N);
@@ -661,9 +664,20 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const 
   return QLORA_OK;
 }
 
-qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
-                              const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX, int32_t dx_dtype,
-                              float* dA, float* dB, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
+                              int32_t r, float s, void* Y, int32_t y_dtype, float* U_out, void* ws,
+                              size_t ws_bytes, int32_t* d_status, void* stream) {
+  return linear_fwd_impl(X, X, M, W, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
+}
+
+// The backward; X is the adapter's input (X itself, or X after dropout, for
+// dA).  With `drop`, the GEMM's adapter stages are left out: dX's frozen-path
+// term goes to an fp32 buffer after the caller's workspace and a second pass
+// adds keep * c * (dU A) and writes dX.
+static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
+                                    const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX,
+                                    int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                    int32_t* d_status, void* stream, const DropoutArgs* drop) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
   if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
@@ -674,13 +688,18 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
     return QLORA_ERR_ALIGN;
   const int64_t N = W.n_out, K = W.k_in;
   const BwdPlan p = plan_bwd(M, N, K, r);
-  if (!ws || ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
+  const size_t need = p.total + (drop ? align256(static_cast<size_t>(M) * K * 4) : 0);
+  if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   if (qlora_status st = check_device()) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* sucat = reinterpret_cast<uint16_t*>(wsb + p.off_sucat);
   uint16_t* ducat = reinterpret_cast<uint16_t*>(wsb + p.off_ducat);
+  float* dx32 = drop ? reinterpret_cast<float*>(wsb + p.total) : nullptr;
+  void* dx_gemm = drop ? static_cast<void*>(dx32) : dX;           // where the GEMM writes
+  const int gemm_f32 = drop ? 1 : (dx_dtype == QLORA_DTYPE_F32);
+  const int gemm_r = drop ? 0 : r;                                // adapter stages in the GEMM
   const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
 
   SkinnyArgs sa{};
@@ -725,14 +744,14 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
     FusedArgs fa{};
     fa.c8 = W.c8;
     fa.s2 = W.s2;
-    fa.out = dX;
-    fa.out_f32 = dx_dtype == QLORA_DTYPE_F32;
+    fa.out = dx_gemm;
+    fa.out_f32 = gemm_f32;
     fa.ld_out = K;
     fa.M = Mi;
     fa.rows = Ki;
     fa.n_out = Ni;
     fa.k_in = Ki;
-    fa.r = r;
+    fa.r = gemm_r;
     fa.kt_total = static_cast<int>(N / 32);
     fa.kt_per_split = fa.kt_total;
     fa.status = d_status;
@@ -749,15 +768,15 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   FusedArgs fa{};
   fa.c8 = W.c8;
   fa.s2 = W.s2;
-  fa.out = dX;
-  fa.out_f32 = dx_dtype == QLORA_DTYPE_F32;
+  fa.out = dx_gemm;
+  fa.out_f32 = gemm_f32;
   fa.ld_out = K;
   fa.split_stride = 0;
   fa.M = Mi;
   fa.rows = Ki;
   fa.n_out = Ni;
   fa.k_in = Ki;
-  fa.r = r;
+  fa.r = gemm_r;
   fa.kt_total = static_cast<int>(N / 64);
   fa.kt_per_split = static_cast<int>(N / 64);
   fa.status = d_status;
@@ -766,6 +785,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
     ProfScope ps(kKFusedDX, cs);
     if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, cs))) return st;
   }
+  }
+  if (drop) {  // dX = dX_main + keep * c * (dU A), on the caller's stream after the GEMM
+    ProfScope ps(kKDropoutDx, cs);
+    if (qlora_status st = from_cuda(
+            launch_dropout_dx(dx32, ducat, A, dX, dx_dtype == QLORA_DTYPE_F32, Mi, Ki, r, *drop, cs)))
+      return st;
   }
 
   // dB = dY^T (sU)  (contraction over M split over a cluster)
@@ -801,6 +826,68 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   }
 
   return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
+                              const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX, int32_t dx_dtype,
+                              float* dA, float* dB, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  return linear_bwd_impl(dY, X, U, M, W, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream, nullptr);
+}
+
+// ------------------------------------------------------------------ LoRA dropout
+
+// Host constants of the mask: keep when the Philox word is below
+// T = floor((1 - p) 2^32) (fp64), every element for p = 0; c = fp32(1/(1-p)).
+static bool dropout_args(float p, uint64_t seed, DropoutArgs* d) {
+  if (!(p >= 0.0f && p < 1.0f)) return false;
+  const double keep = 1.0 - static_cast<double>(p);
+  const double t = std::floor(keep * 4294967296.0);
+  d->seed = seed;
+  d->keep_all = t >= 4294967296.0 ? 1 : 0;
+  d->threshold = d->keep_all ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  d->c = static_cast<float>(1.0 / keep);
+  return true;
+}
+
+size_t qlora_bwd_dropout_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+  return plan_bwd(M, N, K, r).total + align256(static_cast<size_t>(M) * K * 4);
+}
+
+qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A,
+                                      const uint16_t* B, int32_t r, float s, float p, uint64_t seed,
+                                      uint16_t* X_drop, void* Y, int32_t y_dtype, float* U_out, void* ws,
+                                      size_t ws_bytes, int32_t* d_status, void* stream) {
+  DropoutArgs d{};
+  if (!dropout_args(p, seed, &d)) return QLORA_ERR_SHAPE;
+  if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
+  if (M == 0) return QLORA_OK;
+  if (!X || !X_drop || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;
+  if (qlora_status st = check_weight_ptrs(W)) return st;
+  if (!aligned16(X) || !aligned16(X_drop) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
+      !aligned16(U_out) || (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  const FwdPlan pl = plan_fwd(M, W.n_out, W.k_in, r);
+  if (!ws || ws_bytes < pl.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  {
+    ProfScope ps(kKDropout, static_cast<cudaStream_t>(stream));
+    if (qlora_status st =
+            from_cuda(launch_dropout_apply(X, X_drop, M * W.k_in, d, static_cast<cudaStream_t>(stream))))
+      return st;
+  }
+  return linear_fwd_impl(X, X_drop, M, W, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
+}
+
+qlora_status qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X_drop, const float* U, int64_t M,
+                                      nf4_weight W, const uint16_t* A, const uint16_t* B, int32_t r, float s, float p,
+                                      uint64_t seed, void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws,
+                                      size_t ws_bytes, int32_t* d_status, void* stream) {
+  DropoutArgs d{};
+  if (!dropout_args(p, seed, &d)) return QLORA_ERR_SHAPE;
+  return linear_bwd_impl(dY, X_drop, U, M, W, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream, &d);
 }
 
 // ------------------------------------------------------------------ optimizer

@@ -1,0 +1,144 @@
+// dropout.cu — LoRA dropout on the adapter input ("Tutorial fine-tuning LLM
+// LoRA/QLoRA 2026", nexusinovation, section "Mão na Massa": the adapter
+// configuration's lora_dropout).  The frozen path sees X, the adapter sees
+// X_drop; the backward's dropout derivative is keep * c.
+//
+// Mask: Philox-4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011), key (seed mod 2^32, seed div 2^32),
+// counter (g mod 2^32, g div 2^32, 0, 0) for the group g of four consecutive
+// elements of the flattened [M, K] tensor; word i of the call decides element
+// 4g + i, kept when the word is below T = floor((1 - p) 2^32).  A kept element
+// is bf16(RN32(x * c)) with c = fp32(1 / (1 - p)), a dropped one +0.
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace qnf4 {
+
+namespace {
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 ctr, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t lo0 = 0xD2511F53u * ctr.x, hi0 = __umulhi(0xD2511F53u, ctr.x);
+    const uint32_t lo1 = 0xCD9E8D57u * ctr.z, hi1 = __umulhi(0xCD9E8D57u, ctr.z);
+    ctr = make_uint4(hi1 ^ ctr.y ^ k0, lo1, hi0 ^ ctr.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;  // the bump after the last round is never used
+    k1 += 0xBB67AE85u;
+  }
+  return ctr;
+}
+
+// Bit i set when element 4g + i is kept.
+__device__ __forceinline__ uint32_t keep4(uint64_t g, const DropoutArgs& d) {
+  if (d.keep_all) return 0xFu;
+  const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), 0u, 0u),
+                                static_cast<uint32_t>(d.seed), static_cast<uint32_t>(d.seed >> 32));
+  return (w.x < d.threshold ? 1u : 0u) | (w.y < d.threshold ? 2u : 0u) | (w.z < d.threshold ? 4u : 0u) |
+         (w.w < d.threshold ? 8u : 0u);
+}
+
+__device__ __forceinline__ uint32_t drop_pair(uint32_t xx, uint32_t keep2, float c) {
+  const uint32_t lo = (keep2 & 1u) ? bf16_bits(__fmul_rn(bf16_bits_to_float(xx & 0xFFFFu), c)) : 0u;
+  const uint32_t hi = (keep2 & 2u) ? bf16_bits(__fmul_rn(bf16_bits_to_float(xx >> 16), c)) : 0u;
+  return lo | (hi << 16);
+}
+
+// X_drop = dropout(X): one Philox call per group of four elements, 8-byte
+// loads and stores, grid-stride.
+__global__ void __launch_bounds__(256) dropout_apply_kernel(const uint16_t* __restrict__ X, uint16_t* __restrict__ Xd,
+                                                            int64_t groups, const DropoutArgs d) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint2 x = *reinterpret_cast<const uint2*>(X + 4 * g);
+    const uint32_t k = keep4(static_cast<uint64_t>(g), d);
+    *reinterpret_cast<uint2*>(Xd + 4 * g) = make_uint2(drop_pair(x.x, k, d.c), drop_pair(x.y, k >> 2, d.c));
+  }
+}
+
+// dX = dX_main + keep * c * (dU A), dX_main fp32 [M, K] from the GEMM without
+// its adapter stages, dU from the bf16 hi/lo pairs of the interleaved layout
+// (column c holds part (c/16)%2 of j = 16 floor(c/32) + c%16), A bf16 [r, K].
+// A CTA computes a 64 x 64 block of (m, k) on the CUDA cores (r <= 64 terms,
+// fp32); each thread a 4 x 4 micro-block whose four k form one mask group.
+constexpr int kDxTile = 64;
+
+__global__ void __launch_bounds__(256) dropout_dx_kernel(const float* __restrict__ dx32,
+                                                         const uint16_t* __restrict__ ducat,
+                                                         const uint16_t* __restrict__ A, void* __restrict__ out,
+                                                         int out_f32, int M, int K, int r, const DropoutArgs d) {
+  __shared__ float su[kDxTile][kDxTile + 1];  // [m][j]
+  __shared__ float sa[kDxTile][kDxTile];      // [j][k]
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * kDxTile, k0 = blockIdx.x * kDxTile;
+  grid_dependency_wait();
+  grid_dependents_launch();
+  for (int e = tid; e < kDxTile * kDxTile; e += 256) {
+    const int mm = e / kDxTile, j = e % kDxTile;
+    float v = 0.0f;
+    if (m0 + mm < M && j < r) {
+      const uint16_t* row = ducat + static_cast<int64_t>(m0 + mm) * 2 * r;
+      const int col = 32 * (j >> 4) + (j & 15);
+      v = __fadd_rn(bf16_bits_to_float(row[col]), bf16_bits_to_float(row[col + 16]));
+    }
+    su[mm][j] = v;
+    const int jj = e / kDxTile, kk = e % kDxTile;
+    sa[jj][kk] = jj < r ? bf16_bits_to_float(A[static_cast<int64_t>(jj) * K + k0 + kk]) : 0.0f;
+  }
+  __syncthreads();
+  float acc[4][4] = {};
+  for (int j = 0; j < r; ++j) {
+    float av[4], uv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      av[i] = sa[j][4 * tx + i];
+      uv[i] = su[4 * ty + i][j];
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(uv[a], av[b], acc[a][b]);
+  }
+  const int k = k0 + 4 * tx;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int m = m0 + 4 * ty + a;
+    if (m >= M) continue;
+    const int64_t e = static_cast<int64_t>(m) * K + k;  // a multiple of 4: one mask group
+    const uint32_t keep = keep4(static_cast<uint64_t>(e >> 2), d);
+    const float4 base = *reinterpret_cast<const float4*>(dx32 + e);
+    const float bv[4] = {base.x, base.y, base.z, base.w};
+    float v[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v[b] = (keep >> b) & 1u ? __fadd_rn(bv[b], __fmul_rn(d.c, acc[a][b])) : bv[b];
+    if (out_f32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+      const uint32_t lo = static_cast<uint32_t>(bf16_bits(v[0])) | (static_cast<uint32_t>(bf16_bits(v[1])) << 16);
+      const uint32_t hi = static_cast<uint32_t>(bf16_bits(v[2])) | (static_cast<uint32_t>(bf16_bits(v[3])) << 16);
+      *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + e) = make_uint2(lo, hi);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dropout_apply(const uint16_t* X, uint16_t* Xd, int64_t count, const DropoutArgs& d,
+                                 cudaStream_t stream) {
+  if (count % 4 != 0) return cudaErrorInvalidValue;
+  const int64_t groups = count / 4;
+  const int64_t ctas = std::min<int64_t>((groups + 255) / 256, 148 * 16);
+  return launch_kernel(dropout_apply_kernel, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, stream,
+                       dim3(1, 1, 1), X, Xd, groups, d);
+}
+
+cudaError_t launch_dropout_dx(const float* dx32, const uint16_t* ducat, const uint16_t* A, void* out, int out_f32,
+                              int M, int K, int r, const DropoutArgs& d, cudaStream_t stream) {
+  if (K % kDxTile != 0 || r > kDxTile) return cudaErrorInvalidValue;
+  return launch_kernel(dropout_dx_kernel, dim3(K / kDxTile, (M + kDxTile - 1) / kDxTile), dim3(256), 0, stream,
+                       dim3(1, 1, 1), dx32, ducat, A, out, out_f32, M, K, r, d);
+}
+
+}  // namespace qnf4

@@ -76,6 +76,21 @@ struct SkinnyArgs {
   int32_t* status;
 };
 
+// LoRA dropout on the adapter input (dropout.cu).
+struct DropoutArgs {
+  uint64_t seed;        // Philox key: (seed mod 2^32, seed div 2^32)
+  uint32_t threshold;   // keep when the 32-bit word is below this
+  int keep_all;         // p = 0: every element kept
+  float c;              // fp32(1 / (1 - p))
+};
+//   X_drop = dropout(X) over `count` elements (a multiple of 4).
+cudaError_t launch_dropout_apply(const uint16_t* X, uint16_t* Xd, int64_t count, const DropoutArgs& d,
+                                 cudaStream_t stream);
+//   out = dx32 + keep * c * (dU A): dx32 fp32 [M, K], dU as the bf16 hi/lo pairs
+//   of the interleaved [M, 2r] layout, A bf16 [r, K]; K % 64 == 0, r <= 64.
+cudaError_t launch_dropout_dx(const float* dx32, const uint16_t* ducat, const uint16_t* A, void* out, int out_f32,
+                              int M, int K, int r, const DropoutArgs& d, cudaStream_t stream);
+
 // AdamW step with 8-bit states (optim.cu).
 struct AdamW8Args {
   uint16_t* p;       // [n] bf16 parameters, in place
@@ -164,9 +179,10 @@ struct LowmArgs {
 };
 
 //   tm_codes: codes [N, K/2] u8 box {128, 128} SW128; tm_a: A [r, K] bf16
-//   box {64, 32} SW128; tm_x: X [M, K] bf16 box {64, mpad} SW128.
+//   box {64, 32} SW128; tm_x: X [M, K] bf16 box {64, mpad} SW128; tm_xa: the
+//   adapter's input (X, or X after dropout) with the same box.
 cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                            const LowmArgs& a, cudaStream_t stream);
+                            const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream);
 cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream);
 
 // Fixed-order sum of the small-M forward's split-K partials of Y.

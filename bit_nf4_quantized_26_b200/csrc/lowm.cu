@@ -118,7 +118,8 @@ __device__ __forceinline__ void load_consts(const LowmArgs& a, int tile, int kci
 // stage i % kStages once the eight warps have released its previous use.
 template <int NT>
 __device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_a,
-                                           const CUtensorMap* tm_x, const LowmArgs& a, uint8_t* smem,
+                                           const CUtensorMap* tm_x, const CUtensorMap* tm_xa, const LowmArgs& a,
+                                           uint8_t* smem,
                                            uint64_t* full, uint64_t* empty, int i, int tile, int kci,
                                            const WaitCtx& wc) {
   using P = LowmPlan<NT>;
@@ -133,15 +134,18 @@ __device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CU
     for (int b = 0; b < 4; ++b)
       tma_load_2d(st + b * kLowmABox, tm_a, &full[s], kci * 256 + b * 64, (tile - a.tiles) * kLowmARows);
   }
+  // W tiles multiply X; the adapter's A tiles multiply its input (X, or X after dropout).
+  const CUtensorMap* tx = tile < a.tiles ? tm_x : tm_xa;
 #pragma unroll
-  for (int b = 0; b < 4; ++b) tma_load_2d(st + kLowmCodes + b * P::kXBox, tm_x, &full[s], kci * 256 + b * 64, 0);
+  for (int b = 0; b < 4; ++b) tma_load_2d(st + kLowmCodes + b * P::kXBox, tx, &full[s], kci * 256 + b * 64, 0);
   return true;
 }
 
 template <int NT>
 __global__ void __launch_bounds__(kLowmThreads, 2)
     lowm_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_a,
-                    const __grid_constant__ CUtensorMap tm_x, const LowmArgs a) {
+                    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xa,
+                    const LowmArgs a) {
   using P = LowmPlan<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -167,6 +171,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_xa);
   }
   __syncthreads();
   const WaitCtx wc{abort_flag, a.status};
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   int issued = 0, itile = tile0, ikci = kci0;
   bool ok = true;
   auto issue_next = [&]() {
-    ok = lowm_issue<NT>(&tm_codes, &tm_a, &tm_x, a, smem, full, empty, issued, itile, ikci, wc);
+    ok = lowm_issue<NT>(&tm_codes, &tm_a, &tm_x, &tm_xa, a, smem, full, empty, issued, itile, ikci, wc);
     if (ok) {
       ++issued;
       if (++ikci == a.kc) {
@@ -396,7 +401,7 @@ __global__ void __launch_bounds__(512) lowm_finish_kernel(const LowmArgs a) {
 
 template <int NT>
 static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                                    const LowmArgs& a, cudaStream_t stream) {
+                                    const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream) {
   static bool attr_set = false;  // benign race: setting the same value twice is harmless
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(lowm_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -405,17 +410,17 @@ static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorM
     attr_set = true;
   }
   return launch_kernel(lowm_fwd_kernel<NT>, dim3(a.ctas), dim3(kLowmThreads), LowmPlan<NT>::kSmem, stream,
-                       dim3(1, 1, 1), tm_codes, tm_a, tm_x, a);
+                       dim3(1, 1, 1), tm_codes, tm_a, tm_x, tm_xa, a);
 }
 
 }  // namespace
 
 cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                            const LowmArgs& a, cudaStream_t stream) {
+                            const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream) {
   switch (a.mpad) {
-    case 8: return launch_lowm_impl<1>(tm_codes, tm_a, tm_x, a, stream);
-    case 16: return launch_lowm_impl<2>(tm_codes, tm_a, tm_x, a, stream);
-    case 32: return launch_lowm_impl<4>(tm_codes, tm_a, tm_x, a, stream);
+    case 8: return launch_lowm_impl<1>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
+    case 16: return launch_lowm_impl<2>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
+    case 32: return launch_lowm_impl<4>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

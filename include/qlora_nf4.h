@@ -167,6 +167,41 @@ QLORA_API size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32
 QLORA_API size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
 
 /*
+ * LoRA dropout on the adapter input ("Tutorial fine-tuning LLM LoRA/QLoRA
+ * 2026", "Mão na Massa": the adapter configuration's lora_dropout; where it
+ * acts is this library's reading).  The frozen path sees X, the adapter sees
+ * X_drop:
+ *
+ *   forward:   X_drop = dropout(X);  U = X_drop A^T;  Y = X W'^T + s U B^T
+ *   backward:  dU = s dY B;  dX = dY W' + keep * c * (dU A);
+ *              dA = dU^T X_drop;  dB = s dY^T U
+ *
+ * Mask: Philox-4x32-10 (Salmon et al., SC 2011) with key (seed mod 2^32,
+ * seed div 2^32) and counter (g mod 2^32, g div 2^32, 0, 0) for the group g of
+ * four consecutive elements of the flattened [M, K] X; word i decides element
+ * 4g + i, kept when below T = floor((1 - p) 2^32) (all kept for p = 0).  A kept
+ * element is bf16(RN32(x * c)) with c = fp32(1 / (1 - p)), a dropped one +0.
+ *
+ * qlora_linear_fwd_dropout writes X_drop [M, K] bf16 (caller-owned; keep it for
+ * the backward) and then runs the forward with X_drop as the adapter's input;
+ * its workspace is qlora_fwd_workspace_size.  qlora_linear_bwd_dropout takes
+ * X_drop (X itself is not needed) and the same p and seed, and needs
+ * qlora_bwd_dropout_workspace_size bytes (the plain backward's plus an fp32
+ * [M, K] buffer for dX's frozen-path term).  0 <= p < 1, else QLORA_ERR_SHAPE;
+ * everything else as for qlora_linear_fwd / qlora_linear_bwd.
+ */
+QLORA_API size_t qlora_bwd_dropout_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
+QLORA_API qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A,
+                                                const uint16_t* B, int32_t r, float s, float p, uint64_t seed,
+                                                uint16_t* X_drop, void* Y, int32_t y_dtype, float* U_out, void* ws,
+                                                size_t ws_bytes, int32_t* d_status, void* stream);
+QLORA_API qlora_status qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X_drop, const float* U,
+                                                int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
+                                                int32_t r, float s, float p, uint64_t seed, void* dX,
+                                                int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                                int32_t* d_status, void* stream);
+
+/*
  * qlora_linear_fwd_noalloc — the forward of qlora_linear_fwd for callers that
  * cannot provide a workspace.  The pages have no counterpart; it exists for
  * callers that may not allocate device memory at call time: a plugin that a

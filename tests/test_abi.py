@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 16
+    assert len(names) == 19
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -148,3 +148,19 @@ def test_paged_calls_reject_null_pointers():
     assert q._lib.qlora_paged_alloc(None, 16) == NULL
     assert q._lib.qlora_paged_prefetch(None, 16, 0, None) == NULL
     assert q._lib.qlora_paged_free(None) == OK
+
+
+def test_dropout_rejects_bad_probability_before_touching_a_device():
+    f = q._lib.qlora_linear_fwd_dropout
+    P = ctypes.c_void_p
+    w = q._NF4Weight(256, 256, 256, 4096, 4096)
+    for p in (-0.1, 1.0, float("nan")):
+        assert f(P(256), 64, w, P(256), P(256), 16, 1.0, p, 7, P(256), P(256), 0, P(256), P(256), 1 << 20,
+                 None, None) == SHAPE
+    g = q._lib.qlora_linear_bwd_dropout
+    assert g(P(256), P(256), P(256), 64, w, P(256), P(256), 16, 1.0, 1.5, 7, P(256), 0, P(256), P(256), P(256),
+             1 << 20, None, None) == SHAPE
+    assert f(P(256), 64, w, P(256), P(256), 16, 1.0, 0.1, 7, None, P(256), 0, P(256), P(256), 1 << 20,
+             None, None) == NULL
+    assert q.qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) == \
+        q.qlora_bwd_workspace_size(4096, 4096, 4096, 64) + 4096 * 4096 * 4
