@@ -438,6 +438,7 @@ def run_ours(args, rank, world):
 
     # ------------------------------------------- adapter optimizer step
     adamw = adamw8_timing(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
+    drop = dropout_timing(lib, synth, torch, dev, flush) if (rank == 0 and not args.no_sweep) else None
 
     # ------------------------------------------- 65B-shaped forward sweep
     c5 = c5_forward_sweep(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
@@ -505,10 +506,51 @@ def run_ours(args, rank, world):
             "c5_forward": c5,
             "c1_graph": c1g,
             "adamw8": adamw,
+            "lora_dropout": drop,
             "nf4_hbm_frac": {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
                              "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
         }
         print(json.dumps(line), flush=True)
+
+
+def dropout_timing(lib, synth, torch, dev, flush, p=0.05, reps=10):
+    """The c2 forward + backward with LoRA dropout (p = 0.05, the tutorial's
+    lora_dropout) against the same step without it; L2 flushed before each."""
+    import statistics
+    M = N = K = 4096
+    r, s = 64, 0.25
+    d = {k: v.to(dev) for k, v in synth.linear_inputs(synth.Linear("c2", N, K), M, r, 0).items()}
+    W = lib.quantize_weight(d["W"])
+    fws = torch.empty(lib.qlora_fwd_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
+    bws = torch.empty(lib.qlora_bwd_dropout_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
+    Y, U, Xd = lib.qlora_linear_fwd_dropout(d["X"], W, d["A"], d["B"], s, p, 1, ws=fws)
+    dX, dA, dB = lib.qlora_linear_bwd_dropout(d["dY"], Xd, U, W, d["A"], d["B"], s, p, 1, ws=bws)
+
+    def with_dropout(i):
+        lib.qlora_linear_fwd_dropout(d["X"], W, d["A"], d["B"], s, p, i, Y=Y, U=U, X_drop=Xd, ws=fws)
+        lib.qlora_linear_bwd_dropout(d["dY"], Xd, U, W, d["A"], d["B"], s, p, i, dX=dX, dA=dA, dB=dB, ws=bws)
+
+    def plain(i):
+        lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], s, Y=Y, U=U, ws=fws)
+        lib.qlora_linear_bwd(d["dY"], d["X"], U, W, d["A"], d["B"], s, dX=dX, dA=dA, dB=dB, ws=bws)
+
+    out = {"p": p, "workload": "c2 (4096x4096, 4x1024 tokens, r=64): forward + backward"}
+    fl = flops_fwd_bwd(M, N, K, r)
+    for name, fn in (("dropout", with_dropout), ("plain", plain)):
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(i + 1)
+            e1.record()
+            e1.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        out[name] = {"us": ms * 1e3, "tflops": fl / (ms * 1e-3) / 1e12}
+    out["overhead"] = out["dropout"]["us"] / out["plain"]["us"] - 1.0
+    return out
 
 
 def adamw8_timing(lib, synth, torch, dev, flush, peaks, layers=10, reps=10):
