@@ -34,11 +34,14 @@ Modules:
   FP8 states (every operation one fp32 rounding: the GPU must match bit for
   bit).
 * :mod:`oracle.dropout` — LoRA dropout on the adapter input with a
-  Philox-4x32-10 mask (no CUDA path yet).
+  Philox-4x32-10 mask (the GPU must match X_drop bit for bit and the
+  products within the GEMM tolerances).
+* :mod:`oracle.dq_centered` — double quantisation with mean centring, for an
+  error ablation against the plain scheme (no CUDA path).
 
 Parity status per function is listed in each module header.  Every function
 here is pinned by ``tests/test_oracle_*.py`` to facts the pages or
 mathematics fix; functions whose pin is partial say so.
 """
 
-from . import numerics, nf4, linear, optim, dropout  # noqa: F401
+from . import numerics, nf4, linear, optim, dropout, dq_centered  # noqa: F401

@@ -1,0 +1,75 @@
+"""Double quantisation with mean centring (a variant of the constants'
+encoding, for an error ablation against the plain scheme).
+
+TEST INFRASTRUCTURE ONLY (see the package header).  No CUDA path uses it
+yet; this module fixes what one must compute.
+
+The pages describe double quantisation as "the quantisation constants are
+themselves quantised to FP8 in blocks of 256" ("QLoRA" encyclopedia entry,
+tonho.wtf, section "como funciona") and say nothing of centring; the
+original QLoRA paper (outside the pages) subtracts the mean of the constants
+first, because they are all positive and a symmetric FP8 grid would waste
+its sign.  Readings taken here:
+
+* one mean per tensor: mean = fp32(S / n) for the n block constants c_i,
+  where S is summed in fp64 in a fixed order — sequentially within each group
+  of 256 constants, then sequentially over the group sums — so a parallel
+  implementation can reproduce it exactly;
+* per group: c' = RN32(c - mean); s2 = RN32(max|c'| / 448);
+  c8 = E4M3_RNE_satfinite(RN32(c' / s2)) (0 when s2 = 0);
+* dequantised constant: c_hat = RN32(RN32(e4m3(c8) * s2) + mean).
+
+The 4-bit codes are unchanged (they come from the exact constants).
+
+Parity status: pinned (constant constants reconstruct exactly; the fixed-
+order mean against an exact rational mean within one fp32 rounding; the
+reconstruction error within the E4M3 half-step bound per group; the plain
+scheme's error bound recovered when the mean is forced to zero).
+"""
+
+import numpy as np
+
+from .nf4 import GROUP, FP8_MAX
+from .numerics import e4m3_decode, e4m3_encode
+
+
+def constants_mean(c):
+    """fp32 mean of the block constants, summed in fp64 in the fixed order
+    (sequential within groups of 256, then sequential over the groups)."""
+    c = np.asarray(c, dtype=np.float32).astype(np.float64)
+    n = c.size
+    ng = -(-n // GROUP)
+    pad = np.zeros(ng * GROUP, dtype=np.float64)
+    pad[:n] = c
+    group_sums = np.cumsum(pad.reshape(ng, GROUP), axis=1)[:, -1]   # sequential within a group
+    total = np.cumsum(group_sums)[-1]                                # sequential over groups
+    return np.float32(total / n)
+
+
+def double_quantize_centered(c, mean=None):
+    """(c8, s2, mean) for the block constants ``c``; ``mean`` overrides the
+    tensor mean (used by the pins)."""
+    c = np.asarray(c, dtype=np.float32)
+    mean = constants_mean(c) if mean is None else np.float32(mean)
+    n = c.size
+    ng = -(-n // GROUP)
+    cp = np.zeros(ng * GROUP, dtype=np.float32)
+    cp[:n] = (c - mean).astype(np.float32)
+    cg = cp.reshape(ng, GROUP)
+    # padding entries of a short last group are 0 after centring: they cannot
+    # raise the group's maximum
+    amax = np.max(np.abs(cg), axis=1).astype(np.float32)
+    s2 = (amax / np.float32(FP8_MAX)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = (cg / s2[:, None]).astype(np.float32)
+    y[s2 == 0] = 0.0
+    c8 = e4m3_encode(y).reshape(-1)[:n]
+    return c8, s2, mean
+
+
+def dequantized_constants_centered(c8, s2, mean):
+    """c_hat = RN32(RN32(e4m3(c8) * s2[group]) + mean)."""
+    c8 = np.asarray(c8, dtype=np.uint8)
+    s2 = np.asarray(s2, dtype=np.float32)
+    g = np.arange(c8.size) // GROUP
+    return ((e4m3_decode(c8) * s2[g]).astype(np.float32) + np.float32(mean)).astype(np.float32)

@@ -1,7 +1,6 @@
 """LoRA dropout on the adapter input, with a counter-based mask.
 
-TEST INFRASTRUCTURE ONLY (see the package header).  The CUDA path of this
-row is not built yet; this module fixes what it must compute.
+TEST INFRASTRUCTURE ONLY (see the package header).
 
 Source: "Tutorial fine-tuning LLM LoRA/QLoRA 2026" (nexusinovation), section
 "Mão na Massa": the adapter configuration sets ``lora_dropout=0.05``.  The

@@ -1,0 +1,71 @@
+"""Pins for oracle.dq_centered (double quantisation with mean centring) and
+the error ablation against the plain scheme."""
+
+from fractions import Fraction
+
+import numpy as np
+
+import synth
+from oracle import dq_centered as dqc
+from oracle import nf4
+from oracle import numerics as nm
+
+
+def _constants(n_out, k_in, seed):
+    w = synth.bf16_bits(synth.weight_bf16(n_out, k_in, seed=seed))
+    return nf4.absmax_constants(w.reshape(-1), w.size)
+
+
+def test_constant_constants_reconstruct_exactly():
+    """All constants equal: the mean is that value, every centred constant is
+    0, s2 = 0, and c_hat = mean = c exactly."""
+    c = np.full(1000, np.float32(0.0371), dtype=np.float32)
+    c8, s2, mean = dqc.double_quantize_centered(c)
+    assert mean == c[0] and not c8.any() and not s2.any()
+    assert np.array_equal(dqc.dequantized_constants_centered(c8, s2, mean), c)
+
+
+def test_mean_is_the_exact_mean_within_one_rounding():
+    """The fixed-order fp64 sum of a few thousand fp32 constants is exact
+    enough that the fp32 mean is the exact rational mean rounded once (or
+    its neighbour when the exact mean lies within fp64 noise of a tie)."""
+    c = _constants(64, 4096, 3)
+    exact = sum(Fraction(float(x)) for x in c) / c.size
+    got = dqc.constants_mean(c)
+    lo = np.nextafter(got, np.float32(-np.inf))
+    hi = np.nextafter(got, np.float32(np.inf))
+    assert Fraction(float(lo)) < exact < Fraction(float(hi))
+
+
+def test_reconstruction_within_e4m3_half_step():
+    """|c_hat - c| <= (half an E4M3 step at the group's scale) plus the two
+    fp32 roundings, group by group."""
+    c = _constants(256, 4096, 4)
+    c8, s2, mean = dqc.double_quantize_centered(c)
+    ch = dqc.dequantized_constants_centered(c8, s2, mean).astype(np.float64)
+    g = np.arange(c.size) // nf4.GROUP
+    # E4M3 relative step is 2^-3 for normals; half of it, times the largest
+    # magnitude 448 * s2 of the group, bounds the error of every member
+    bound = 0.5 * 2.0 ** -3 * 448.0 * s2[g].astype(np.float64) + 2 * np.abs(ch) * 2.0 ** -24
+    assert np.all(np.abs(ch - c.astype(np.float64)) <= bound)
+
+
+def test_zero_mean_matches_plain_double_quantisation():
+    """Forcing the mean to 0 gives the plain scheme's codes and scales."""
+    c = _constants(128, 2048, 5)
+    c8, s2, _ = dqc.double_quantize_centered(c, mean=0.0)
+    p8, ps2 = nf4.double_quantize(c)
+    assert np.array_equal(c8, p8) and np.array_equal(s2.view(np.uint32), ps2.view(np.uint32))
+
+
+def test_centring_lowers_the_constant_error_on_normal_weights():
+    """The ablation: on N(0, 0.02) weights the centred constants are closer
+    to the exact ones than the plain FP8 constants (RMS relative error)."""
+    c = _constants(1024, 4096, 6).astype(np.float64)
+    p8, ps2 = nf4.double_quantize(c.astype(np.float32))
+    plain = nf4.dequantized_constants(p8, ps2).astype(np.float64)
+    c8, s2, mean = dqc.double_quantize_centered(c.astype(np.float32))
+    cent = dqc.dequantized_constants_centered(c8, s2, mean).astype(np.float64)
+    e_plain = np.sqrt(np.mean(((plain - c) / c) ** 2))
+    e_cent = np.sqrt(np.mean(((cent - c) / c) ** 2))
+    assert e_cent < e_plain
