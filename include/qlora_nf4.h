@@ -24,6 +24,9 @@
  *              dA = dU^T X                dB = s dY^T U
  *
  * where W' = dequantize(NF4(W)) in bf16.  There is no dW (the base is frozen).
+ * The same calls with LoRA dropout on the adapter input are declared below
+ * (qlora_linear_{fwd,bwd}_dropout); the adapter optimizer step is in
+ * qlora_optim.h.
  *
  * NF4 storage of a tensor of `numel` elements (flattened row-major):
  *   codes  uint8[ceil(numel/64)*32]  two 4-bit codes per byte; element 2j in
