@@ -399,3 +399,16 @@ def qlora_linear_bwd_dropout(dY, X_drop, U, W, A, B, s, p, seed, dx_dtype=DTYPE_
                                          _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
            "qlora_linear_bwd_dropout")
     return dX, dA, dB
+
+
+# ------------------------------------------------------ bounded-wait self-test
+
+_lib.qlora_selftest_timeout.argtypes = [_P, _I64, _P]
+_lib.qlora_selftest_timeout.restype = ctypes.c_int
+EXPORTED = EXPORTED + ("qlora_selftest_timeout",)
+
+
+def qlora_selftest_timeout(status, limit_ns, stream=None):
+    """Run the kernels' bounded wait against a barrier nothing completes, with
+    a ``limit_ns`` limit; sets DEV_TIMEOUT in the int32 device tensor ``status``."""
+    _check(_lib.qlora_selftest_timeout(_ptr(status), int(limit_ns), _stream(stream)), "qlora_selftest_timeout")

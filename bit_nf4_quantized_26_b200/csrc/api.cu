@@ -834,6 +834,14 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   return linear_bwd_impl(dY, X, U, M, W, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream, nullptr);
 }
 
+qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_ns, void* stream) {
+  if (!d_status) return QLORA_ERR_NULL;
+  if (limit_ns < 1000 || limit_ns > 2000000000) return QLORA_ERR_SHAPE;
+  if (!aligned16(d_status)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  return from_cuda(launch_selftest_timeout(d_status, static_cast<uint64_t>(limit_ns), static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------------------ LoRA dropout
 
 // Host constants of the mask: keep when the Philox word is below

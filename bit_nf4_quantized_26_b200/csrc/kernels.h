@@ -76,6 +76,10 @@ struct SkinnyArgs {
   int32_t* status;
 };
 
+// One CTA waits on an mbarrier nothing completes, with a `limit_ns` bound,
+// then reports QLORA_DEV_TIMEOUT (quant.cu; diagnostics).
+cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
+
 // LoRA dropout on the adapter input (dropout.cu).
 struct DropoutArgs {
   uint64_t seed;        // Philox key: (seed mod 2^32, seed div 2^32)

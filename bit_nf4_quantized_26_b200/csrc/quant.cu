@@ -239,4 +239,32 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const
                        dim3(1, 1, 1), tm_out ? *tm_out : none, tm_out ? 1 : 0, codes, c8, s2, numel, out, tab);
 }
 
+// ------------------------------------------------------- bounded-wait self-test
+//
+// The wait below is the kernels' bounded wait (try_wait on the barrier's
+// phase, %globaltimer deadline) with a caller-chosen limit; the barrier
+// expects one arrival that never comes, so the limit always passes.
+__global__ void selftest_timeout_kernel(int32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicOr(status, QLORA_DEV_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
+cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream) {
+  selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 }  // namespace qnf4

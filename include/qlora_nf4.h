@@ -256,6 +256,17 @@ QLORA_API void qlora_profile_enable(int32_t enable);
 QLORA_API int32_t qlora_profile_collect(int32_t* kernel_ids, float* ms, int32_t capacity);
 QLORA_API const char* qlora_kernel_name(int32_t kernel_id);
 
+/*
+ * qlora_selftest_timeout — exercises the bounded-wait path every kernel uses
+ * (diagnostics).  Launches one CTA whose thread waits on a shared-memory
+ * mbarrier that nothing completes, polling it with the kernels' bounded wait
+ * but a time limit of `limit_ns` nanoseconds (1e3 .. 2e9) instead of the
+ * kernels' 2 s; when the limit passes it ORs QLORA_DEV_TIMEOUT into
+ * *d_status (required) and returns, leaving the context usable.  Nothing
+ * faults, traps or hangs.  limit_ns out of range returns QLORA_ERR_SHAPE.
+ */
+QLORA_API qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_ns, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 QLORA_API const char* qlora_strerror(qlora_status status);
 

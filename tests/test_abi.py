@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 19
+    assert len(names) == 20
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -164,3 +164,12 @@ def test_dropout_rejects_bad_probability_before_touching_a_device():
              None, None) == NULL
     assert q.qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) == \
         q.qlora_bwd_workspace_size(4096, 4096, 4096, 64) + 4096 * 4096 * 4
+
+
+def test_selftest_timeout_argument_checks():
+    f = q._lib.qlora_selftest_timeout
+    P = ctypes.c_void_p
+    assert f(None, 5_000_000, None) == NULL
+    assert f(P(256), 10, None) == SHAPE
+    assert f(P(256), 3_000_000_000, None) == SHAPE
+    assert f(P(260), 5_000_000, None) == ALIGN
