@@ -35,7 +35,7 @@ WORKLOAD_NAME = "LLaMA-7B attention projection: W 4096x4096 NF4/64 + FP8/256, 4x
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # tensor-core kernels of this workload, from one ncu capture of the CTA-pair
-# kernels (profiles/fused_pair_c2.md); emptied whenever those kernels change.
+# kernels on this workload (c2 forward and dX); emptied whenever those kernels change.
 NCU_TRAFFIC_BYTES = {"fused_fwd": 43.871232e6 + 3.50336e6, "fused_dx": 43.949312e6 + 2.96576e6}
 
 
