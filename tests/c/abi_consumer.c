@@ -64,6 +64,18 @@ int main(void) {
         QLORA_ERR_NULL);
   CHECK(qlora_adamw8_step(odd, p, p, p, p, p, 10, 1e-3f, 0.9f, 0.999f, 1e-8f, 0.0f, 1, NULL, NULL) ==
         QLORA_ERR_ALIGN);
+  /* LoRA dropout: p outside [0, 1) and a missing X_drop are rejected first. */
+  CHECK(qlora_linear_fwd_dropout(p, 64, w, p, p, 16, 1.0f, 1.0f, 7u, p, p, QLORA_DTYPE_BF16, p, p, 1u << 20, NULL,
+                                 NULL) == QLORA_ERR_SHAPE);
+  CHECK(qlora_linear_fwd_dropout(p, 64, w, p, p, 16, 1.0f, 0.05f, 7u, NULL, p, QLORA_DTYPE_BF16, p, p, 1u << 20,
+                                 NULL, NULL) == QLORA_ERR_NULL);
+  CHECK(qlora_linear_bwd_dropout(p, p, p, 64, w, p, p, 16, 1.0f, -0.5f, 7u, p, QLORA_DTYPE_BF16, p, p, p, 1u << 20,
+                                 NULL, NULL) == QLORA_ERR_SHAPE);
+  CHECK(qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) ==
+        qlora_bwd_workspace_size(4096, 4096, 4096, 64) + (size_t)4096 * 4096 * 4);
+  /* Bounded-wait self-test: argument checks only (no device here). */
+  CHECK(qlora_selftest_timeout(NULL, 5000000, NULL) == QLORA_ERR_NULL);
+  CHECK(qlora_selftest_timeout(p, 10, NULL) == QLORA_ERR_SHAPE);
   CHECK(qlora_paged_alloc(NULL, 16) == QLORA_ERR_NULL);
   CHECK(qlora_paged_free(NULL) == QLORA_OK);
   printf("c abi consumer ok\n");
