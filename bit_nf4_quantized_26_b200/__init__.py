@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m bit_nf4_quantized_26_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python bit_nf4_quantized_26_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
