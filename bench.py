@@ -1,16 +1,28 @@
 #!/usr/bin/env python
 """Benchmark of the QLoRA NF4 linear hot path on B200.
 
-One step = NF4 quantisation of the frozen weight (absmax per 64, FP8 double
-quantisation per 256) + forward (U = X A^T; Y = X W'^T + s U B^T with W'
-dequantised inside the GEMM) + backward (dU, dB, dX, dA), all through the
-library's C ABI, on the LLaMA-7B-shaped attention projection: W 4096x4096,
-4 x 1024 tokens, LoRA r=64, alpha=16, synthetic seeded inputs.
+Headline workload: the seven linears of a LLaMA-7B-shaped decoder layer
+(q, k, v, o 4096x4096; gate, up 4096->11008; down 11008->4096), every weight
+NF4 with FP8 double quantisation, LoRA r=64 alpha=16 on all seven,
+8 x 2048 = 16384 tokens per GPU, synthetic seeded inputs.  One step, all
+through the library's C ABI:
 
-value = algorithmic fwd+bwd FLOPs (4MNK + 6MKr + 6MNr) / device time per
-step, summed over all ranks (each rank runs its own batch: weak scaling; the
-adapter gradients dA, dB are summed across ranks with NCCL, the one exchange
-of data-parallel training).
+  * NF4 quantisation of the seven frozen bf16 weights (absmax per 64, FP8
+    double quantisation per 256);
+  * forward of every linear in layer order: U = X A^T, Y = X W'^T + s U B^T
+    with W' dequantised inside the GEMM (q, k, v read the same input and so do
+    gate and up; with grouping on they run as one call per group);
+  * backward in reverse order: dU, dB, dX, dA (a group's dX is the sum over
+    its members, the gradient of the shared input);
+  * with N > 1 ranks, the sum of each linear's dA/dB over ranks (NCCL,
+    issued as soon as that linear's backward is enqueued, so it overlaps the
+    next linear's backward);
+  * the 8-bit AdamW step on every adapter.
+
+value = algorithmic fwd+bwd FLOPs of the seven linears (sum of
+4MNK + 6MKr + 6MNr) / device time per step, summed over ranks (each rank runs
+its own batch: weak scaling).  Quantisation and the optimizer step are in
+the timed step but not in the FLOP count.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -30,24 +42,21 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s (% bf16 peak); NF4 quant/dequant HBM GB/s"
-WORKLOAD = "c2"
-WORKLOAD_NAME = "LLaMA-7B attention projection: W 4096x4096 NF4/64 + FP8/256, 4x1024 tokens, r=64, alpha=16"
+WORKLOAD_NAME = ("LLaMA-7B-shaped decoder layer, all 7 linears (q,k,v,o 4096x4096; gate,up 4096->11008; "
+                 "down 11008->4096), NF4/64 + FP8/256, LoRA r=64 alpha=16 on every linear, 8x2048 = 16384 tokens")
+M_TOKENS = 8 * 2048
+RANK_R = 64
+ALPHA = 16.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+NF4_BYTES_PER_PARAM = 2 + 0.5 + 1 / 64 + 4 / 16384
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# tensor-core kernels of this workload, from one ncu capture of the CTA-pair
-# kernels on this workload (c2 forward and dX); emptied whenever those kernels change.
-NCU_TRAFFIC_BYTES = {"fused_fwd": 43.871232e6 + 3.50336e6, "fused_dx": 43.949312e6 + 2.96576e6}
+# tensor-core kernels in one layer step (mean over the step's launches of that
+# kernel), from an ncu capture of the current kernels; None until captured.
+NCU_TRAFFIC_BYTES = {}
 
 
 def flops_fwd_bwd(M, N, K, r):
     return 4 * M * N * K + 6 * M * K * r + 6 * M * N * r
-
-
-def kernel_flops(name, M, N, K, r):
-    """Algorithmic FLOPs of one launch of the tensor-core kernels."""
-    return {"fused_fwd": 2 * M * N * K + 2 * M * N * r, "fused_dx": 2 * M * N * K + 2 * M * K * r,
-            "lora_down": 2 * M * K * r, "lora_du": 2 * M * N * r, "lora_db": 2 * M * N * r,
-            "lora_da": 2 * M * K * r}.get(name)
 
 
 def load_peaks():
@@ -57,7 +66,7 @@ def load_peaks():
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
-    return dict(FALLBACK_PEAKS, source="fallback")
+    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"], source="fallback")
 
 
 # ------------------------------------------------------------------ clocks
@@ -112,35 +121,8 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU baseline
 
-def cpu_oracle_sample(reps=1, m_s=512, n_s=2048, seed=0):
-    """Time the oracle on a bounded sample of the workload.
-
-    Sample: the first n_s output features of the 4096x4096 weight and m_s
-    tokens: NF4-quantise + dequantise those weight rows, then the fp64
-    forward and backward on (m_s tokens, n_s features, K=4096, r=64).
-    Returns (TFLOP/s on the sample's fwd+bwd FLOPs, seconds, description).
-    """
-    import synth
-    from oracle import linear as ol
-    from oracle import nf4
-    wl = synth.WORKLOADS[WORKLOAD]
-    lin = wl.linears[0]
-    d = synth.linear_inputs(synth.Linear("sample", n_s, lin.k_in), m_s, wl.r, seed)
-    b = {k: synth.bf16_bits(v) for k, v in d.items()}
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        codes, c8, s2 = nf4.quantize(b["W"].reshape(-1))
-        wd = nf4.dequantize(codes, c8, s2, b["W"].size).reshape(b["W"].shape)
-        ol.linear_fwd(b["X"], wd, b["A"], b["B"], wl.s)
-        ol.linear_bwd(b["dY"], b["X"], wd, b["A"], b["B"], wl.s)
-    dt = time.perf_counter() - t0
-    fl = flops_fwd_bwd(m_s, n_s, lin.k_in, wl.r) * reps
-    desc = (f"{reps} x (quantize+dequantize {n_s}x{lin.k_in} weight rows, fp64 fwd+bwd on {m_s} tokens x "
-            f"{n_s} features x K={lin.k_in}, r={wl.r})")
-    return fl / dt / 1e12, dt, desc
-
-
 def cpu_cores():
+    """(cores this process may run on, BLAS threads numpy uses)."""
     try:
         n = len(os.sched_getaffinity(0))
     except AttributeError:
@@ -153,14 +135,252 @@ def cpu_cores():
     return n, blas
 
 
-# ------------------------------------------------------------------ arms
+_SAMPLE_CACHE = {}
+
+
+def _sample_inputs(m_s, n_s):
+    """Seeded inputs of the oracle's sample, drawn once per size."""
+    import synth
+    key = (m_s, n_s)
+    if key not in _SAMPLE_CACHE:
+        _SAMPLE_CACHE[key] = [
+            {k: synth.bf16_bits(v) for k, v in
+             synth.linear_inputs(synth.Linear("sample", n_s, lin.k_in), m_s, RANK_R, 10 + i).items()}
+            for i, lin in enumerate(synth.LLAMA7B_LAYER)]
+    return _SAMPLE_CACHE[key]
+
+
+def cpu_oracle_layer_sample(m_s=512, n_s=1024):
+    """Time the oracle on a bounded sample of the layer workload.
+
+    Sample, for each of the seven linears: the first n_s output features of
+    its weight (all K input features) and m_s tokens; NF4-quantise and
+    dequantise those weight rows, then the fp64 forward and backward
+    (U, Y, dU, dX, dA, dB) on (m_s tokens, n_s features, K, r=64).
+    Returns (TFLOP/s on the sample's fwd+bwd FLOPs, seconds, description).
+    """
+    import synth
+    from oracle import linear as ol
+    from oracle import nf4
+    s = ALPHA / RANK_R
+    fl, dt = 0.0, 0.0
+    for b, lin in zip(_sample_inputs(m_s, n_s), synth.LLAMA7B_LAYER):
+        t0 = time.perf_counter()
+        codes, c8, s2 = nf4.quantize(b["W"].reshape(-1))
+        wd = nf4.dequantize(codes, c8, s2, b["W"].size).reshape(b["W"].shape)
+        ol.linear_fwd(b["X"], wd, b["A"], b["B"], s)
+        ol.linear_bwd(b["dY"], b["X"], wd, b["A"], b["B"], s)
+        dt += time.perf_counter() - t0
+        fl += flops_fwd_bwd(m_s, n_s, lin.k_in, RANK_R)
+    desc = (f"per linear of the layer: quantize+dequantize {n_s} weight rows (all K), fp64 fwd+bwd on {m_s} "
+            f"tokens x {n_s} output features x K, r={RANK_R}")
+    return fl / dt / 1e12, dt, desc
+
+
+def cpu_oracle_nf4_rates(n_rows=4096, k=8192, seed=0):
+    """Oracle NF4 quantise and dequantise throughput on an n_rows x k weight:
+    params/s and the equivalent GB/s at 2.5159 B/param (bf16 in, NF4 out)."""
+    import synth
+    from oracle import nf4
+    wb = synth.bf16_bits(synth.weight_bf16(n_rows, k, seed)).reshape(-1)
+    t0 = time.perf_counter()
+    codes, c8, s2 = nf4.quantize(wb)
+    tq = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    nf4.dequantize(codes, c8, s2, wb.size)
+    tdq = time.perf_counter() - t0
+    n = wb.size
+    return {"params": n, "quantize_params_per_s": n / tq, "quantize_gbs": n * NF4_BYTES_PER_PARAM / tq / 1e9,
+            "dequantize_params_per_s": n / tdq, "dequantize_gbs": n * NF4_BYTES_PER_PARAM / tdq / 1e9,
+            "seconds": tq + tdq}
+
+
+# ------------------------------------------------------------ the layer step
+
+class LayerStep:
+    """The decoder layer's seven QLoRA linears on one GPU: buffers, and the
+    quantise / forward / backward / optimizer phases of one training step."""
+
+    def __init__(self, lib, synth, torch, dev, M, rank=0, world=1, grouped=False):
+        self.lib, self.torch, self.dev = lib, torch, dev
+        self.M, self.r, self.s = M, RANK_R, ALPHA / RANK_R
+        self.world = world
+        self.grouped = grouped and hasattr(lib, "qlora_group_fwd")
+        self.lins = synth.LLAMA7B_LAYER
+        self.input_of = synth.LAYER_INPUT_OF
+        r = self.r
+        params = synth.decoder_layer_params(r, seed=0, device=dev)
+        self.X, self.dY = synth.decoder_layer_activations(M, rank=rank, device=dev)
+        self.Wb = [p["W"] for p in params]
+        self.W, self.param, self.grad, self.A, self.B, self.dA, self.dB = [], [], [], [], [], [], []
+        self.U, self.Y, self.dX, self.opt = [], [], [], []
+        for i, lin in enumerate(self.lins):
+            N, K = lin.n_out, lin.k_in
+            nc, nb, ns = lib.nf4_sizes(N * K)
+            self.W.append(lib.NF4Weight(torch.empty(nc, dtype=torch.uint8, device=dev),
+                                        torch.empty(nb, dtype=torch.uint8, device=dev),
+                                        torch.empty(ns, dtype=torch.float32, device=dev), N, K))
+            # A and B of a linear are views of one flat bf16 parameter; dA and
+            # dB views of one flat fp32 gradient (one all-reduce, one
+            # optimizer call per linear).
+            p = torch.empty(r * K + N * r, dtype=torch.bfloat16, device=dev)
+            p[: r * K].copy_(params[i]["A"].reshape(-1))
+            p[r * K:].copy_(params[i]["B"].reshape(-1))
+            g = torch.empty(r * K + N * r, dtype=torch.float32, device=dev)
+            self.param.append(p)
+            self.grad.append(g)
+            self.A.append(p[: r * K].view(r, K))
+            self.B.append(p[r * K:].view(N, r))
+            self.dA.append(g[: r * K].view(r, K))
+            self.dB.append(g[r * K:].view(N, r))
+            self.U.append(torch.empty((M, r), dtype=torch.float32, device=dev))
+            self.Y.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+            self.dX.append(torch.empty((M, K), dtype=torch.bfloat16, device=dev))
+            self.opt.append(lib.AdamW8State(p.numel(), paged=False, device=dev))
+        kmax = max(lin.k_in for lin in self.lins)
+        nmax = max(lin.n_out for lin in self.lins)
+        self.ws_f = torch.empty(max(lib.qlora_fwd_workspace_size(M, nmax, kmax, r), 16), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(max(lib.qlora_bwd_workspace_size(M, nmax, kmax, r), 16), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.t = 0
+        self.pending = []
+
+    def flops(self):
+        return sum(flops_fwd_bwd(self.M, lin.n_out, lin.k_in, self.r) for lin in self.lins)
+
+    def kernel_flops(self, name):
+        """Algorithmic FLOPs per step of the named tensor-core kernel."""
+        M, r = self.M, self.r
+        tot = 0
+        for lin in self.lins:
+            N, K = lin.n_out, lin.k_in
+            tot += {"fused_fwd": 2 * M * N * K + 2 * M * N * r, "fused_dx": 2 * M * N * K + 2 * M * K * r,
+                    "lora_down": 2 * M * K * r, "lora_du": 2 * M * N * r, "lora_db": 2 * M * N * r,
+                    "lora_da": 2 * M * K * r}.get(name, 0)
+        return tot
+
+    def quantize(self):
+        lib = self.lib
+        for i in range(len(self.lins)):
+            W = self.W[i]
+            lib.nf4_quantize(self.Wb[i].reshape(-1), W.codes, W.c8, W.s2, status=self.status)
+
+    def forward(self):
+        lib = self.lib
+        for i in range(len(self.lins)):
+            lib.qlora_linear_fwd(self.X[self.input_of[i]], self.W[i], self.A[i], self.B[i], self.s, Y=self.Y[i],
+                                 U=self.U[i], ws=self.ws_f, status=self.status)
+
+    def backward(self):
+        lib = self.lib
+        for i in reversed(range(len(self.lins))):
+            lib.qlora_linear_bwd(self.dY[i], self.X[self.input_of[i]], self.U[i], self.W[i], self.A[i], self.B[i],
+                                 self.s, dX=self.dX[i], dA=self.dA[i], dB=self.dB[i], ws=self.ws_b,
+                                 status=self.status)
+            self._reduce(i)
+
+    def _reduce(self, i):
+        # Sum of the adapter gradients over ranks, issued right after this
+        # linear's backward: NCCL's stream waits for it and then runs beside
+        # the next linear's backward.
+        if self.world > 1:
+            import torch.distributed as dist
+            self.pending.append(dist.all_reduce(self.grad[i], async_op=True))
+
+    def optimizer(self):
+        for h in self.pending:
+            h.wait()
+        self.pending = []
+        self.t += 1
+        for i in range(len(self.lins)):
+            self.lib.qlora_adamw8_step(self.param[i], self.grad[i], self.opt[i], lr=2e-4, step=self.t,
+                                       status=self.status)
+
+    def step(self):
+        self.quantize()
+        self.forward()
+        self.backward()
+        self.optimizer()
+
+    def close(self):
+        for o in self.opt:
+            o.close()
+
+
+def time_steps(torch, step, stream, steps, flush, dist=None):
+    """Per-step device times (ms) of `steps` steps, one event pair each, L2
+    flushed (512 MB memset) before every step outside its events."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def kernel_table(records, steps):
+    kern = {}
+    for name, t in records:
+        k = kern.setdefault(name, {"launches": 0, "ms_total": 0.0})
+        k["launches"] += 1
+        k["ms_total"] += t
+    tot = sum(k["ms_total"] for k in kern.values()) or 1.0
+    for k in kern.values():
+        k["share"] = k["ms_total"] / tot
+        k["ms_avg"] = k["ms_total"] / k["launches"]
+        k["ms_per_step"] = k["ms_total"] / steps
+    return kern
+
+
+# ------------------------------------------------------------------ extras
+
+def c2_step_timing(lib, synth, torch, dev, flush, reps=20):
+    """The single 4096x4096 projection (4 x 1024 tokens, r=64): quantise +
+    forward + backward, L2 flushed before each step."""
+    wl = synth.WORKLOADS["c2"]
+    lin = wl.linears[0]
+    M, N, K, r, s = wl.m_tokens, lin.n_out, lin.k_in, wl.r, wl.s
+    g = {k: v.to(dev) for k, v in synth.linear_inputs(lin, M, r, 0).items()}
+    W = lib.quantize_weight(g["W"])
+    out = {"Y": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+           "U": torch.empty((M, r), dtype=torch.float32, device=dev),
+           "dX": torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+           "dA": torch.empty((r, K), dtype=torch.float32, device=dev),
+           "dB": torch.empty((N, r), dtype=torch.float32, device=dev)}
+    ws_f = torch.empty(lib.qlora_fwd_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(lib.qlora_bwd_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step():
+        lib.nf4_quantize(g["W"].reshape(-1), W.codes, W.c8, W.s2)
+        lib.qlora_linear_fwd(g["X"], W, g["A"], g["B"], s, Y=out["Y"], U=out["U"], ws=ws_f)
+        lib.qlora_linear_bwd(g["dY"], g["X"], out["U"], W, g["A"], g["B"], s, dX=out["dX"], dA=out["dA"],
+                             dB=out["dB"], ws=ws_b)
+
+    for _ in range(3):
+        step()
+    ts = time_steps(torch, step, torch.cuda.current_stream(), reps, flush)
+    ms = statistics.median(ts)
+    return {"workload": "4096x4096 projection, 4x1024 tokens, r=64: quantize + fwd + bwd (L2 flushed)",
+            "ms": ms, "tflops": flops_fwd_bwd(M, N, K, r) / (ms * 1e-3) / 1e12}
+
 
 def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
     """Forward of the 65B-shaped 8192<->22016 linears over M in {1,16,128,2048,16384}.
 
     Per case: algorithmic bytes 0.5159 N K + 2 M K + 2 M N + 2 r (K + N) and
     FLOPs 2 M N K + 2 M K r + 2 M N r, over the mean device time of the
-    forward call (L2 flushed before each run).
+    forward call (L2 flushed before each run).  kernels_ms: per-kernel event
+    times averaged over `reps` further calls with every kernel bracketed by
+    events (the brackets serialise the kernels, which otherwise overlap
+    through programmatic dependent launch); ms_bracketed is the outer time of
+    those same calls.
     """
     out = {}
     r, s = 64, 0.25
@@ -176,36 +396,66 @@ def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             U = torch.empty((M, r), dtype=torch.float32, device=dev)
             ws = torch.empty(max(lib.qlora_fwd_workspace_size(M, N, K, r), 16), dtype=torch.uint8, device=dev)
-            for _ in range(2):
+
+            def call():
                 lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
-            ts = []
-            for _ in range(reps):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
-                e1.record()
-                e1.synchronize()
-                ts.append(e0.elapsed_time(e1))
+
+            for _ in range(3):
+                call()
+            ts = time_steps(torch, call, torch.cuda.current_stream(), reps, flush)
             ms = float(np.mean(ts))
-            # one more call with per-kernel event brackets (not part of ms)
-            flush.zero_()
             lib.profile_enable(True)
-            lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
-            torch.cuda.synchronize()
+            tb = time_steps(torch, call, torch.cuda.current_stream(), reps, flush)
             lib.profile_enable(False)
             kern = {}
             for name, kms in lib.profile_collect():
-                kern[name] = round(kern.get(name, 0.0) + kms, 5)
+                kern[name] = kern.get(name, 0.0) + kms / reps
             byts = 0.51587 * N * K + 2 * M * K + 2 * M * N + 2 * r * (K + N)
             fl = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
             out[f"{lin.name}_{N}x{K}_M{M}"] = {
                 "ms": round(ms, 5), "tflops": round(fl / ms / 1e9, 2), "gbs": round(byts / ms / 1e6, 1),
                 "hbm_frac": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
-                "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "kernels_ms": kern}
+                "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4),
+                "ms_bracketed": round(float(np.mean(tb)), 5),
+                "kernels_ms": {k: round(v, 5) for k, v in kern.items()}}
             del X, Y, U, ws
         del W, A, B
     return out
+
+
+def c5_quantize_sweep(lib, synth, torch, dev):
+    """NF4 quantisation of every linear weight of the 80-layer 65B-shaped
+    model (hidden 8192, intermediate 22016; 64.76 G parameters).  Each layer's
+    seven bf16 weights are drawn on the device, quantised, and dropped: only
+    the NF4 storage (33.4 GB) stays resident.  GB/s counts 2.5159 B/param over
+    the summed device time of the quantise calls; the wall time includes the
+    random draws.  Weight seeds: 650000 + 10 * layer + index (the GPU test
+    of this sweep redraws layers with the same seeds)."""
+    t_wall = time.perf_counter()
+    kept, total_ms, params = [], 0.0, 0
+    for layer in range(synth.C5_LAYERS):
+        for j, lin in enumerate(synth.c5_layer_linears()):
+            w = synth.weight_bf16(lin.n_out, lin.k_in, seed=650000 + 10 * layer + j, device=dev)
+            nc, nb, ns = lib.nf4_sizes(w.numel())
+            codes = torch.empty(nc, dtype=torch.uint8, device=dev)
+            c8 = torch.empty(nb, dtype=torch.uint8, device=dev)
+            s2 = torch.empty(ns, dtype=torch.float32, device=dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            lib.nf4_quantize(w.reshape(-1), codes, c8, s2)
+            e1.record()
+            kept.append((codes, c8, s2, e0, e1))
+            params += w.numel()
+            del w
+    torch.cuda.synchronize()
+    for k in kept:
+        total_ms += k[3].elapsed_time(k[4])
+    wall = time.perf_counter() - t_wall
+    resident = sum(k[0].numel() + k[1].numel() + 4 * k[2].numel() for k in kept)
+    del kept
+    return {"layers": synth.C5_LAYERS, "params": params, "resident_nf4_bytes": resident,
+            "quantize_ms_total": total_ms, "quantize_gbs": params * NF4_BYTES_PER_PARAM / (total_ms * 1e-3) / 1e9,
+            "wall_s_with_draws": wall}
 
 
 def c1_graph_timing(lib, synth, torch, dev, reps=200):
@@ -275,248 +525,9 @@ def c1_graph_timing(lib, synth, torch, dev, reps=200):
             "workload": "512x512 NF4, 64 tokens, r=16: quantize + fwd + bwd back to back (L2-resident)"}
 
 
-def run_reference(args, rank, world):
-    """The CPU oracle as the reference arm (rank 0 only)."""
-    if rank != 0:
-        return
-    cores, blas = cpu_cores()
-    times, vals = [], []
-    for i in range(args.warmup + args.steps):
-        v, dt, desc = cpu_oracle_sample(reps=1, m_s=256, n_s=1024, seed=i)
-        if i >= args.warmup:
-            times.append(dt)
-            vals.append(v)
-    value = float(np.mean(vals))
-    ms = 1e3 * float(np.mean(times))
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD_NAME, "sample": desc},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas, "kind": "oracle", "sample": desc},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def run_ours(args, rank, world):
-    import torch
-    import torch.distributed as dist
-
-    import bit_nf4_quantized_26_b200 as lib
-    import synth
-
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    wl = synth.WORKLOADS[WORKLOAD]
-    lin = wl.linears[0]
-    M, N, K, r, s = wl.m_tokens, lin.n_out, lin.k_in, wl.r, wl.s
-    d = synth.dp_shard_inputs(lin, M, r, rank)
-    g = {k: v.to(dev) for k, v in d.items()}
-    W_bf16 = g["W"]
-    nc, nb, ns = lib.nf4_sizes(N * K)
-    codes = torch.empty(nc, dtype=torch.uint8, device=dev)
-    c8 = torch.empty(nb, dtype=torch.uint8, device=dev)
-    s2 = torch.empty(ns, dtype=torch.float32, device=dev)
-    W = lib.NF4Weight(codes, c8, s2, N, K)
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    U = torch.empty((M, r), dtype=torch.float32, device=dev)
-    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    dA = torch.empty((r, K), dtype=torch.float32, device=dev)
-    dB = torch.empty((N, r), dtype=torch.float32, device=dev)
-    ws_f = torch.empty(lib.qlora_fwd_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(lib.qlora_bwd_workspace_size(M, N, K, r), dtype=torch.uint8, device=dev)
-    status = torch.zeros(4, dtype=torch.int32, device=dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        lib.nf4_quantize(W_bf16.reshape(-1), codes, c8, s2, status=status)
-        lib.qlora_linear_fwd(g["X"], W, g["A"], g["B"], s, Y=Y, U=U, ws=ws_f, status=status)
-        lib.qlora_linear_bwd(g["dY"], g["X"], U, W, g["A"], g["B"], s, dX=dX, dA=dA, dB=dB, ws=ws_b,
-                             status=status)
-        if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-
-    # ---------------------------------------------------------- timed region
-    # Phase A (the reported value): K steps, one event pair per step, nothing
-    # else in the stream between the step's kernels (they chain through
-    # programmatic dependent launch).  Phase B: the same K steps again with
-    # every library kernel bracketed by events, for the per-kernel table and
-    # the roofline of the dominant kernel.
-    sampler = ClockSampler(dev.index)
-    sampler.start()
-    time.sleep(0.3)
-
-    def timed_steps():
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        for e0, e1 in evs:
-            flush.zero_()
-            e0.record(stream)
-            step()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return [a.elapsed_time(b) for a, b in evs]
-
-    step_ms = timed_steps()
-    lib.profile_enable(True)
-    step_ms_profiled = timed_steps()
-    lib.profile_enable(False)
-    clocks = sampler.stop()
-    records = lib.profile_collect()
-    ms = float(sum(step_ms) / len(step_ms))
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    assert int(status[0].item()) == 0, f"device status {int(status[0].item())}"
-
-    # per-kernel statistics from the library's event brackets
-    kern = {}
-    for name, t in records:
-        k = kern.setdefault(name, {"launches": 0, "ms_total": 0.0})
-        k["launches"] += 1
-        k["ms_total"] += t
-    tot = sum(k["ms_total"] for k in kern.values()) or 1.0
-    for k in kern.values():
-        k["share"] = k["ms_total"] / tot
-        k["ms_avg"] = k["ms_total"] / k["launches"]
-    peaks = load_peaks()
-    tc = {n: k for n, k in kern.items() if n in ("fused_fwd", "fused_dx")}
-    dom = max(tc, key=lambda n: tc[n]["ms_total"]) if tc else None
-    roofline = None
-    if dom:
-        fl = kernel_flops(dom, M, N, K, r)
-        ach = fl / (kern[dom]["ms_avg"] * 1e-3) / 1e12
-        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": NCU_TRAFFIC_BYTES.get(dom),
-                    "peak_source": f"{peaks['source']} bf16 burst"}
-        for n in tc:
-            kf = kernel_flops(n, M, N, K, r)
-            kern[n]["tflops"] = kf / (kern[n]["ms_avg"] * 1e-3) / 1e12
-
-    if args.kernels_only:
-        if rank == 0:
-            print(json.dumps({"kernels_only": True, "ms_per_step": ms,
-                              "ms_per_step_profiled": float(np.mean(step_ms_profiled)), "kernels": kern}), flush=True)
-        return
-
-    # ------------------------------------------------ NF4 stream bandwidth
-    # Separate launches on a weight larger than L2 (22016x8192, 65B-shaped).
-    big = synth.weight_bf16(22016, 8192, seed=99, device=dev)
-    bcodes, bc8, bs2 = lib.nf4_quantize(big.reshape(-1))
-    bout = torch.empty(big.numel(), dtype=torch.bfloat16, device=dev)
-    lib.profile_enable(True)
-    for _ in range(5):
-        flush.zero_()
-        lib.nf4_quantize(big.reshape(-1), bcodes, bc8, bs2)
-        flush.zero_()
-        lib.nf4_dequantize(bcodes, bc8, bs2, big.numel(), out=bout)
-    torch.cuda.synchronize()
-    lib.profile_enable(False)
-    qrec = lib.profile_collect()
-    bytes_nf4 = big.numel() * (2 + 0.5 + 1 / 64 + 4 / 16384)
-    qt = [t for n, t in qrec if n == "nf4_quantize"]
-    dqt = [t for n, t in qrec if n == "nf4_dequantize"]
-    quant_gbs = bytes_nf4 / (statistics.median(qt) * 1e-3) / 1e9
-    dequant_gbs = bytes_nf4 / (statistics.median(dqt) * 1e-3) / 1e9
-    del big, bcodes, bc8, bs2, bout
-
-    # ------------------------------------------- adapter optimizer step
-    adamw = adamw8_timing(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
-    drop = dropout_timing(lib, synth, torch, dev, flush) if (rank == 0 and not args.no_sweep) else None
-
-    # ------------------------------------------- 65B-shaped forward sweep
-    c5 = c5_forward_sweep(lib, synth, torch, dev, flush, peaks) if (rank == 0 and not args.no_sweep) else None
-    c1g = c1_graph_timing(lib, synth, torch, dev) if (rank == 0 and not args.no_sweep) else None
-
-    # ------------------------------------------------------------- e2e
-    host = {k: torch.empty_like(g[k], device="cpu").pin_memory() for k in ("W", "X", "dY")}
-    for k in host:
-        host[k].copy_(d[k])
-    hout = {"Y": torch.empty_like(Y, device="cpu").pin_memory(), "dX": torch.empty_like(dX, device="cpu").pin_memory(),
-            "dA": torch.empty_like(dA, device="cpu").pin_memory(), "dB": torch.empty_like(dB, device="cpu").pin_memory()}
-    outs = {"Y": Y, "dX": dX, "dA": dA, "dB": dB}
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in hout.values())
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for k in host:
-            g[k].copy_(host[k], non_blocking=True)
-        step()
-        for k in hout:
-            hout[k].copy_(outs[k], non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e = float(np.mean(e2e_ms))
-    if world > 1:
-        t = torch.tensor([e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e = float(t.item())
-
-    fl = flops_fwd_bwd(M, N, K, r)
-    value = world * fl / (ms * 1e-3) / 1e12
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        cores, blas = cpu_cores()
-        v, dt, desc = cpu_oracle_sample(reps=4)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": blas, "kind": "oracle", "sample": desc,
-               "seconds": dt}
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME, "M": M, "N": N, "K": K, "r": r, "alpha": wl.alpha,
-                       "parallelism": f"dp{world}", "global_batch": M * world,
-                       "step": "nf4_quantize + qlora_linear_fwd + qlora_linear_bwd (+ dA/dB all-reduce if N>1)",
-                       "l2": "flushed before every step (512 MB memset outside the step's events)",
-                       "pdl": os.environ.get("QLORA_PDL", "1") != "0"},
-            "pct_bf16_peak": value / world / peaks["bf16_tflops"],
-            "roofline": roofline,
-            "cpu_baseline": cpu,
-            "e2e": {"value": world * fl / (e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": len(records),
-            "timing": {"value_from": "phase A: K steps, step-level events only",
-                       "kernels_from": "phase B: the same K steps with per-kernel event brackets",
-                       "ms_per_step_phase_b": float(np.mean(step_ms_profiled))},
-            "clocks": clocks,
-            "kernels": {n: {kk: round(vv, 5) if isinstance(vv, float) else vv for kk, vv in k.items()}
-                        for n, k in sorted(kern.items(), key=lambda x: -x[1]["ms_total"])},
-            "nf4_quantize_gbs": quant_gbs, "nf4_dequantize_gbs": dequant_gbs,
-            "c5_forward": c5,
-            "c1_graph": c1g,
-            "adamw8": adamw,
-            "lora_dropout": drop,
-            "nf4_hbm_frac": {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
-                             "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]},
-        }
-        print(json.dumps(line), flush=True)
-
-
 def dropout_timing(lib, synth, torch, dev, flush, p=0.05, reps=10):
     """The c2 forward + backward with LoRA dropout (p = 0.05, the tutorial's
     lora_dropout) against the same step without it; L2 flushed before each."""
-    import statistics
     M = N = K = 4096
     r, s = 64, 0.25
     d = {k: v.to(dev) for k, v in synth.linear_inputs(synth.Linear("c2", N, K), M, r, 0).items()}
@@ -559,7 +570,6 @@ def adamw8_timing(lib, synth, torch, dev, flush, peaks, layers=10, reps=10):
     states in device memory and in paged (managed, device-resident) memory.
     Algorithmic bytes per parameter: bf16 p read + write, fp32 gradient, two
     state bytes read + write, two fp32 scales per 256 read + write."""
-    import statistics
     r = 64
     per_layer = sum(r * (lin.n_out + lin.k_in) for lin in synth.c5_layer_linears())
     n = per_layer * layers
@@ -590,17 +600,233 @@ def adamw8_timing(lib, synth, torch, dev, flush, peaks, layers=10, reps=10):
     return out
 
 
+def nf4_stream_timing(lib, synth, torch, dev, flush, reps=5):
+    """Standalone quantise and dequantise of a 22016x8192 weight (larger than
+    L2), L2 flushed before each launch; median of the per-launch event times."""
+    big = synth.weight_bf16(22016, 8192, seed=99, device=dev)
+    bcodes, bc8, bs2 = lib.nf4_quantize(big.reshape(-1))
+    bout = torch.empty(big.numel(), dtype=torch.bfloat16, device=dev)
+    lib.profile_enable(True)
+    for _ in range(reps):
+        flush.zero_()
+        lib.nf4_quantize(big.reshape(-1), bcodes, bc8, bs2)
+        flush.zero_()
+        lib.nf4_dequantize(bcodes, bc8, bs2, big.numel(), out=bout)
+    torch.cuda.synchronize()
+    lib.profile_enable(False)
+    qrec = lib.profile_collect()
+    nbytes = big.numel() * NF4_BYTES_PER_PARAM
+    qt = [t for n, t in qrec if n == "nf4_quantize"]
+    dqt = [t for n, t in qrec if n == "nf4_dequantize"]
+    return nbytes / (statistics.median(qt) * 1e-3) / 1e9, nbytes / (statistics.median(dqt) * 1e-3) / 1e9
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm (rank 0 only), on a bounded sample
+    of the layer workload per step."""
+    if rank != 0:
+        return
+    cores, blas = cpu_cores()
+    times, vals = [], []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        v, dt, desc = cpu_oracle_layer_sample(m_s=128, n_s=256)
+        if i >= args.warmup:
+            times.append(dt)
+            vals.append(v)
+    value = float(np.mean(vals))
+    ms = 1e3 * float(np.mean(times))
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD_NAME, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "blas_threads": blas, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import bit_nf4_quantized_26_b200 as lib
+    import synth
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    M = args.tokens
+    layer = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=not args.no_group)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    dd = dist if world > 1 else None
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer.step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    # ---------------------------------------------------------- timed region
+    # Phase A (the reported value): K steps, one event pair per step, nothing
+    # else in the stream between the step's kernels (they chain through
+    # programmatic dependent launch).  Phase B: the same K steps again with
+    # every library kernel bracketed by events, for the per-kernel table and
+    # the roofline of the dominant kernel.
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    step_ms = time_steps(torch, layer.step, stream, args.steps, flush, dd)
+    lib.profile_enable(True)
+    step_ms_profiled = time_steps(torch, layer.step, stream, args.steps, flush, dd)
+    lib.profile_enable(False)
+    clocks = sampler.stop()
+    records = lib.profile_collect()
+    ms = float(sum(step_ms) / len(step_ms))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert int(layer.status[0].item()) == 0, f"device status {int(layer.status[0].item())}"
+
+    kern = kernel_table(records, args.steps)
+    peaks = load_peaks()
+    tc = {n: k for n, k in kern.items() if n in ("fused_fwd", "fused_dx")}
+    roofline = None
+    if tc:
+        dom = max(tc, key=lambda n: tc[n]["ms_total"])
+        for n in tc:
+            kern[n]["tflops"] = layer.kernel_flops(n) / (kern[n]["ms_per_step"] * 1e-3) / 1e12
+        ach = kern[dom]["tflops"]
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": NCU_TRAFFIC_BYTES.get(dom),
+                    "peak_source": f"{peaks['source']} bf16 burst",
+                    "launches_per_step": kern[dom]["launches"] // args.steps,
+                    "achieved_from": "algorithmic FLOPs of the kernel's launches in a step / their summed "
+                                     "event time per step (phase B)"}
+
+    if args.kernels_only:
+        if rank == 0:
+            print(json.dumps({"kernels_only": True, "ms_per_step": ms,
+                              "ms_per_step_profiled": float(np.mean(step_ms_profiled)), "kernels": kern}), flush=True)
+        layer.close()
+        return
+
+    # ------------------------------------------------------------- e2e
+    # The same step through the same API, with the step's inputs (the four
+    # layer inputs and the seven upstream gradients) copied in from pinned
+    # host memory and its result (the summed adapter gradients) copied back,
+    # inside the timed region.
+    host_in = {f"X_{k}": (v, torch.empty_like(v, device="cpu").pin_memory()) for k, v in layer.X.items()}
+    host_in.update({f"dY_{i}": (v, torch.empty_like(v, device="cpu").pin_memory()) for i, v in enumerate(layer.dY)})
+    for dv, hv in host_in.values():
+        hv.copy_(dv)
+    host_out = [(g, torch.empty_like(g, device="cpu").pin_memory()) for g in layer.grad]
+    h2d = sum(hv.numel() * hv.element_size() for _, hv in host_in.values())
+    d2h = sum(hv.numel() * hv.element_size() for _, hv in host_out)
+
+    def e2e_step():
+        for dv, hv in host_in.values():
+            dv.copy_(hv, non_blocking=True)
+        layer.step()
+        for dv, hv in host_out:
+            hv.copy_(dv, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_ms = time_steps(torch, e2e_step, stream, max(3, args.steps // 4), flush, dd)
+    e2e = float(np.mean(e2e_ms))
+    if world > 1:
+        t = torch.tensor([e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e = float(t.item())
+    fl = layer.flops()
+    layer.close()
+    del layer, host_in, host_out
+
+    extras = {}
+    if rank == 0 and not args.no_sweep:
+        quant_gbs, dequant_gbs = nf4_stream_timing(lib, synth, torch, dev, flush)
+        extras["nf4_quantize_gbs"] = quant_gbs
+        extras["nf4_dequantize_gbs"] = dequant_gbs
+        extras["nf4_hbm_frac"] = {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
+                                  "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]}
+        extras["c2_step"] = c2_step_timing(lib, synth, torch, dev, flush)
+        extras["adamw8"] = adamw8_timing(lib, synth, torch, dev, flush, peaks)
+        extras["lora_dropout"] = dropout_timing(lib, synth, torch, dev, flush)
+        extras["c5_forward"] = c5_forward_sweep(lib, synth, torch, dev, flush, peaks)
+        extras["c5_quantize_sweep"] = c5_quantize_sweep(lib, synth, torch, dev)
+        extras["c5_quantize_sweep"]["hbm_frac"] = extras["c5_quantize_sweep"]["quantize_gbs"] / peaks["hbm_gbs"]
+        extras["c1_graph"] = c1_graph_timing(lib, synth, torch, dev)
+
+    value = world * fl / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cores, blas = cpu_cores()
+        v, dt, desc = cpu_oracle_layer_sample()
+        rates = cpu_oracle_nf4_rates()
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "blas_threads": blas, "kind": "oracle",
+               "sample": desc, "seconds": dt, "nf4": rates}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, "tokens_per_gpu": M, "r": RANK_R, "alpha": ALPHA,
+                       "linears": [[lin.name, lin.n_out, lin.k_in] for lin in synth.LLAMA7B_LAYER],
+                       "parallelism": f"dp{world}", "global_batch_tokens": M * world,
+                       "grouped_projections": bool(getattr(lib, "qlora_group_fwd", None)) and not args.no_group,
+                       "step": "nf4_quantize x7 + forward x7 + backward x7 (+ dA/dB all-reduce per linear if N>1) "
+                               "+ 8-bit AdamW on every adapter",
+                       "flops_per_step_per_gpu": fl,
+                       "l2": "flushed before every step (512 MB memset outside the step's events)",
+                       "pdl": os.environ.get("QLORA_PDL", "1") != "0"},
+            "pct_bf16_peak": value / world / peaks["bf16_tflops"],
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * fl / (e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(records),
+            "timing": {"value_from": "phase A: K steps, step-level events only",
+                       "kernels_from": "phase B: the same K steps with per-kernel event brackets",
+                       "ms_per_step_phase_b": float(np.mean(step_ms_profiled)),
+                       "ms_per_step_min": float(min(step_ms)), "ms_per_step_max": float(max(step_ms))},
+            "clocks": clocks,
+            "kernels": {n: {kk: round(vv, 5) if isinstance(vv, float) else vv for kk, vv in k.items()}
+                        for n, k in sorted(kern.items(), key=lambda x: -x[1]["ms_total"])},
+            "peaks": peaks,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+
+
 def run_case(args):
     """Profiler driver: time one entry point on one shape (no JSON contract).
 
     --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), quant:N:K / dequant:N:K (NF4
-    quantisation / dequantisation of an N x K weight), or adamw8:n (one 8-bit AdamW
-    step over n parameters), --steps calls after 2 warm-up calls.
+    quantisation / dequantisation of an N x K weight), adamw8:n (one 8-bit AdamW
+    step over n parameters), or layer:M (the decoder-layer step with M tokens);
+    --steps calls after 2 warm-up calls.
     """
     import torch
 
     import bit_nf4_quantized_26_b200 as lib
     import synth
+    dev = torch.device("cuda", 0)
+    if args.case.startswith("layer:"):
+        M = int(args.case.split(":")[1])
+        layer = LayerStep(lib, synth, torch, dev, M, grouped=not args.no_group)
+        for _ in range(2 + args.steps):
+            layer.step()
+        torch.cuda.synchronize()
+        layer.close()
+        print(json.dumps({"case": args.case, "ok": True}))
+        return
     if args.case.startswith("adamw8:"):
         n = int(args.case.split(":")[1])
         gen = torch.Generator(device="cuda").manual_seed(5)
@@ -653,12 +879,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=M_TOKENS, help="tokens per GPU (default 8 x 2048)")
+    ap.add_argument("--no-group", action="store_true", help="run every linear as its own call")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--no-sweep", action="store_true", help="skip the 65B-shaped forward sweep")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the extra measurements after the headline")
     ap.add_argument("--kernels-only", action="store_true",
-                    help="only the timed steps (for profiler captures): no e2e, no NF4 stream test, no CPU baseline")
+                    help="only the timed steps (for profiler captures): no e2e, no extras, no CPU baseline")
     ap.add_argument("--case", default=None,
-                    help="profiler driver: fwd:M:N:K, bwd:M:N:K, quant:N:K, dequant:N:K or adamw8:n")
+                    help="profiler driver: fwd:M:N:K, bwd:M:N:K, quant:N:K, dequant:N:K, adamw8:n or layer:M")
     args = ap.parse_args()
     if args.case:
         run_case(args)

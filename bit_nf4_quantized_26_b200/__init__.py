@@ -37,7 +37,7 @@ DEV_TIMEOUT = 2
 
 STATUS = {0: "QLORA_OK", 1: "QLORA_ERR_NULL", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
           4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_NONFINITE", 6: "QLORA_ERR_TIMEOUT",
-          7: "QLORA_ERR_CUDA", 8: "QLORA_ERR_ARCH", 9: "QLORA_ERR_DTYPE"}
+          7: "QLORA_ERR_CUDA", 8: "QLORA_ERR_ARCH", 9: "QLORA_ERR_DTYPE", 10: "QLORA_ERR_INTERNAL"}
 
 
 class QloraError(RuntimeError):

@@ -2,7 +2,6 @@
 // workspace planning, TMA descriptor creation and kernel launches.
 #include <algorithm>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -38,6 +37,12 @@ double normal_quantile(double p) {
   return 0.5 * (lo + hi);
 }
 
+// Set when the bucket table below fails its construction checks (a midpoint
+// on or next to a bucket edge, or two midpoints in one bucket); every compute
+// entry point then returns QLORA_ERR_INTERNAL.  The checks are on fixed
+// constants, so this never happens with the NF4 levels.
+bool g_tables_bad = false;
+
 Nf4Tables build_tables() {
   const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
   std::vector<double> lv;
@@ -67,9 +72,9 @@ Nf4Tables build_tables() {
       else if (m <= hi) { ++inside; thr = mid[i]; }
       // A midpoint on (or next to) a bucket edge would make the bucket
       // choice matter; the NF4 midpoints sit at least 4e-3 from every edge.
-      if (std::fabs(m - lo) < 1e-6 || std::fabs(m - hi) < 1e-6) std::abort();
+      if (std::fabs(m - lo) < 1e-6 || std::fabs(m - hi) < 1e-6) g_tables_bad = true;
     }
-    if (inside > 1) std::abort();
+    if (inside > 1) g_tables_bad = true;
     t.base[b] = below;
     t.thr[b] = thr;
   }
@@ -160,6 +165,8 @@ bool use_pair(int64_t rows) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 qlora_status check_device() {
+  (void)tables();
+  if (g_tables_bad) return QLORA_ERR_INTERNAL;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
   static int arch_ok[64] = {0};  // 0 unknown, 1 ok, 2 not sm_100
@@ -274,9 +281,11 @@ bool fork_enabled() {
 }
 
 // The current device's side stream, created on first use; `lk` holds the
-// lock (one fork/join sequence at a time).  nullptr: no fork.
+// lock (one fork/join sequence at a time).  nullptr: no fork.  While kernel
+// timing is on there is no fork either, so that each kernel's event pair
+// brackets that kernel alone rather than its overlap with the dX GEMM.
 SideStream* side_stream(std::unique_lock<std::mutex>& lk) {
-  if (!fork_enabled()) return nullptr;
+  if (!fork_enabled() || g_prof_on) return nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   lk = std::unique_lock<std::mutex>(g_side_mu);
@@ -477,6 +486,7 @@ const char* qlora_strerror(qlora_status s) {
     case QLORA_ERR_CUDA: return "a CUDA call failed";
     case QLORA_ERR_ARCH: return "the current device is not sm_100";
     case QLORA_ERR_DTYPE: return "unknown output dtype";
+    case QLORA_ERR_INTERNAL: return "an internal constant table failed its construction check";
   }
   return "unknown status";
 }
@@ -525,11 +535,11 @@ qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float
                                          static_cast<cudaStream_t>(stream)));
 }
 
-// The forward; Xa is the adapter's input: X itself, or X after dropout.
-static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64_t M, nf4_weight W,
-                                    const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y,
-                                    int32_t y_dtype, float* U_out, void* ws, size_t ws_bytes, int32_t* d_status,
-                                    void* stream) {
+}  // extern "C"
+
+qlora_status qnf4::check_fwd_args(const uint16_t* X, const uint16_t* Xa, int64_t M, const nf4_weight& W,
+                                  const uint16_t* A, const uint16_t* B, int32_t r, const void* Y, int32_t y_dtype,
+                                  const float* U_out, const int32_t* d_status) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
@@ -538,6 +548,18 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   if (!aligned16(X) || !aligned16(Xa) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(U_out) ||
       (d_status && !aligned16(d_status)))
     return QLORA_ERR_ALIGN;
+  return QLORA_OK;
+}
+
+extern "C" {
+
+// The forward; Xa is the adapter's input: X itself, or X after dropout.
+static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64_t M, nf4_weight W,
+                                    const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y,
+                                    int32_t y_dtype, float* U_out, void* ws, size_t ws_bytes, int32_t* d_status,
+                                    void* stream) {
+  if (qlora_status st = check_fwd_args(X, Xa, M, W, A, B, r, Y, y_dtype, U_out, d_status)) return st;
+  if (M == 0) return QLORA_OK;
   const int64_t N = W.n_out, K = W.k_in;
   const FwdPlan p = plan_fwd(M, N, K, r);
   if (!ws || ws_bytes < p.total) return QLORA_ERR_WORKSPACE;

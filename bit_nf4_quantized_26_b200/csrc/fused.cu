@@ -22,13 +22,6 @@
 
 namespace qnf4 {
 
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
-  }
-}
-
 // Ring plan.  For a handful of tokens (BN <= 64) the kernel only streams the
 // weight: two CTAs share an SM (3-4 stages each) so more dequantiser warps
 // hide the lookup latency; larger tiles run one CTA per SM with a deep ring.
@@ -142,7 +135,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       }
       // Do not leave the CTA while a copy into its shared memory is in flight.
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
-        mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+        mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
     }
     __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
     if (!waited) {  // lanes 1..31, a split without extension stages, or a producer that gave up
@@ -178,7 +171,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         umma_commit(&empty[s]);
       }
       umma_commit(accf);
-      if (aborted) mbar_wait_drain(accf, 0);
+      if (aborted) mbar_drain(accf, 0, a.status);
     }
     __syncwarp();
     grid_dependency_wait();
@@ -444,7 +437,7 @@ __global__ void __launch_bounds__(192, 1)
         issued = t + 1;
       }
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
-        mbar_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+        mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
     }
     __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
     if (!waited) {  // lanes 1..31, or a producer that gave up
@@ -482,7 +475,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(&empty[s]);
       }
       umma_commit(accf);
-      if (aborted) mbar_wait_drain(accf, 0);
+      if (aborted) mbar_drain(accf, 0, a.status);
     }
     __syncwarp();
     grid_dependency_wait();

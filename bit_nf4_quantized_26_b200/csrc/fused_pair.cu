@@ -25,13 +25,6 @@ namespace qnf4 {
 
 namespace {
 
-__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
-  }
-}
-
 struct PlanPair {
   static constexpr uint32_t kBq = 128 * 64;  // 128 tokens x 32 bf16, one accumulator's half
   static constexpr uint32_t kB = 2 * kBq;    // 16 KB
@@ -149,8 +142,8 @@ __global__ void __launch_bounds__(192, 1)
       // Leave nothing in flight into this CTA's shared memory: codes land on the
       // local barrier; the leader also waits for the pair's tiles.
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t) {
-        if (t < nmain) wait_drain(&cfull[t % P::kStages], (t / P::kStages) & 1);
-        if (rank == 0) wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+        if (t < nmain) mbar_drain(&cfull[t % P::kStages], (t / P::kStages) & 1, a.status);
+        if (rank == 0) mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
       }
     }
     __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
@@ -190,7 +183,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit_pair(&empty[s], 0x3);
       }
       umma_commit_pair(accf, 0x3);
-      if (aborted) wait_drain(accf, 0);
+      if (aborted) mbar_drain(accf, 0, a.status);
     }
     __syncwarp();
     grid_dependency_wait();

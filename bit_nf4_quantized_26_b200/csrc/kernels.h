@@ -13,6 +13,13 @@ namespace qnf4 {
 // Whether launches use programmatic dependent launch (QLORA_PDL=0 disables).
 bool pdl_enabled();
 
+// Every check qlora_linear_fwd makes before it looks at the workspace, in the
+// same order (shape, output dtype, M == 0 -> QLORA_OK, null pointers, weight
+// pointers, alignment).  Xa is the adapter's input (X, or X after dropout).
+qlora_status check_fwd_args(const uint16_t* X, const uint16_t* Xa, int64_t M, const nf4_weight& W,
+                            const uint16_t* A, const uint16_t* B, int32_t r, const void* Y, int32_t y_dtype,
+                            const float* U_out, const int32_t* d_status);
+
 // cudaLaunchKernelEx with programmatic stream serialisation (when enabled)
 // and an optional thread-block cluster shape.
 template <typename... KArgs, typename... Args>

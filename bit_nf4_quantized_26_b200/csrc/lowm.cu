@@ -68,13 +68,6 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
-__device__ __forceinline__ void lowm_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
-  }
-}
-
 __device__ __forceinline__ int64_t unit_start(int64_t c, int64_t units, int ctas) { return c * units / ctas; }
 
 // CTA whose range holds unit u: the largest c with floor(c * L / P) <= u.
@@ -293,7 +286,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   // (after a normal run every stage's last phase has completed already).
   if (issuer) {
     for (int i = max(0, issued - P::kStages); i < issued; ++i)
-      lowm_drain(&full[i % P::kStages], (i / P::kStages) & 1);
+      mbar_drain(&full[i % P::kStages], (i / P::kStages) & 1, a.status);
   }
 }
 

@@ -49,12 +49,12 @@ extern "C" {
 qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A,
                                       const uint16_t* B, int32_t r, float s, void* Y, int32_t y_dtype,
                                       float* U_out, int32_t* d_status, void* stream) {
-  const int64_t N = W.n_out, K = W.k_in;
-  if (M < 0 || N < 64 || K < 64 || N % 64 != 0 || K % 64 != 0 || r < 16 || r > 64 || r % 16 != 0)
-    return QLORA_ERR_SHAPE;
+  // The same checks, in the same order, as qlora_linear_fwd; then, in place
+  // of its workspace check, the problem must fit the fixed scratch.  Nothing
+  // is enqueued when a check fails.
+  if (qlora_status st = qnf4::check_fwd_args(X, X, M, W, A, B, r, Y, y_dtype, U_out, d_status)) return st;
   if (M == 0) return QLORA_OK;
-  // The problem must fit the fixed scratch; nothing is enqueued otherwise.
-  if (qlora_fwd_workspace_size(M, N, K, r) > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (qlora_fwd_workspace_size(M, W.n_out, W.k_in, r) > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (qlora_status st = scratch_for_current_device(&scratch)) return st;
   return qlora_linear_fwd(X, M, W, A, B, r, s, Y, y_dtype, U_out, scratch, kNoAllocScratchBytes, d_status,

@@ -241,29 +241,32 @@ cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const
 
 // ------------------------------------------------------- bounded-wait self-test
 //
-// The wait below is the kernels' bounded wait (try_wait on the barrier's
-// phase, %globaltimer deadline) with a caller-chosen limit; the barrier
-// expects one arrival that never comes, so the limit always passes.
+// Two warps wait on one shared-memory mbarrier that expects an arrival that
+// never comes, through the same waits the kernels' roles use, with the
+// kernels' WaitCtx (CTA abort flag, device status word) and a caller-chosen
+// limit in place of the 2 s: warp 0 as a producer / MMA issuer does (lane 0
+// polls, mbar_wait_warp), warp 1 as the dequantisers do (every lane polls,
+// mbar_wait_all).  Whichever runs out first records QLORA_DEV_TIMEOUT and
+// raises the abort flag; the other then gives up on the flag.  Each warp whose
+// wait returned false adds 1 to status[1].
 __global__ void selftest_timeout_kernel(int32_t* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
+  __shared__ int abort_flag;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
+    abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(&bar, 0)) {
-      if (global_timer_ns() - t0 > limit_ns) {
-        atomicOr(status, QLORA_DEV_TIMEOUT);
-        break;
-      }
-    }
-  }
+  WaitCtx wc{&abort_flag, status};
+  wc.limit_ns = limit_ns;
+  const int warp = threadIdx.x >> 5;
+  const bool ok = warp == 0 ? mbar_wait_warp(&bar, 0, wc) : mbar_wait_all(&bar, 0, wc);
+  if ((threadIdx.x & 31) == 0 && !ok) atomicAdd(status + 1, 1);
 }
 
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t stream) {
-  selftest_timeout_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  selftest_timeout_kernel<<<1, 64, 0, stream>>>(status, limit_ns);
   return cudaGetLastError();
 }
 

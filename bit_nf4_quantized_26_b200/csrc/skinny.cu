@@ -21,13 +21,6 @@
 
 namespace qnf4 {
 
-__device__ __forceinline__ void sk_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) return;
-  }
-}
-
 // Shared-memory ring per mode: about 97 KB, so two CTAs fit on an SM (each
 // with three or four 24-32 KB stages in flight).
 template <int MODE>
@@ -140,7 +133,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         issued = t + 1;
       }
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t)
-        sk_wait_drain(&full[t % P::kStages], (t / P::kStages) & 1);
+        mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -164,7 +157,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         umma_commit(&empty[s]);
       }
       umma_commit(accf);
-      if (aborted) sk_wait_drain(accf, 0);
+      if (aborted) mbar_drain(accf, 0, a.status);
     }
   } else {
     // ------------------------------------------------ TMEM -> own partial tile

@@ -61,8 +61,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // timeout the waiter records QLORA_DEV_TIMEOUT, raises the CTA's abort flag so
 // the other roles stop waiting too, and returns false.
 struct WaitCtx {
-  volatile int* abort_flag;  // shared memory
-  int32_t* status;           // global memory, may be null
+  volatile int* abort_flag;              // shared memory
+  int32_t* status;                       // global memory, may be null
+  uint64_t limit_ns = kWaitTimeoutNs;    // give up after this long
 };
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
@@ -72,13 +73,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > w.limit_ns) {
         *w.abort_flag = 1;
         if (w.status) atomicOr(w.status, QLORA_DEV_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// Wait for copies or MMAs already in flight before a CTA that gave up leaves
+// (or frees the TMEM they write): bounded like every other wait, ignoring the
+// abort flag.  A drain that runs out records QLORA_DEV_TIMEOUT and returns
+// false; the state of the memory those operations write is then unknown, but
+// the CTA still releases its TMEM, which it must do before it exits.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32_t* status) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
 }
 
 // Warp-uniform wait: lane 0 polls, the outcome is broadcast, so the whole warp
@@ -291,7 +308,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > w.limit_ns) {
         *w.abort_flag = 1;
         if (w.status) atomicOr(w.status, QLORA_DEV_TIMEOUT);
         return false;

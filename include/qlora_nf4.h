@@ -78,7 +78,8 @@ typedef enum {
   QLORA_ERR_TIMEOUT = 6,    /* (reserved for host-visible timeout reports)     */
   QLORA_ERR_CUDA = 7,       /* a CUDA runtime/driver call failed               */
   QLORA_ERR_ARCH = 8,       /* current device is not sm_100                    */
-  QLORA_ERR_DTYPE = 9       /* unknown output dtype code                       */
+  QLORA_ERR_DTYPE = 9,      /* unknown output dtype code                       */
+  QLORA_ERR_INTERNAL = 10   /* the library's constant tables failed a check    */
 } qlora_status;
 
 /* Device status bits OR-ed into d_status by the kernels. */
@@ -249,21 +250,28 @@ QLORA_API void nf4_levels(float out[16]);
  * allocated).  qlora_profile_collect waits for the recorded events, writes up
  * to `capacity` (kernel id, milliseconds) pairs in launch order, clears the
  * record list and returns the number of records (or -1 on a CUDA error).
- * qlora_kernel_name maps an id to a static name.  Not thread-safe with
- * respect to concurrent launches from several host threads.
+ * qlora_kernel_name maps an id to a static name.  While enabled, the
+ * backward's dB and dA kernels run on the caller's stream instead of beside
+ * the dX GEMM, so each event pair times one kernel alone.  Not thread-safe
+ * with respect to concurrent launches from several host threads.
  */
 QLORA_API void qlora_profile_enable(int32_t enable);
 QLORA_API int32_t qlora_profile_collect(int32_t* kernel_ids, float* ms, int32_t capacity);
 QLORA_API const char* qlora_kernel_name(int32_t kernel_id);
 
 /*
- * qlora_selftest_timeout — exercises the bounded-wait path every kernel uses
- * (diagnostics).  Launches one CTA whose thread waits on a shared-memory
- * mbarrier that nothing completes, polling it with the kernels' bounded wait
- * but a time limit of `limit_ns` nanoseconds (1e3 .. 2e9) instead of the
- * kernels' 2 s; when the limit passes it ORs QLORA_DEV_TIMEOUT into
- * *d_status (required) and returns, leaving the context usable.  Nothing
- * faults, traps or hangs.  limit_ns out of range returns QLORA_ERR_SHAPE.
+ * qlora_selftest_timeout — exercises the bounded waits every kernel uses
+ * (diagnostics).  Launches one CTA of two warps that wait on a shared-memory
+ * mbarrier that nothing completes, through the kernels' own wait functions
+ * and their CTA abort flag, with a time limit of `limit_ns` nanoseconds
+ * (1e3 .. 2e9) in place of the kernels' 2 s: warp 0 the way a producer or
+ * MMA issuer waits (lane 0 polls), warp 1 the way the dequantiser warps wait
+ * (every lane polls).  The first to run out ORs QLORA_DEV_TIMEOUT into
+ * d_status[0] and raises the abort flag, on which the other gives up; each
+ * warp whose wait gave up adds 1 to d_status[1] (so 2 is expected).
+ * d_status is required: int32[2], zeroed by the caller.  The kernel returns
+ * and the context stays usable; nothing faults, traps or hangs.  limit_ns out
+ * of range returns QLORA_ERR_SHAPE.
  */
 QLORA_API qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_ns, void* stream);
 

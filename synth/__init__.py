@@ -152,3 +152,34 @@ def bf16_bits(t):
 def random_bf16_bits(shape, seed, std=1.0):
     """Convenience: seeded N(0, std) draws as numpy bf16 bit patterns."""
     return bf16_bits(normal_bf16(shape, std, seed))
+
+
+# Which input each linear of the decoder layer reads: q, k and v read the
+# same normalised hidden state, gate and up the same MLP input; o reads the
+# attention output and down the MLP activation.
+LAYER_INPUT_OF = ("attn", "attn", "attn", "o", "mlp", "mlp", "down")
+LAYER_INPUT_WIDTH = {"attn": 4096, "o": 4096, "mlp": 4096, "down": 11008}
+
+
+def decoder_layer_params(r, seed=0, device="cpu", linears=LLAMA7B_LAYER):
+    """Frozen weights and adapters of one decoder layer's linears, the same on
+    every data-parallel rank: a list of {"W", "A", "B"} (bf16), in layer
+    order.  W ~ N(0, 0.02), A ~ N(0, 1/in) (std), B ~ N(0, 0.01)."""
+    base = int(seed) * 1000
+    out = []
+    for i, lin in enumerate(linears):
+        out.append({"W": weight_bf16(lin.n_out, lin.k_in, base + 10 * i + 1, device=device),
+                    "A": normal_bf16((r, lin.k_in), 1.0 / lin.k_in, base + 10 * i + 2, device),
+                    "B": normal_bf16((lin.n_out, r), B_STD, base + 10 * i + 3, device)})
+    return out
+
+
+def decoder_layer_activations(m_tokens, rank=0, seed=0, device="cpu", linears=LLAMA7B_LAYER):
+    """One rank's batch for the layer's linears: the four distinct inputs
+    {"attn", "o", "mlp", "down"} [m, in] and one upstream gradient per
+    linear [m, out], all N(0, 1) bf16, drawn from seeds derived from ``rank``."""
+    base = (int(seed) + 1 + int(rank)) * 100000
+    X = {name: normal_bf16((m_tokens, width), 1.0, base + j, device)
+         for j, (name, width) in enumerate(LAYER_INPUT_WIDTH.items())}
+    dY = [normal_bf16((m_tokens, lin.n_out), 1.0, base + 100 + i, device) for i, lin in enumerate(linears)]
+    return X, dY

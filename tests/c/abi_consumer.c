@@ -36,7 +36,7 @@ int main(void) {
 
   /* Status strings. */
   CHECK(strcmp(qlora_strerror(QLORA_OK), "ok") == 0);
-  for (int s = 0; s <= QLORA_ERR_DTYPE; ++s) CHECK(qlora_strerror((qlora_status)s) != NULL);
+  for (int s = 0; s <= QLORA_ERR_INTERNAL; ++s) CHECK(qlora_strerror((qlora_status)s) != NULL);
 
   /* Argument checks that return before any device work. */
   void* p = (void*)(uintptr_t)256; /* 16-byte aligned, never dereferenced */
@@ -73,6 +73,12 @@ int main(void) {
                                  NULL, NULL) == QLORA_ERR_SHAPE);
   CHECK(qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) ==
         qlora_bwd_workspace_size(4096, 4096, 4096, 64) + (size_t)4096 * 4096 * 4);
+  /* Allocation-free forward: the forward's checks, then the fixed-scratch limit. */
+  nf4_weight w128 = {(const uint8_t*)p, (const uint8_t*)p, (const float*)p, 128, 128};
+  CHECK(qlora_linear_fwd_noalloc(p, 70000, w128, p, p, 64, 0.25f, p, QLORA_DTYPE_BF16, p, NULL, NULL) ==
+        QLORA_ERR_WORKSPACE);
+  CHECK(qlora_linear_fwd_noalloc(p, 64, w, p, p, 8, 0.25f, p, QLORA_DTYPE_BF16, p, NULL, NULL) == QLORA_ERR_SHAPE);
+  CHECK(qlora_linear_fwd_noalloc(p, 0, w, p, p, 16, 0.25f, p, 7, p, NULL, NULL) == QLORA_ERR_DTYPE);
   /* Bounded-wait self-test: argument checks only (no device here). */
   CHECK(qlora_selftest_timeout(NULL, 5000000, NULL) == QLORA_ERR_NULL);
   CHECK(qlora_selftest_timeout(p, 10, NULL) == QLORA_ERR_SHAPE);

@@ -42,7 +42,7 @@ def test_library_levels_equal_oracle_codebook():
 
 
 def test_strerror():
-    for code in range(10):
+    for code in range(11):
         assert isinstance(q.qlora_strerror(code), str) and q.qlora_strerror(code)
     assert q.qlora_strerror(0) == "ok"
 
@@ -94,6 +94,27 @@ def test_fwd_argument_errors():
     assert _fwd(ws=None) == WS
     assert _fwd(wsb=16) == WS
     assert _fwd(M=0, X=None, Y=None, U=None, ws=None) == OK   # no-op
+
+
+def _noalloc(X=FAKE, M=64, W=None, A=FAKE, B=FAKE, r=64, Y=FAKE, ydt=0, U=FAKE, status=None):
+    W = _w() if W is None else W
+    return q.raw().qlora_linear_fwd_noalloc(X, M, W, A, B, r, 0.25, Y, ydt, U, status, None)
+
+
+def test_noalloc_argument_errors_match_the_forward():
+    """The allocation-free forward makes the forward's checks in the same
+    order, and refuses a problem whose workspace exceeds its fixed 16 MiB
+    scratch, all before touching a device."""
+    wsmall = _w(n=128, k=128)
+    assert q.qlora_fwd_workspace_size(70000, 128, 128, 64) > 16 << 20
+    assert _noalloc(M=70000, W=wsmall) == WS
+    assert _noalloc(r=8) == SHAPE
+    assert _noalloc(M=1 << 31) == SHAPE
+    assert _noalloc(M=0, ydt=7) == DTYPE == _fwd(M=0, ydt=7)
+    assert _noalloc(M=0, X=None, Y=None, U=None) == OK
+    assert _noalloc(X=None) == NULL
+    assert _noalloc(X=FAKE + 8) == ALIGN
+    assert _noalloc(W=_w(codes=None)) == NULL
 
 
 def test_bwd_argument_errors():

@@ -193,5 +193,17 @@ def test_c5_forward_sweep(N, K, M):
     _check_sampled(N, K, M, 64, 0.25, 5, nrows=32, bwd=False)
 
 
-def test_c5_forward_largest_m():
-    _check_sampled(22016, 8192, 16384, 64, 0.25, 6, nrows=16, bwd=False)
+@pytest.mark.parametrize("N,K", [(22016, 8192), (8192, 22016)])
+def test_c5_forward_largest_m(N, K):
+    """65B-shaped up (8192 -> 22016) and down (22016 -> 8192) at 16384 tokens."""
+    _check_sampled(N, K, 16384, 64, 0.25, 6, nrows=16, bwd=False)
+
+
+@pytest.mark.parametrize("index", range(len(synth.LLAMA7B_LAYER)))
+def test_c4_decoder_layer_linear(index):
+    """c4: each of the seven linears of the LLaMA-7B-shaped decoder layer (q, k,
+    v, o 4096x4096; gate, up 4096->11008; down 11008->4096) at 8 x 2048 =
+    16384 tokens, r=64, alpha=16, forward and backward: 32 sampled token rows
+    of Y and dX against the oracle, and the full dA and dB."""
+    lin = synth.LLAMA7B_LAYER[index]
+    _check_sampled(lin.n_out, lin.k_in, 16384, 64, 0.25, 40 + index, nrows=32)

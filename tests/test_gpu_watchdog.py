@@ -1,6 +1,8 @@
-"""Failure detection without a GPU fault: the bounded wait every kernel uses
-runs out against a barrier that nothing completes, reports QLORA_DEV_TIMEOUT
-in the device status word, and the context stays usable."""
+"""Failure detection without a GPU fault: the bounded waits every kernel uses
+(lane 0 polling for a warp, and every lane polling) run out against a barrier
+that nothing completes; the first reports QLORA_DEV_TIMEOUT in the device
+status word and raises the CTA's abort flag, the other gives up on the flag,
+and the context stays usable."""
 
 import numpy as np
 import pytest
@@ -18,6 +20,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     q.qlora_selftest_timeout(status, 5_000_000)  # 5 ms limit
     torch.cuda.synchronize()
     assert int(status[0]) & q.DEV_TIMEOUT
+    assert int(status[1]) == 2  # both waiting warps gave up
     # the same context still runs kernels correctly
     w = synth.weight_bf16(64, 512, seed=2).cuda()
     W = q.quantize_weight(w)
