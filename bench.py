@@ -197,53 +197,78 @@ def cpu_oracle_nf4_rates(n_rows=4096, k=8192, seed=0):
 
 # ------------------------------------------------------------ the layer step
 
+# The decoder layer's linears by shared input: q/k/v read the attention
+# input, gate/up the MLP input; o and down read their own.
+LAYER_GROUPS = (("attn", (0, 1, 2)), ("o", (3,)), ("mlp", (4, 5)), ("down", (6,)))
+
+
 class LayerStep:
     """The decoder layer's seven QLoRA linears on one GPU: buffers, and the
-    quantise / forward / backward / optimizer phases of one training step."""
+    quantise / forward / backward / optimizer phases of one training step.
+    grouped: the linears that share an input run as one grouped call (their
+    weights, adapters, outputs and gradients stacked along the output
+    dimension, their input gradient summed); otherwise every linear is its
+    own call."""
 
-    def __init__(self, lib, synth, torch, dev, M, rank=0, world=1, grouped=False):
+    def __init__(self, lib, synth, torch, dev, M, rank=0, world=1, grouped=True):
         self.lib, self.torch, self.dev = lib, torch, dev
         self.M, self.r, self.s = M, RANK_R, ALPHA / RANK_R
         self.world = world
         self.grouped = grouped and hasattr(lib, "qlora_group_fwd")
         self.lins = synth.LLAMA7B_LAYER
-        self.input_of = synth.LAYER_INPUT_OF
         r = self.r
         params = synth.decoder_layer_params(r, seed=0, device=dev)
-        self.X, self.dY = synth.decoder_layer_activations(M, rank=rank, device=dev)
-        self.Wb = [p["W"] for p in params]
-        self.W, self.param, self.grad, self.A, self.B, self.dA, self.dB = [], [], [], [], [], [], []
-        self.U, self.Y, self.dX, self.opt = [], [], [], []
-        for i, lin in enumerate(self.lins):
-            N, K = lin.n_out, lin.k_in
-            nc, nb, ns = lib.nf4_sizes(N * K)
-            self.W.append(lib.NF4Weight(torch.empty(nc, dtype=torch.uint8, device=dev),
-                                        torch.empty(nb, dtype=torch.uint8, device=dev),
-                                        torch.empty(ns, dtype=torch.float32, device=dev), N, K))
-            # A and B of a linear are views of one flat bf16 parameter; dA and
-            # dB views of one flat fp32 gradient (one all-reduce, one
-            # optimizer call per linear).
-            p = torch.empty(r * K + N * r, dtype=torch.bfloat16, device=dev)
-            p[: r * K].copy_(params[i]["A"].reshape(-1))
-            p[r * K:].copy_(params[i]["B"].reshape(-1))
-            g = torch.empty(r * K + N * r, dtype=torch.float32, device=dev)
-            self.param.append(p)
-            self.grad.append(g)
-            self.A.append(p[: r * K].view(r, K))
-            self.B.append(p[r * K:].view(N, r))
-            self.dA.append(g[: r * K].view(r, K))
-            self.dB.append(g[r * K:].view(N, r))
-            self.U.append(torch.empty((M, r), dtype=torch.float32, device=dev))
-            self.Y.append(torch.empty((M, N), dtype=torch.bfloat16, device=dev))
-            self.dX.append(torch.empty((M, K), dtype=torch.bfloat16, device=dev))
-            self.opt.append(lib.AdamW8State(p.numel(), paged=False, device=dev))
-        kmax = max(lin.k_in for lin in self.lins)
-        nmax = max(lin.n_out for lin in self.lins)
-        self.ws_f = torch.empty(max(lib.qlora_fwd_workspace_size(M, nmax, kmax, r), 16), dtype=torch.uint8, device=dev)
-        self.ws_b = torch.empty(max(lib.qlora_bwd_workspace_size(M, nmax, kmax, r), 16), dtype=torch.uint8, device=dev)
+        X, dY = synth.decoder_layer_activations(M, rank=rank, device=dev)
+        self.X = X
+        if self.grouped:
+            units = [(name, idx) for name, idx in LAYER_GROUPS]
+        else:
+            units = [(synth.LAYER_INPUT_OF[i], (i,)) for i in range(len(self.lins))]
+        self.units = []
+        for name, idx in units:
+            K = self.lins[idx[0]].k_in
+            ns = [self.lins[i].n_out for i in idx]
+            N = sum(ns)
+            G = len(idx)
+            u = {"x": name, "members": ns, "G": G, "N": N, "K": K}
+            u["Wb"] = torch.cat([params[i]["W"] for i in idx], 0).contiguous() if G > 1 else params[idx[0]]["W"]
+            nc, nb, nsz = lib.nf4_sizes(N * K)
+            u["W"] = lib.NF4Weight(torch.empty(nc, dtype=torch.uint8, device=dev),
+                                   torch.empty(nb, dtype=torch.uint8, device=dev),
+                                   torch.empty(nsz, dtype=torch.float32, device=dev), N, K)
+            # The stacked adapters A [G r, K] and B [N, r] are views of one flat
+            # bf16 parameter, dA and dB of one flat fp32 gradient (one
+            # all-reduce and one optimizer call per unit).
+            p = torch.empty(G * r * K + N * r, dtype=torch.bfloat16, device=dev)
+            p[: G * r * K].copy_(torch.cat([params[i]["A"] for i in idx], 0).reshape(-1))
+            p[G * r * K:].copy_(torch.cat([params[i]["B"] for i in idx], 0).reshape(-1))
+            gr = torch.empty_like(p, dtype=torch.float32)
+            u.update(param=p, grad=gr, A=p[: G * r * K].view(G * r, K), B=p[G * r * K:].view(N, r),
+                     dA=gr[: G * r * K].view(G * r, K), dB=gr[G * r * K:].view(N, r))
+            u["dY"] = torch.cat([dY[i] for i in idx], 1).contiguous() if G > 1 else dY[idx[0]]
+            u["U"] = torch.empty((M, G * r), dtype=torch.float32, device=dev)
+            u["Y"] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            u["dX"] = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            u["opt"] = lib.AdamW8State(p.numel(), paged=False, device=dev)
+            self.units.append(u)
+        del params, dY
+        wsf = max(lib.qlora_group_fwd_workspace_size(M, u["N"], u["K"], u["G"], r) if self.grouped else
+                  lib.qlora_fwd_workspace_size(M, u["N"], u["K"], r) for u in self.units)
+        wsb = max(lib.qlora_group_bwd_workspace_size(M, u["N"], u["K"], u["G"], r) if self.grouped else
+                  lib.qlora_bwd_workspace_size(M, u["N"], u["K"], r) for u in self.units)
+        self.ws_f = torch.empty(max(wsf, 16), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         self.t = 0
         self.pending = []
+
+    @property
+    def dY(self):
+        return [u["dY"] for u in self.units]
+
+    @property
+    def grad(self):
+        return [u["grad"] for u in self.units]
 
     def flops(self):
         return sum(flops_fwd_bwd(self.M, lin.n_out, lin.k_in, self.r) for lin in self.lins)
@@ -260,41 +285,49 @@ class LayerStep:
         return tot
 
     def quantize(self):
-        lib = self.lib
-        for i in range(len(self.lins)):
-            W = self.W[i]
-            lib.nf4_quantize(self.Wb[i].reshape(-1), W.codes, W.c8, W.s2, status=self.status)
+        for u in self.units:
+            W = u["W"]
+            self.lib.nf4_quantize(u["Wb"].reshape(-1), W.codes, W.c8, W.s2, status=self.status)
 
     def forward(self):
         lib = self.lib
-        for i in range(len(self.lins)):
-            lib.qlora_linear_fwd(self.X[self.input_of[i]], self.W[i], self.A[i], self.B[i], self.s, Y=self.Y[i],
-                                 U=self.U[i], ws=self.ws_f, status=self.status)
+        for u in self.units:
+            X = self.X[u["x"]]
+            if self.grouped:
+                lib.qlora_group_fwd(X, u["W"], u["members"], u["A"], u["B"], self.s, Y=u["Y"], U=u["U"],
+                                    ws=self.ws_f, status=self.status)
+            else:
+                lib.qlora_linear_fwd(X, u["W"], u["A"], u["B"], self.s, Y=u["Y"], U=u["U"], ws=self.ws_f,
+                                     status=self.status)
 
     def backward(self):
         lib = self.lib
-        for i in reversed(range(len(self.lins))):
-            lib.qlora_linear_bwd(self.dY[i], self.X[self.input_of[i]], self.U[i], self.W[i], self.A[i], self.B[i],
-                                 self.s, dX=self.dX[i], dA=self.dA[i], dB=self.dB[i], ws=self.ws_b,
-                                 status=self.status)
-            self._reduce(i)
+        for i in reversed(range(len(self.units))):
+            u = self.units[i]
+            X = self.X[u["x"]]
+            if self.grouped:
+                lib.qlora_group_bwd(u["dY"], X, u["U"], u["W"], u["members"], u["A"], u["B"], self.s, dX=u["dX"],
+                                    dA=u["dA"], dB=u["dB"], ws=self.ws_b, status=self.status)
+            else:
+                lib.qlora_linear_bwd(u["dY"], X, u["U"], u["W"], u["A"], u["B"], self.s, dX=u["dX"], dA=u["dA"],
+                                     dB=u["dB"], ws=self.ws_b, status=self.status)
+            self._reduce(u)
 
-    def _reduce(self, i):
+    def _reduce(self, u):
         # Sum of the adapter gradients over ranks, issued right after this
-        # linear's backward: NCCL's stream waits for it and then runs beside
-        # the next linear's backward.
+        # unit's backward: NCCL's stream waits for it and then runs beside
+        # the next unit's backward.
         if self.world > 1:
             import torch.distributed as dist
-            self.pending.append(dist.all_reduce(self.grad[i], async_op=True))
+            self.pending.append(dist.all_reduce(u["grad"], async_op=True))
 
     def optimizer(self):
         for h in self.pending:
             h.wait()
         self.pending = []
         self.t += 1
-        for i in range(len(self.lins)):
-            self.lib.qlora_adamw8_step(self.param[i], self.grad[i], self.opt[i], lr=2e-4, step=self.t,
-                                       status=self.status)
+        for u in self.units:
+            self.lib.qlora_adamw8_step(u["param"], u["grad"], u["opt"], lr=2e-4, step=self.t, status=self.status)
 
     def step(self):
         self.quantize()
@@ -303,8 +336,8 @@ class LayerStep:
         self.optimizer()
 
     def close(self):
-        for o in self.opt:
-            o.close()
+        for u in self.units:
+            u["opt"].close()
 
 
 def time_steps(torch, step, stream, steps, flush, dist=None):
@@ -746,10 +779,22 @@ def run_ours(args, rank, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e = float(t.item())
     fl = layer.flops()
+    grouped = layer.grouped
     layer.close()
     del layer, host_in, host_out
 
     extras = {}
+    if rank == 0 and not args.no_sweep and grouped:
+        # The same step with every linear its own call (no grouping).
+        flat = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=False)
+        for _ in range(3):
+            flat.step()
+        ts = time_steps(torch, flat.step, stream, args.steps, flush)
+        fms = float(np.mean(ts))
+        extras["per_linear_step"] = {"ms_per_step": fms, "tflops": fl / (fms * 1e-3) / 1e12,
+                                     "grouped_ms_per_step": ms, "grouped_speedup": fms / ms}
+        flat.close()
+        del flat
     if rank == 0 and not args.no_sweep:
         quant_gbs, dequant_gbs = nf4_stream_timing(lib, synth, torch, dev, flush)
         extras["nf4_quantize_gbs"] = quant_gbs
@@ -780,7 +825,7 @@ def run_ours(args, rank, world):
             "config": {"workload": WORKLOAD_NAME, "tokens_per_gpu": M, "r": RANK_R, "alpha": ALPHA,
                        "linears": [[lin.name, lin.n_out, lin.k_in] for lin in synth.LLAMA7B_LAYER],
                        "parallelism": f"dp{world}", "global_batch_tokens": M * world,
-                       "grouped_projections": bool(getattr(lib, "qlora_group_fwd", None)) and not args.no_group,
+                       "grouped_projections": grouped,
                        "step": "nf4_quantize x7 + forward x7 + backward x7 (+ dA/dB all-reduce per linear if N>1) "
                                "+ 8-bit AdamW on every adapter",
                        "flops_per_step_per_gpu": fl,

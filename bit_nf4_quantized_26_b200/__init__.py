@@ -412,3 +412,83 @@ def qlora_selftest_timeout(status, limit_ns, stream=None):
     """Run the kernels' bounded wait against a barrier nothing completes, with
     a ``limit_ns`` limit; sets DEV_TIMEOUT in the int32 device tensor ``status``."""
     _check(_lib.qlora_selftest_timeout(_ptr(status), int(limit_ns), _stream(stream)), "qlora_selftest_timeout")
+
+
+# ------------------------------------------------------ grouped projections
+# (include/qlora_nf4.h: linears sharing one input, stacked along the outputs)
+
+_lib.qlora_group_fwd_workspace_size.argtypes = [_I64, _I64, _I64, _I32, _I32]
+_lib.qlora_group_fwd_workspace_size.restype = _SZ
+_lib.qlora_group_bwd_workspace_size.argtypes = [_I64, _I64, _I64, _I32, _I32]
+_lib.qlora_group_bwd_workspace_size.restype = _SZ
+_lib.qlora_group_fwd.argtypes = [_P, _I64, _NF4Weight, _I32, _P, _P, _P, _I32, ctypes.c_float, _P, _I32, _P, _P,
+                                 _SZ, _P, _P]
+_lib.qlora_group_fwd.restype = ctypes.c_int
+_lib.qlora_group_bwd.argtypes = [_P, _P, _P, _I64, _NF4Weight, _I32, _P, _P, _P, _I32, ctypes.c_float, _P, _I32,
+                                 _P, _P, _P, _SZ, _P, _P]
+_lib.qlora_group_bwd.restype = ctypes.c_int
+
+EXPORTED = EXPORTED + ("qlora_group_fwd_workspace_size", "qlora_group_bwd_workspace_size", "qlora_group_fwd",
+                       "qlora_group_bwd")
+
+
+def qlora_group_fwd_workspace_size(M, N, K, members, r):
+    return int(_lib.qlora_group_fwd_workspace_size(M, N, K, members, r))
+
+
+def qlora_group_bwd_workspace_size(M, N, K, members, r):
+    return int(_lib.qlora_group_bwd_workspace_size(M, N, K, members, r))
+
+
+def _members(n_member):
+    arr = (ctypes.c_int64 * len(n_member))(*[int(n) for n in n_member])
+    return len(n_member), arr
+
+
+def quantize_group(weights, stream=None):
+    """NF4-quantise the members of a group (bf16 [n_g, K] each) as one stacked
+    weight; returns ``(NF4Weight [sum n_g, K], [n_g ...])``."""
+    stacked = torch.cat([w.reshape(w.shape[0], -1) for w in weights], 0).contiguous()
+    return quantize_weight(stacked, stream=stream), [int(w.shape[0]) for w in weights]
+
+
+def qlora_group_fwd(X, W, n_member, A, B, s, y_dtype=DTYPE_BF16, Y=None, U=None, ws=None, status=None, stream=None):
+    """Forward of a group of linears sharing ``X``: W stacked [N, K], A [G r, K],
+    B [N, r]; returns ``(Y [M, N], U [M, G r])``."""
+    M = X.shape[0]
+    G, arr = _members(n_member)
+    N, K, r = int(W.n_out), int(W.k_in), A.shape[0] // G
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32 if y_dtype == DTYPE_F32 else torch.bfloat16, device=dev)
+    if U is None:
+        U = torch.empty((M, G * r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(max(qlora_group_fwd_workspace_size(M, N, K, G, r), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.qlora_group_fwd(_ptr(X), M, _weight(W), G, ctypes.cast(arr, _P), _ptr(A), _ptr(B), r, float(s),
+                                _ptr(Y), y_dtype, _ptr(U), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)),
+           "qlora_group_fwd")
+    return Y, U
+
+
+def qlora_group_bwd(dY, X, U, W, n_member, A, B, s, dx_dtype=DTYPE_BF16, dX=None, dA=None, dB=None, ws=None,
+                    status=None, stream=None):
+    """Backward of :func:`qlora_group_fwd`; returns ``(dX [M, K] summed over the
+    members, dA [G r, K], dB [N, r])``."""
+    M = X.shape[0]
+    G, arr = _members(n_member)
+    N, K, r = int(W.n_out), int(W.k_in), A.shape[0] // G
+    dev = X.device
+    if dX is None:
+        dX = torch.empty((M, K), dtype=torch.float32 if dx_dtype == DTYPE_F32 else torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((G * r, K), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(max(qlora_group_bwd_workspace_size(M, N, K, G, r), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.qlora_group_bwd(_ptr(dY), _ptr(X), _ptr(U), M, _weight(W), G, ctypes.cast(arr, _P), _ptr(A),
+                                _ptr(B), r, float(s), _ptr(dX), dx_dtype, _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                                _ptr(status), _stream(stream)),
+           "qlora_group_bwd")
+    return dX, dA, dB

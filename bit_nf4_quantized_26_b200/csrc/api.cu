@@ -359,13 +359,13 @@ struct FwdPlan {
 
 // Few tokens: persistent CTAs (two per SM, and at least one per row tile so
 // that no CTA's range spans more than two tiles) over (tiles + atiles) * kc
-// units.
-FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r) {
+// units.  G members: the rows of A are the G members' adapters stacked.
+FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   FwdPlan p{};
   p.low = true;
   p.low_mpad = M <= 8 ? 8 : (M <= 16 ? 16 : 32);
   p.low_tiles = static_cast<int>(cdiv(N, kLowmRows));
-  p.low_atiles = static_cast<int>(cdiv(r, kLowmARows));
+  p.low_atiles = static_cast<int>(cdiv(static_cast<int64_t>(G) * r, kLowmARows));
   p.low_kc = static_cast<int>(cdiv(K / 64, 4));
   const int64_t all_tiles = p.low_tiles + p.low_atiles;
   const int64_t units = all_tiles * p.low_kc;
@@ -375,11 +375,11 @@ FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r) {
   return p;
 }
 
-FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
-  if (M <= kLowmMaxM) return plan_fwd_low(M, N, K, r);
+FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
+  if (M <= kLowmMaxM) return plan_fwd_low(M, N, K, r, G);
   FwdPlan p{};
   const int64_t kst = K / 64;
-  split_plan(cdiv(M, 128), kst, 4, 2 * kSms, p.s_down, p.per_down);
+  split_plan(cdiv(M, 128) * G, kst, 4, 2 * kSms, p.s_down, p.per_down);
   if (M > kWideM) {
     // The wide GEMM needs U only in its last stages and does not wait for it
     // before then, so U = X A^T runs beside the GEMM's main loop: one CTA per
@@ -406,7 +406,7 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r) {
   }
   size_t off = 0;
   p.off_ucat = off;
-  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
   p.off_pfwd = off;
   if (p.s_fwd > 1) off += align256(static_cast<size_t>(p.s_fwd) * M * N * 4);
   p.total = off;
@@ -418,25 +418,82 @@ struct BwdPlan {
   size_t off_sucat, off_ducat, total;
 };
 
-BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r) {
+// G members, the longest with n_max outputs (the dU contraction); sizes
+// depend on M, G and r only.
+BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r, int G, int64_t n_max) {
   BwdPlan p{};
-  split_plan(cdiv(M, 128), N / 64, 4, 2 * kSms, p.s_du, p.per_du);
+  split_plan(cdiv(M, 128) * G, n_max / 64, 4, 2 * kSms, p.s_du, p.per_du);
   if (M > kWideM) {  // dU runs beside the wide dX GEMM's main loop (as U beside Y)
     p.s_du = 1;
-    p.per_du = static_cast<int>(N / 64);
+    p.per_du = static_cast<int>(n_max / 64);
   }
   // dB and dA run on the side stream beside dX: few CTAs with long
   // contractions take fewer SM-cycles from it than many short ones.
   split_plan(cdiv(N, 128), cdiv(M, 64), 4, kSms / 2, p.s_db, p.per_db);
-  split_plan(cdiv(K, 128), cdiv(M, 64), 4, kSms / 2, p.s_da, p.per_da);
+  split_plan(cdiv(K, 128) * G, cdiv(M, 64), 4, kSms / 2, p.s_da, p.per_da);
   p.bn = M > 128 ? 256 : 128;
   size_t off = 0;
   p.off_sucat = off;
-  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
   p.off_ducat = off;
-  off += align256(static_cast<size_t>(M) * 2 * r * 2);
+  off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
   p.total = off;
   return p;
+}
+
+// A group of linears that read the same input, stacked along the output
+// dimension: member g owns rows off[g] .. off[g+1]-1 of the stacked weight,
+// B, Y, dY and dB.  A single linear is the group of one.
+struct Group {
+  int G = 1;
+  int64_t off[5] = {0, 0, 0, 0, 0};
+  int64_t n_max = 0;
+};
+
+Group single_group(int64_t N) {
+  Group g;
+  g.off[1] = N;
+  g.n_max = N;
+  return g;
+}
+
+// Members 1..4, each a multiple of 128 rows (tiles never straddle members),
+// summing to the stacked weight's rows.
+qlora_status make_group(int32_t members, const int64_t* n_member, int64_t N, Group* out) {
+  if (members < 1 || members > 4) return QLORA_ERR_SHAPE;
+  if (!n_member) return QLORA_ERR_NULL;
+  Group g;
+  g.G = members;
+  for (int i = 0; i < members; ++i) {
+    const int64_t n = n_member[i];
+    if (n < 64 || n % 64 != 0 || (members > 1 && n % 128 != 0)) return QLORA_ERR_SHAPE;
+    g.off[i + 1] = g.off[i] + n;
+    g.n_max = std::max(g.n_max, n);
+  }
+  if (g.off[members] != N) return QLORA_ERR_SHAPE;
+  *out = g;
+  return QLORA_OK;
+}
+
+// CTA-pair tiles (256 W rows) need every member boundary on a tile boundary.
+bool group_pairs(const Group& g) {
+  for (int i = 0; i <= g.G; ++i)
+    if (g.off[i] % 256 != 0) return false;
+  return true;
+}
+
+void fill_group(const Group& g, FusedArgs* fa) {
+  fa->groups = g.G;
+  for (int i = 0; i < 3; ++i) fa->grp_end[i] = static_cast<int>(i + 1 < g.G ? g.off[i + 1] : g.off[g.G]);
+}
+void fill_group(const Group& g, SkinnyArgs* sa) {
+  sa->groups = g.G;
+  for (int i = 0; i < 5; ++i) sa->grp_n[i] = static_cast<int>(i <= g.G ? g.off[i] : g.off[g.G]);
+}
+void fill_group(const Group& g, LowmArgs* la, int32_t r) {
+  la->ra = g.G * r;
+  la->groups = g.G;
+  for (int i = 0; i < 3; ++i) la->grp_end[i] = static_cast<int>(i + 1 < g.G ? g.off[i + 1] : g.off[g.G]);
 }
 
 }  // namespace
@@ -497,12 +554,12 @@ void nf4_levels(float out[16]) {
 
 size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
-  return plan_fwd(M, N, K, r).total;
+  return plan_fwd(M, N, K, r, 1).total;
 }
 
 size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
-  return plan_bwd(M, N, K, r).total;
+  return plan_bwd(M, N, K, r, 1, N).total;
 }
 
 qlora_status nf4_quantize(const uint16_t* w_bf16, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
@@ -553,15 +610,19 @@ qlora_status qnf4::check_fwd_args(const uint16_t* X, const uint16_t* Xa, int64_t
 
 extern "C" {
 
-// The forward; Xa is the adapter's input: X itself, or X after dropout.
-static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64_t M, nf4_weight W,
+// The forward of a group of linears sharing X (a single linear is the group
+// of one); Xa is the adapter's input: X itself, or X after dropout.  A is the
+// members' adapters stacked [G r, K], B stacked [N, r], Y [M, N], U [M, G r].
+static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64_t M, nf4_weight W, const Group& grp,
                                     const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y,
                                     int32_t y_dtype, float* U_out, void* ws, size_t ws_bytes, int32_t* d_status,
                                     void* stream) {
   if (qlora_status st = check_fwd_args(X, Xa, M, W, A, B, r, Y, y_dtype, U_out, d_status)) return st;
   if (M == 0) return QLORA_OK;
   const int64_t N = W.n_out, K = W.k_in;
-  const FwdPlan p = plan_fwd(M, N, K, r);
+  const int G = grp.G;
+  const int ra = G * r;
+  const FwdPlan p = plan_fwd(M, N, K, r, G);
   if (!ws || ws_bytes < p.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   if (qlora_status st = check_device()) return st;
@@ -594,8 +655,9 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     la.mpad = p.low_mpad;
     la.status = d_status;
     la.tab = tables();
+    fill_group(grp, &la, r);
     CUtensorMap lc, la_map, lx, lxa;
-    if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, r, K, 64, kLowmARows, 128) ||
+    if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, ra, K, 64, kLowmARows, 128) ||
         !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128) ||
         !map_bf16(&lxa, Xa, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
       return QLORA_ERR_CUDA;
@@ -607,9 +669,10 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     return from_cuda(launch_lowm_finish(la, cs));
   }
 
-  // U = Xa A^T (contraction split over a cluster), plus the bf16 hi/lo of s*U.
+  // U = Xa A^T for every member (contraction split over a cluster), plus the
+  // bf16 hi/lo of s*U; the G CTAs of a token tile read the same X rows.
   CUtensorMap mx_down, ma_down;
-  if (!map_bf16(&mx_down, Xa, M, K, 64, 128) || !map_bf16(&ma_down, A, r, K, 64, 64)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mx_down, Xa, M, K, 64, 128) || !map_bf16(&ma_down, A, ra, K, 64, 64)) return QLORA_ERR_CUDA;
   SkinnyArgs sa{};
   sa.M = static_cast<int>(M);
   sa.N = static_cast<int>(N);
@@ -621,20 +684,21 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   sa.out_f32 = U_out;
   sa.out_cat = ucat;
   sa.status = d_status;
+  fill_group(grp, &sa);
   {
     ProfScope ps(kKDown, cs);
-    if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa, static_cast<int>(cdiv(M, 128)),
-                                                  p.s_down, cs)))
+    if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa,
+                                                  static_cast<int>(cdiv(M, 128)) * G, p.s_down, cs)))
       return st;
   }
 
   // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
   if (M > kWideM) {
-    const bool pair = use_pair(N);
+    const bool pair = use_pair(N) && group_pairs(grp);
     const uint32_t tok_box = pair ? 128 : 256;
     CUtensorMap wx, wc, wu, wb;
     if (!map_bf16(&wx, X, M, K, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
-        !map_bf16(&wu, ucat, M, 2 * r, 32, tok_box, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
+        !map_bf16(&wu, ucat, M, 2 * ra, 32, tok_box, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
       return QLORA_ERR_CUDA;
     FusedArgs fa{};
     fa.c8 = W.c8;
@@ -651,13 +715,14 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     fa.kt_per_split = fa.kt_total;
     fa.status = d_status;
     fa.tab = tables();
+    fill_group(grp, &fa);
     ProfScope ps(kKFusedFwd, cs);
     return from_cuda(pair ? launch_fused_pair(false, wx, wc, wu, wb, fa, cs)
                           : launch_fused2x(false, wx, wc, wu, wb, fa, cs));
   }
   CUtensorMap mx, mc, mu, mb;
   if (!map_bf16(&mx, X, M, K, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 32, 128) ||
-      !map_bf16(&mu, ucat, M, 2 * r, 64, p.bn) || !map_bf16(&mb, B, N, r, 64, 128))
+      !map_bf16(&mu, ucat, M, 2 * ra, 64, p.bn) || !map_bf16(&mb, B, N, r, 64, 128))
     return QLORA_ERR_CUDA;
   FusedArgs fa{};
   fa.c8 = W.c8;
@@ -675,6 +740,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   fa.kt_per_split = p.per_fwd;
   fa.status = d_status;
   fa.tab = tables();
+  fill_group(grp, &fa);
   {
     ProfScope ps(kKFusedFwd, cs);
     if (qlora_status st = from_cuda(launch_fused_fwd(p.bn, mx, mc, mu, mb, fa, p.s_fwd, cs))) return st;
@@ -689,16 +755,19 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
 qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
                               int32_t r, float s, void* Y, int32_t y_dtype, float* U_out, void* ws,
                               size_t ws_bytes, int32_t* d_status, void* stream) {
-  return linear_fwd_impl(X, X, M, W, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
+  return linear_fwd_impl(X, X, M, W, single_group(W.n_out), A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status,
+                         stream);
 }
 
-// The backward; X is the adapter's input (X itself, or X after dropout, for
-// dA).  With `drop`, the GEMM's adapter stages are left out: dX's frozen-path
-// term goes to an fp32 buffer after the caller's workspace and a second pass
-// adds keep * c * (dU A) and writes dX.
+// The backward of a group (a single linear is the group of one); X is the
+// adapter's input (X itself, or X after dropout, for dA).  dY [M, N] stacked,
+// U [M, G r], A [G r, K], B [N, r], dA [G r, K], dB [N, r]; dX [M, K] is the
+// sum over the members.  With `drop`, the GEMM's adapter stages are left out:
+// dX's frozen-path term goes to an fp32 buffer after the caller's workspace
+// and a second pass adds keep * c * (dU A) and writes dX.
 static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
-                                    const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX,
-                                    int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                    const Group& grp, const uint16_t* A, const uint16_t* B, int32_t r, float s,
+                                    void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
                                     int32_t* d_status, void* stream, const DropoutArgs* drop) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
   if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
@@ -709,7 +778,9 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
       !aligned16(dA) || !aligned16(dB) || (d_status && !aligned16(d_status)))
     return QLORA_ERR_ALIGN;
   const int64_t N = W.n_out, K = W.k_in;
-  const BwdPlan p = plan_bwd(M, N, K, r);
+  const int G = grp.G;
+  const int ra = G * r;
+  const BwdPlan p = plan_bwd(M, N, K, r, G, grp.n_max);
   const size_t need = p.total + (drop ? align256(static_cast<size_t>(M) * K * 4) : 0);
   if (!ws || ws_bytes < need) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
@@ -721,7 +792,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   float* dx32 = drop ? reinterpret_cast<float*>(wsb + p.total) : nullptr;
   void* dx_gemm = drop ? static_cast<void*>(dx32) : dX;           // where the GEMM writes
   const int gemm_f32 = drop ? 1 : (dx_dtype == QLORA_DTYPE_F32);
-  const int gemm_r = drop ? 0 : r;                                // adapter stages in the GEMM
+  const int gemm_r = drop ? 0 : ra;                               // adapter stages in the GEMM (all members)
   const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
 
   SkinnyArgs sa{};
@@ -730,12 +801,13 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   sa.K = Ki;
   sa.r = r;
   sa.status = d_status;
+  fill_group(grp, &sa);
 
-  // dU = s dY B  (contraction over N split over a cluster) -> bf16 hi/lo,
-  // and the bf16 hi/lo of s*U for dB from the saved U.
+  // dU = s dY B per member (contraction over the member's outputs, split over
+  // a cluster) -> bf16 hi/lo, and the bf16 hi/lo of s*U for dB from the saved U.
   CUtensorMap mdy128, mbl;
   if (!map_bf16(&mdy128, dY, M, N, 64, 128) || !map_bf16(&mbl, B, N, r, 64, 64)) return QLORA_ERR_CUDA;
-  sa.stages_total = static_cast<int>(N / 64);
+  sa.stages_total = static_cast<int>(grp.n_max / 64);
   sa.stages_per_split = p.per_du;
   sa.s = s;
   sa.out_f32 = nullptr;
@@ -744,7 +816,8 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   sa.out_cat2 = sucat;
   {
     ProfScope ps(kKDU, cs);
-    if (qlora_status st = from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)), p.s_du, cs)))
+    if (qlora_status st =
+            from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)) * G, p.s_du, cs)))
       return st;
   }
 
@@ -755,13 +828,15 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   Fork fork(cs);
   const cudaStream_t side = fork.side();
 
-  // dX = dY W' + dU A, W' dequantised inside the GEMM.
+  // dX = dY W' + dU A (summed over the members: one contraction over the
+  // stacked outputs, then one over the stacked adapter rank), W' dequantised
+  // inside the GEMM.
   if (M > kWideM) {
     const bool pair = use_pair(K);
     const uint32_t tok_box = pair ? 128 : 256;
     CUtensorMap wdy, wc, wdu, wal;
     if (!map_bf16(&wdy, dY, M, N, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 64, 32) ||
-        !map_bf16(&wdu, ducat, M, 2 * r, 32, tok_box, 64) || !map_bf16(&wal, A, r, K, 64, 16, 128))
+        !map_bf16(&wdu, ducat, M, 2 * ra, 32, tok_box, 64) || !map_bf16(&wal, A, ra, K, 64, 16, 128))
       return QLORA_ERR_CUDA;
     FusedArgs fa{};
     fa.c8 = W.c8;
@@ -778,35 +853,35 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     fa.kt_per_split = fa.kt_total;
     fa.status = d_status;
     fa.tab = tables();
+    fa.groups = 1;
     ProfScope ps(kKFusedDX, cs);
     if (qlora_status st = from_cuda(pair ? launch_fused_pair(true, wdy, wc, wdu, wal, fa, cs)
                                          : launch_fused2x(true, wdy, wc, wdu, wal, fa, cs)))
       return st;
   } else {
-  CUtensorMap mdy, mc, mdu, mal;
-  if (!map_bf16(&mdy, dY, M, N, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 64, 64) ||
-      !map_bf16(&mdu, ducat, M, 2 * r, 64, p.bn) || !map_bf16(&mal, A, r, K, 64, 64))
-    return QLORA_ERR_CUDA;
-  FusedArgs fa{};
-  fa.c8 = W.c8;
-  fa.s2 = W.s2;
-  fa.out = dx_gemm;
-  fa.out_f32 = gemm_f32;
-  fa.ld_out = K;
-  fa.split_stride = 0;
-  fa.M = Mi;
-  fa.rows = Ki;
-  fa.n_out = Ni;
-  fa.k_in = Ki;
-  fa.r = gemm_r;
-  fa.kt_total = static_cast<int>(N / 64);
-  fa.kt_per_split = static_cast<int>(N / 64);
-  fa.status = d_status;
-  fa.tab = tables();
-  {
+    CUtensorMap mdy, mc, mdu, mal;
+    if (!map_bf16(&mdy, dY, M, N, 64, p.bn) || !map_u8(&mc, W.codes, N, K / 2, 64, 64) ||
+        !map_bf16(&mdu, ducat, M, 2 * ra, 64, p.bn) || !map_bf16(&mal, A, ra, K, 64, 64))
+      return QLORA_ERR_CUDA;
+    FusedArgs fa{};
+    fa.c8 = W.c8;
+    fa.s2 = W.s2;
+    fa.out = dx_gemm;
+    fa.out_f32 = gemm_f32;
+    fa.ld_out = K;
+    fa.split_stride = 0;
+    fa.M = Mi;
+    fa.rows = Ki;
+    fa.n_out = Ni;
+    fa.k_in = Ki;
+    fa.r = gemm_r;
+    fa.kt_total = static_cast<int>(N / 64);
+    fa.kt_per_split = static_cast<int>(N / 64);
+    fa.status = d_status;
+    fa.tab = tables();
+    fa.groups = 1;
     ProfScope ps(kKFusedDX, cs);
     if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, cs))) return st;
-  }
   }
   if (drop) {  // dX = dX_main + keep * c * (dU A), on the caller's stream after the GEMM
     ProfScope ps(kKDropoutDx, cs);
@@ -815,9 +890,9 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
       return st;
   }
 
-  // dB = dY^T (sU)  (contraction over M split over a cluster)
+  // dB = s dY^T U per member (contraction over M split over a cluster)
   CUtensorMap mdy64, msu;
-  if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * r, 64, 64)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mdy64, dY, M, N, 64, 64) || !map_bf16(&msu, sucat, M, 2 * ra, 64, 64)) return QLORA_ERR_CUDA;
   sa.stages_total = static_cast<int>(cdiv(M, 64));
   sa.stages_per_split = p.per_db;
   sa.s = 1.0f;
@@ -832,9 +907,9 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
       return st;
   }
 
-  // dA = dU^T X  (contraction over M split over a cluster)
+  // dA = dU^T X per member (contraction over M split over a cluster)
   CUtensorMap mduc, mx;
-  if (!map_bf16(&mduc, ducat, M, 2 * r, 64, 64) || !map_bf16(&mx, X, M, K, 64, 64)) return QLORA_ERR_CUDA;
+  if (!map_bf16(&mduc, ducat, M, 2 * ra, 64, 64) || !map_bf16(&mx, X, M, K, 64, 64)) return QLORA_ERR_CUDA;
   {
     SkinnyArgs da = sa;
     da.stages_total = static_cast<int>(cdiv(M, 64));
@@ -843,7 +918,8 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     da.out_f32 = dA;
     da.out_cat = nullptr;
     ProfScope ps(kKDA, side);
-    if (qlora_status st = from_cuda(launch_skinny(kSkDA, mduc, mx, da, static_cast<int>(cdiv(K, 128)), p.s_da, side)))
+    if (qlora_status st = from_cuda(
+            launch_skinny(kSkDA, mduc, mx, da, static_cast<int>(cdiv(K, 128)) * G, p.s_da, side)))
       return st;
   }
 
@@ -853,7 +929,40 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
 qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
                               const uint16_t* A, const uint16_t* B, int32_t r, float s, void* dX, int32_t dx_dtype,
                               float* dA, float* dB, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
-  return linear_bwd_impl(dY, X, U, M, W, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream, nullptr);
+  return linear_bwd_impl(dY, X, U, M, W, single_group(W.n_out), A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes,
+                         d_status, stream, nullptr);
+}
+
+// ------------------------------------------------------------ grouped linears
+
+size_t qlora_group_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t members, int32_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0 || members < 1 || members > 4) return 0;
+  return plan_fwd(M, N, K, r, members).total;
+}
+
+size_t qlora_group_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t members, int32_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0 || members < 1 || members > 4) return 0;
+  return plan_bwd(M, N, K, r, members, N).total;
+}
+
+qlora_status qlora_group_fwd(const uint16_t* X, int64_t M, nf4_weight W, int32_t members, const int64_t* n_member,
+                             const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y, int32_t y_dtype,
+                             float* U_out, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  Group grp;
+  if (qlora_status st = make_group(members, n_member, W.n_out, &grp)) return st;
+  return linear_fwd_impl(X, X, M, W, grp, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
+}
+
+qlora_status qlora_group_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M, nf4_weight W,
+                             int32_t members, const int64_t* n_member, const uint16_t* A, const uint16_t* B,
+                             int32_t r, float s, void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws,
+                             size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  Group grp;
+  if (qlora_status st = make_group(members, n_member, W.n_out, &grp)) return st;
+  return linear_bwd_impl(dY, X, U, M, W, grp, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream,
+                         nullptr);
 }
 
 qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_ns, void* stream) {
@@ -881,7 +990,7 @@ static bool dropout_args(float p, uint64_t seed, DropoutArgs* d) {
 
 size_t qlora_bwd_dropout_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
-  return plan_bwd(M, N, K, r).total + align256(static_cast<size_t>(M) * K * 4);
+  return plan_bwd(M, N, K, r, 1, N).total + align256(static_cast<size_t>(M) * K * 4);
 }
 
 qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A,
@@ -898,7 +1007,7 @@ qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W
   if (!aligned16(X) || !aligned16(X_drop) || !aligned16(A) || !aligned16(B) || !aligned16(Y) ||
       !aligned16(U_out) || (d_status && !aligned16(d_status)))
     return QLORA_ERR_ALIGN;
-  const FwdPlan pl = plan_fwd(M, W.n_out, W.k_in, r);
+  const FwdPlan pl = plan_fwd(M, W.n_out, W.k_in, r, 1);
   if (!ws || ws_bytes < pl.total) return QLORA_ERR_WORKSPACE;
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   if (qlora_status st = check_device()) return st;
@@ -908,7 +1017,8 @@ qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W
             from_cuda(launch_dropout_apply(X, X_drop, M * W.k_in, d, static_cast<cudaStream_t>(stream))))
       return st;
   }
-  return linear_fwd_impl(X, X_drop, M, W, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
+  return linear_fwd_impl(X, X_drop, M, W, single_group(W.n_out), A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes,
+                         d_status, stream);
 }
 
 qlora_status qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X_drop, const float* U, int64_t M,
@@ -917,7 +1027,8 @@ qlora_status qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X_drop
                                       size_t ws_bytes, int32_t* d_status, void* stream) {
   DropoutArgs d{};
   if (!dropout_args(p, seed, &d)) return QLORA_ERR_SHAPE;
-  return linear_bwd_impl(dY, X_drop, U, M, W, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream, &d);
+  return linear_bwd_impl(dY, X_drop, U, M, W, single_group(W.n_out), A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes,
+                         d_status, stream, &d);
 }
 
 // ------------------------------------------------------------------ optimizer

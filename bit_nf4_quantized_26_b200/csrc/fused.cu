@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     bool waited = false;
+    // Grouped forward: this tile's member reads its own columns of the hi/lo copy of s*U.
+    const int uc0 = DX ? 0 : group_member(a.grp_end, a.groups, row0) * 2 * a.r;
     if (lane == 0) {
       int issued = 0;
       for (int t = 0; t < T; ++t) {
@@ -121,12 +123,12 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
           const int e = t - nmain;
           if (!DX) {
             mbar_arrive_expect_tx(&full[s], P::kB + 16384);
-            tma_load_2d(st, &tm_uc, &full[s], 64 * e, m0);
+            tma_load_2d(st, &tm_uc, &full[s], uc0 + 64 * e, m0);
             tma_load_2d(st + P::kB, &tm_ext, &full[s], 32 * e, row0);
           } else {
             const bool second = row0 + 64 < a.rows;
             mbar_arrive_expect_tx(&full[s], P::kB + (second ? 16384 : 8192));
-            tma_load_2d(st, &tm_uc, &full[s], 64 * e, m0);
+            tma_load_2d(st, &tm_uc, &full[s], uc0 + 64 * e, m0);
             tma_load_2d(st + P::kB, &tm_ext, &full[s], row0, 32 * e);
             if (second) tma_load_2d(st + P::kB + 8192, &tm_ext, &full[s], row0 + 64, 32 * e);
           }
@@ -403,6 +405,8 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     bool waited = false;
+    // Grouped forward: this tile's member reads its own columns of the hi/lo copy of s*U.
+    const int uc0 = DX ? 0 : group_member(a.grp_end, a.groups, row0) * 2 * a.r;
     if (lane == 0) {
       int issued = 0;
       const bool a2 = !DX || row0 + 64 < a.rows;  // dX ext: second 64-column half inside K
@@ -431,8 +435,8 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(st + P::kB, &tm_ext, &full[s], row0, 16 * e);  // A_lora [16 j x 64 k]
             if (a2) tma_load_2d(st + P::kB + 4096, &tm_ext, &full[s], row0 + 64, 16 * e);
           }
-          tma_load_2d(st, &tm_uc, &full[s], 32 * e, m0);
-          tma_load_2d(st + P::kBh, &tm_uc, &full[s], 32 * e, m0 + 256);
+          tma_load_2d(st, &tm_uc, &full[s], uc0 + 32 * e, m0);
+          tma_load_2d(st + P::kBh, &tm_uc, &full[s], uc0 + 32 * e, m0 + 256);
         }
         issued = t + 1;
       }

@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     bool waited = false;
+    // Grouped forward: this tile's member reads its own columns of the hi/lo copy of s*U.
+    const int uc0 = DX ? 0 : group_member(a.grp_end, a.groups, row0) * 2 * a.r;
     if (lane == 0) {
       int issued = 0;
       // Extension bytes of one CTA: token/U halves plus the LoRA tile.
@@ -128,8 +130,8 @@ __global__ void __launch_bounds__(192, 1)
           }
           const int e = t - nmain;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (P::kB + ext_a));
-          tma_load_2d_pair(st, &tm_uc, full0, 32 * e, mt);
-          tma_load_2d_pair(st + P::kBq, &tm_uc, full0, 32 * e, mt + 256);
+          tma_load_2d_pair(st, &tm_uc, full0, uc0 + 32 * e, mt);
+          tma_load_2d_pair(st + P::kBq, &tm_uc, full0, uc0 + 32 * e, mt + 256);
           if (!DX) {
             tma_load_2d_pair(st + P::kB, &tm_ext, full0, 16 * e, row0);  // B_lora [128 n x 32 j]
           } else {

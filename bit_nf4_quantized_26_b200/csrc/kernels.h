@@ -67,20 +67,41 @@ struct FusedArgs {
   int kt_per_split;    // stages per blockIdx.z slice
   int32_t* status;
   Nf4Tables tab;
+  // Grouped forward (several linears sharing X, stacked along W's rows): the
+  // W-side rows where members 0..groups-2 end.  A tile of member g reads its
+  // adapter operand from columns g * 2r of the stacked hi/lo copy of s*U.
+  int groups;          // 1 for a single linear
+  int grp_end[3];
 };
+
+// Member of a stacked group that W-side row `row` belongs to.
+__host__ __device__ __forceinline__ int group_member(const int* ends, int groups, int row) {
+  int g = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) g += (i < groups - 1 && row >= ends[i]) ? 1 : 0;
+  return g;
+}
 
 enum SkinnyMode { kSkDown = 0, kSkDU = 1, kSkDB = 2, kSkDA = 3 };
 
+// A group of G linears sharing one input, stacked along the output dimension:
+// member g owns output rows grp_n[g] .. grp_n[g+1]-1 of the stacked W, B and
+// dB, rows g*r .. g*r+r-1 of the stacked A and dA, and columns g*r .. of U
+// (row stride G*r) and g*2r .. of the hi/lo copies (row stride 2*G*r).  A
+// single linear is the group of one.  DOWN, DU and DA grids hold G CTAs per
+// row tile (blockIdx.x = tile * G + g); DB finds g from its output rows.
 struct SkinnyArgs {
-  int M, N, K, r;
-  int stages_total;     // contraction stages (64 each)
+  int M, N, K, r;       // N: all members' outputs; r: one member's rank
+  int stages_total;     // contraction stages (64 each); DU: those of the longest member
   int stages_per_split; // stages per CTA of a cluster (the cluster spans the splits)
   float s;              // DOWN: scale of the hi/lo copy of U; DU: the LoRA scale
-  float* out_f32;       // DOWN: U [M, r]; DB: dB [N, r]; DA: dA [r, K]
-  uint16_t* out_cat;    // DOWN: hi/lo of s*U [M, 2r]; DU: hi/lo of dU [M, 2r]
-  const float* in_u;    // DU: the saved U [M, r]
-  uint16_t* out_cat2;   // DU: hi/lo of s*U [M, 2r] (the dB operand)
+  float* out_f32;       // DOWN: U [M, G r]; DB: dB [N, r]; DA: dA [G r, K]
+  uint16_t* out_cat;    // DOWN: hi/lo of s*U [M, 2 G r]; DU: hi/lo of dU [M, 2 G r]
+  const float* in_u;    // DU: the saved U [M, G r]
+  uint16_t* out_cat2;   // DU: hi/lo of s*U [M, 2 G r] (the dB operand)
   int32_t* status;
+  int groups;           // G (1..4)
+  int grp_n[5];         // member offsets along N (grp_n[0] = 0, grp_n[G] = N)
 };
 
 // One CTA waits on an mbarrier nothing completes, with a `limit_ns` bound,
@@ -181,12 +202,17 @@ struct LowmArgs {
   float s;
   int M, N, K, r;
   int tiles;             // ceil(N / 128)
-  int atiles;            // r / 32 rounded up
+  int atiles;            // ra / 32 rounded up
   int kc;                // ceil(K / 256)
   int ctas;              // CTAs of the main kernel (>= tiles + atiles)
   int mpad;              // tokens per partial row: 8 * n8 token tiles (8, 16 or 32)
   int32_t* status;
   Nf4Tables tab;
+  // Grouped forward: A holds the G members' adapters stacked ([ra = G r, K]),
+  // U is [M, ra], B and Y are stacked along N; members end at grp_end.
+  int ra;
+  int groups;
+  int grp_end[3];
 };
 
 //   tm_codes: codes [N, K/2] u8 box {128, 128} SW128; tm_a: A [r, K] bf16

@@ -80,10 +80,10 @@ __device__ __forceinline__ int64_t lowm_units(const LowmArgs& a) {
 }
 
 // Whether this warp has rows in `tile`: all 16 rows of its slice exist (N and
-// r are multiples of 16).  A tiles use warps 0 and 1 only.
+// the rows of A are multiples of 16).  A tiles use warps 0 and 1 only.
 __device__ __forceinline__ bool warp_rows_valid(const LowmArgs& a, int tile, int warp) {
   if (tile < a.tiles) return tile * kLowmRows + warp * 16 + 16 <= a.N;
-  return warp < 2 && (tile - a.tiles) * kLowmARows + warp * 16 + 16 <= a.r;
+  return warp < 2 && (tile - a.tiles) * kLowmARows + warp * 16 + 16 <= a.ra;
 }
 
 // Block constants of rows g and g + 8 of this warp's slice, block t of the
@@ -328,14 +328,17 @@ __device__ __forceinline__ float4 sum_tile_partials(const LowmArgs& a, int tile,
 }
 
 // Y[m, n] = sum of the row tile's partials + s * sum_j U[m, j] B[n, j], with
-// U = the A tiles' partials summed (every CTA forms U; CTA 0 stores it).  The
-// row of B is read before the wait for the main kernel (B is not one of its
-// outputs).
+// U = the A tiles' partials summed (every CTA forms the U of its rows' member;
+// the first CTA of each member stores it).  The row of B is read before the
+// wait for the main kernel (B is not one of its outputs).
 __global__ void __launch_bounds__(512) lowm_finish_kernel(const LowmArgs a) {
   __shared__ float su[kLowmMpad][64];
   const int tid = threadIdx.x;
   const int rl = tid & (kFinRows - 1), q = tid >> 6;
-  const int n = blockIdx.x * kFinRows + rl;
+  const int n0 = blockIdx.x * kFinRows;
+  const int mem = group_member(a.grp_end, a.groups, n0);  // 64-row blocks lie in one member
+  const bool mem_first = mem == 0 ? n0 == 0 : n0 == a.grp_end[mem - 1];
+  const int n = n0 + rl;
   const bool active = n < a.N && 4 * q < a.M;
   uint4 bv[8];
   const uint4* br = reinterpret_cast<const uint4*>(a.B + static_cast<int64_t>(n < a.N ? n : 0) * a.r);
@@ -349,15 +352,16 @@ __global__ void __launch_bounds__(512) lowm_finish_kernel(const LowmArgs a) {
   // U: thread (j = tid & 63, quad q) sums row j of the A tiles for its tokens.
   {
     const int j = tid & 63;
+    const int ja = mem * a.r + j;  // row of the stacked A
     if (j < a.r && 4 * q < a.M) {
-      const float4 u = sum_tile_partials(a, a.tiles + j / kLowmARows, j % kLowmARows, q);
+      const float4 u = sum_tile_partials(a, a.tiles + ja / kLowmARows, ja % kLowmARows, q);
       const float uv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int m = 4 * q + e;
         if (m < a.M) {
           su[m][j] = uv[e];
-          if (blockIdx.x == 0) a.U[static_cast<int64_t>(m) * a.r + j] = uv[e];
+          if (mem_first) a.U[static_cast<int64_t>(m) * a.ra + ja] = uv[e];
         }
       }
     }

@@ -45,11 +45,12 @@ struct SkPlan {
 
 __device__ __forceinline__ int hilo_col(int j) { return 32 * (j >> 4) + (j & 15); }
 
-// v -> (bf16(v), bf16(v - bf16(v))) at the interleaved hi/lo columns of row m.
-__device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int r, int j, float v) {
+// v -> (bf16(v), bf16(v - bf16(v))) at the interleaved hi/lo columns of row m
+// (row stride `ld` elements; the member's columns start at `col0`).
+__device__ __forceinline__ void store_hilo(uint16_t* cat, int m, int ld, int col0, int j, float v) {
   const uint16_t hi = bf16_bits(v);
   const uint16_t lo = bf16_bits(__fsub_rn(v, bf16_bits_to_float(hi)));
-  uint16_t* row = cat + static_cast<int64_t>(m) * 2 * r;
+  uint16_t* row = cat + static_cast<int64_t>(m) * ld + col0;
   row[hilo_col(j)] = hi;
   row[hilo_col(j) + 16] = lo;
 }
@@ -69,11 +70,22 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Tile origin: DOWN/DU rows are tokens, DB rows are output features, DA's
-  // 128 rows are the hi/lo columns of dU and blockIdx.x walks K in 128s.
-  const int row0 = blockIdx.x * 128;
+  // 128 rows are the hi/lo columns of dU and its tiles walk K in 128s.  The
+  // member g: DOWN, DU and DA have G CTAs per tile; DB's rows lie in one member.
+  const int G = a.groups;
+  const bool per_tile = MODE != kSkDB;
+  const int tile = per_tile ? static_cast<int>(blockIdx.x) / G : static_cast<int>(blockIdx.x);
+  const int row0 = tile * 128;
+  int g = per_tile ? static_cast<int>(blockIdx.x) % G : 0;
+  if (!per_tile)
+    for (int i = 1; i < G; ++i) g += row0 >= a.grp_n[i] ? 1 : 0;
+  const int ra = G * a.r;                // U row stride
+  const int ucol = g * 2 * a.r;          // this member's first hi/lo column
+  const int nbase = a.grp_n[g];          // DU: this member's first output feature
   const int z = blockIdx.y;
   const int st0 = z * a.stages_per_split;
-  const int T = min(a.stages_total, st0 + a.stages_per_split) - st0;
+  const int st_all = MODE == kSkDU ? (a.grp_n[g + 1] - nbase) / 64 : a.stages_total;
+  const int T = min(st_all, st0 + a.stages_per_split) - st0;  // <= 0: no MMA, the partial is zero
   const int nc = (2 * a.r > 64) ? 128 : 64;  // DB: width of the sU operand
 
   if (threadIdx.x == 0) {
@@ -110,24 +122,27 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         uint8_t* sa = smem + s * P::kStage;
         uint8_t* sb = sa + P::kA;
         const int kt = st0 + t;
-        if (MODE == kSkDown || MODE == kSkDU) {
+        if (MODE == kSkDown) {
           mbar_arrive_expect_tx(&full[s], 16384 + 8192);
           tma_load_2d(sa, &tmA, &full[s], kt * 64, row0);
-          if (MODE == kSkDown) tma_load_2d(sb, &tmB, &full[s], kt * 64, 0);
-          else tma_load_2d(sb, &tmB, &full[s], 0, kt * 64);
+          tma_load_2d(sb, &tmB, &full[s], kt * 64, g * a.r);       // this member's rows of A
+        } else if (MODE == kSkDU) {
+          mbar_arrive_expect_tx(&full[s], 16384 + 8192);
+          tma_load_2d(sa, &tmA, &full[s], nbase + kt * 64, row0);  // this member's columns of dY
+          tma_load_2d(sb, &tmB, &full[s], 0, nbase + kt * 64);     // and rows of B
         } else if (MODE == kSkDB) {
           const bool a2 = row0 + 64 < a.N;
           mbar_arrive_expect_tx(&full[s], 8192u * ((a2 ? 2 : 1) + nc / 64));
           tma_load_2d(sa, &tmA, &full[s], row0, kt * 64);
           if (a2) tma_load_2d(sa + 8192, &tmA, &full[s], row0 + 64, kt * 64);
-          tma_load_2d(sb, &tmB, &full[s], 0, kt * 64);
-          if (nc == 128) tma_load_2d(sb + 8192, &tmB, &full[s], 64, kt * 64);
+          tma_load_2d(sb, &tmB, &full[s], ucol, kt * 64);
+          if (nc == 128) tma_load_2d(sb + 8192, &tmB, &full[s], ucol + 64, kt * 64);
         } else {  // DA
           int nb = 0;
           for (int i = 0; i < 2; ++i) nb += (row0 + 64 * i < a.K) ? 1 : 0;
           mbar_arrive_expect_tx(&full[s], 8192u * ((nc / 64) + nb));
-          tma_load_2d(sa, &tmA, &full[s], 0, kt * 64);
-          if (nc == 128) tma_load_2d(sa + 8192, &tmA, &full[s], 64, kt * 64);
+          tma_load_2d(sa, &tmA, &full[s], ucol, kt * 64);
+          if (nc == 128) tma_load_2d(sa + 8192, &tmA, &full[s], ucol + 64, kt * 64);
           for (int i = 0; i < nb; ++i) tma_load_2d(sb + 8192 * i, &tmB, &full[s], row0 + 64 * i, kt * 64);
         }
         issued = t + 1;
@@ -173,6 +188,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
           tmem_ld_wait();
+          if (T <= 0)
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
           float* dst = part + rl * P::kLdRows + cb * 32;
           const int nv = min(32, a.r - cb * 32);
 #pragma unroll
@@ -183,11 +200,13 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         }
       } else if (MODE == kSkDB) {
         // rows = output features, columns = hi/lo pairs of j -> combined
-        for (int g = 0; g < a.r / 16; ++g) {
+        for (int jb = 0; jb < a.r / 16; ++jb) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tq + g * 32, v);
+          tmem_ld_32x32b_x32(tq + jb * 32, v);
           tmem_ld_wait();
-          float* dst = part + rl * P::kLdRows + g * 16;
+          if (T <= 0)
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          float* dst = part + rl * P::kLdRows + jb * 16;
 #pragma unroll
           for (int j = 0; j < 16; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(
@@ -203,6 +222,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
           tmem_ld_wait();
+          if (T <= 0)
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
           float sum[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -254,15 +275,16 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         const int m = row0 + row;
         if (m < a.M) {
           if (MODE == kSkDown)
-            *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(m) * a.r + col) = acc;
+            *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(m) * ra + g * a.r + col) = acc;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) store_hilo(a.out_cat, m, a.r, col + i, __fmul_rn(a.s, vals[i]));
+          for (int i = 0; i < 4; ++i) store_hilo(a.out_cat, m, 2 * ra, ucol, col + i, __fmul_rn(a.s, vals[i]));
           if (MODE == kSkDU) {
             // The same rows of the saved U, as the bf16 hi/lo of s*U for dB.
-            const float4 uv = __ldg(reinterpret_cast<const float4*>(a.in_u + static_cast<int64_t>(m) * a.r + col));
+            const float4 uv =
+                __ldg(reinterpret_cast<const float4*>(a.in_u + static_cast<int64_t>(m) * ra + g * a.r + col));
             const float us[4] = {uv.x, uv.y, uv.z, uv.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) store_hilo(a.out_cat2, m, a.r, col + i, __fmul_rn(a.s, us[i]));
+            for (int i = 0; i < 4; ++i) store_hilo(a.out_cat2, m, 2 * ra, ucol, col + i, __fmul_rn(a.s, us[i]));
           }
         }
       } else if (MODE == kSkDB) {
@@ -270,7 +292,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         if (n < a.N) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(n) * a.r + col) = acc;
       } else {
         const int k = row0 + col;
-        if (k < a.K) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(row) * a.K + k) = acc;
+        if (k < a.K) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(g * a.r + row) * a.K + k) = acc;
       }
     }
   }

@@ -171,6 +171,48 @@ QLORA_API size_t qlora_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32
 QLORA_API size_t qlora_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t r);
 
 /*
+ * Grouped projections: several linears that read the same input X — the q, k
+ * and v projections of an attention layer, or the gate and up projections of
+ * its MLP — run as one forward and one backward call ("QLoRA" entry, "como
+ * funciona": adapters on every linear layer; grouping the ones that share an
+ * input reads X once and gives its gradient summed).  The G members (1..4)
+ * are stacked along the output dimension:
+ *
+ *   W        one NF4 weight [N, K], N = sum of the members' n_member[g]: the
+ *            NF4 storage of the members' rows one after another (each
+ *            n_member[g] a multiple of 128, of 64 when G = 1).  nf4_quantize
+ *            of the stacked bf16 weight produces it; when every member holds
+ *            a whole number of double-quantisation groups (n_member[g] * K a
+ *            multiple of 16384) it is also the members' own storages back to
+ *            back;
+ *   A        [G r, K] bf16: member g's adapter A_g in rows g r .. g r + r - 1;
+ *   B        [N, r]   bf16: member g's B_g in the member's rows;
+ *   Y, dY    [M, N]: member g's outputs in its columns;
+ *   U        [M, G r] fp32: U_g = X A_g^T in columns g r .. g r + r - 1;
+ *   dA, dB   [G r, K] and [N, r] fp32, stacked like A and B;
+ *   dX       [M, K] = sum over the members of (dY_g W_g' + s (dY_g B_g) A_g),
+ *            the gradient of the shared input.
+ *
+ * Every member uses the same r and s.  Per member the results are those of
+ * qlora_linear_fwd / qlora_linear_bwd on that member alone (same accuracy);
+ * dX is accumulated over all members in one fp32 accumulator.  n_member is a
+ * host array of G sizes.  Constraints as for the single linear, plus
+ * 1 <= G <= 4 and the member sizes above (QLORA_ERR_SHAPE; a NULL n_member is
+ * QLORA_ERR_NULL).  Workspaces: qlora_group_{fwd,bwd}_workspace_size(M, N,
+ * K, G, r) bytes (with G = 1 the same as the single linear's).
+ */
+QLORA_API size_t qlora_group_fwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t members, int32_t r);
+QLORA_API size_t qlora_group_bwd_workspace_size(int64_t M, int64_t N, int64_t K, int32_t members, int32_t r);
+QLORA_API qlora_status qlora_group_fwd(const uint16_t* X, int64_t M, nf4_weight W, int32_t members,
+                                       const int64_t* n_member, const uint16_t* A, const uint16_t* B, int32_t r,
+                                       float s, void* Y, int32_t y_dtype, float* U_out, void* ws, size_t ws_bytes,
+                                       int32_t* d_status, void* stream);
+QLORA_API qlora_status qlora_group_bwd(const uint16_t* dY, const uint16_t* X, const float* U, int64_t M,
+                                       nf4_weight W, int32_t members, const int64_t* n_member, const uint16_t* A,
+                                       const uint16_t* B, int32_t r, float s, void* dX, int32_t dx_dtype, float* dA,
+                                       float* dB, void* ws, size_t ws_bytes, int32_t* d_status, void* stream);
+
+/*
  * LoRA dropout on the adapter input ("Tutorial fine-tuning LLM LoRA/QLoRA
  * 2026", "Mão na Massa": the adapter configuration's lora_dropout; where it
  * acts is this library's reading).  The frozen path sees X, the adapter sees

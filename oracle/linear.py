@@ -29,7 +29,9 @@ Every product is a plain numpy fp64 matrix product of the exact (bf16 or
 fp32) inputs; nothing is rounded in between.  Parity status: pinned
 (pure-Python brute force on tiny shapes, the merged-weight identity, the
 special cases W' = 0 and B = 0, and central finite differences of
-L = sum(Y * dY) in tests/test_oracle_linear.py).
+L = sum(Y * dY) in tests/test_oracle_linear.py; for a group of linears that
+share X, the same finite differences of the summed loss, and the group of
+one equal to the single linear).
 """
 
 import numpy as np
@@ -62,6 +64,43 @@ def linear_bwd(dY, X, Wd, A, B, s, want_dx=True):
     dA = dU.T @ X
     dB = s * (dY.T @ U)
     return dX, dA, dB, dU
+
+
+def group_fwd(X, Wd, A, B, s, n_member):
+    """Forward of a group of linears that read the same X, stacked along the
+    output dimension: member g owns rows off_g .. off_g + n_member[g] - 1 of
+    Wd and B and rows g r .. g r + r - 1 of A.  Each member is the linear
+    above; returns (U [M, G r], Y [M, N]) with the members side by side."""
+    G = len(n_member)
+    r = np.asarray(A).shape[0] // G
+    off = np.concatenate([[0], np.cumsum(n_member)]).astype(int)
+    Us, Ys = [], []
+    for g in range(G):
+        U, Y = linear_fwd(X, np.asarray(Wd)[off[g]:off[g + 1]], np.asarray(A)[g * r:(g + 1) * r],
+                          np.asarray(B)[off[g]:off[g + 1]], s)
+        Us.append(U)
+        Ys.append(Y)
+    return np.concatenate(Us, axis=1), np.concatenate(Ys, axis=1)
+
+
+def group_bwd(dY, X, Wd, A, B, s, n_member, want_dx=True):
+    """Backward of :func:`group_fwd`: each member's dA, dB as for one linear,
+    stacked like A and B; dX is the sum of the members' dX (X feeds every
+    member, so its gradient is the sum of theirs).  Returns (dX, dA, dB)."""
+    G = len(n_member)
+    r = np.asarray(A).shape[0] // G
+    off = np.concatenate([[0], np.cumsum(n_member)]).astype(int)
+    dX, dAs, dBs = None, [], []
+    for g in range(G):
+        rows = slice(off[g], off[g + 1])
+        Wg = None if Wd is None else np.asarray(Wd)[rows]
+        dXg, dAg, dBg, _ = linear_bwd(np.asarray(dY)[:, rows], X, Wg, np.asarray(A)[g * r:(g + 1) * r],
+                                      np.asarray(B)[rows], s, want_dx=want_dx)
+        if want_dx:
+            dX = dXg if dX is None else dX + dXg
+        dAs.append(dAg)
+        dBs.append(dBg)
+    return dX, np.concatenate(dAs, axis=0), np.concatenate(dBs, axis=0)
 
 
 def rel_frobenius(got, ref):

@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 20
+    assert len(names) == 24
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -115,6 +115,35 @@ def test_noalloc_argument_errors_match_the_forward():
     assert _noalloc(X=None) == NULL
     assert _noalloc(X=FAKE + 8) == ALIGN
     assert _noalloc(W=_w(codes=None)) == NULL
+
+
+def test_group_argument_errors():
+    """Grouped projections: 1..4 members, each a multiple of 128 rows (64 for
+    one member), summing to the stacked weight's rows; checked on the host."""
+    f = q.raw().qlora_group_fwd
+    b = q.raw().qlora_group_bwd
+
+    def members(*n):
+        return ctypes.cast((ctypes.c_int64 * len(n))(*n), ctypes.c_void_p)
+
+    def fwd(G, nm, W=None, M=64, ydt=0):
+        W = _w(n=4096 * 3) if W is None else W
+        return f(FAKE, M, W, G, nm, FAKE, FAKE, 64, 0.25, FAKE, ydt, FAKE, FAKE, 1 << 40, None, None)
+
+    assert fwd(3, None) == NULL
+    assert fwd(0, members(4096)) == SHAPE and fwd(5, members(*[2048] * 5)) == SHAPE
+    assert fwd(3, members(4096, 4096, 4032)) == SHAPE          # sum != stacked rows
+    assert fwd(2, members(6080, 6208), W=_w(n=12288)) == SHAPE  # 6080 % 128 != 0
+    assert fwd(3, members(4096, 4096, 4096), ydt=5) == DTYPE
+    assert fwd(3, members(4096, 4096, 4096), M=0) == OK
+    assert b(FAKE, FAKE, FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 8, 0.25, FAKE, 0, FAKE, FAKE,
+             FAKE, 1 << 40, None, None) == SHAPE                # r = 8
+    assert b(FAKE, FAKE, FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 64, 0.25, FAKE, 0, FAKE, FAKE,
+             FAKE, 16, None, None) == WS
+    assert q.qlora_group_fwd_workspace_size(4096, 12288, 4096, 1, 64) == q.qlora_fwd_workspace_size(4096, 12288,
+                                                                                                    4096, 64)
+    assert q.qlora_group_bwd_workspace_size(4096, 12288, 4096, 3, 64) > q.qlora_bwd_workspace_size(4096, 12288,
+                                                                                                   4096, 64)
 
 
 def test_bwd_argument_errors():
