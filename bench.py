@@ -50,9 +50,10 @@ ALPHA = 16.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 NF4_BYTES_PER_PARAM = 2 + 0.5 + 1 / 64 + 4 / 16384
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# tensor-core kernels in one layer step (mean over the step's launches of that
-# kernel), from an ncu capture of the current kernels; None until captured.
-NCU_TRAFFIC_BYTES = {}
+# CTA-pair GEMMs in the grouped layer step (mean over the step's 4 launches of
+# each), from one ncu capture of the current kernels (the decoder-layer-step
+# summary under profiles/); emptied whenever those kernels change.
+NCU_TRAFFIC_BYTES = {"fused_fwd": 708.1e6, "fused_dx": 724.1e6}
 
 
 def flops_fwd_bwd(M, N, K, r):
@@ -491,6 +492,62 @@ def c5_quantize_sweep(lib, synth, torch, dev):
             "wall_s_with_draws": wall}
 
 
+def centered_cost(lib, synth, torch, dev, flush, reps=5):
+    """What mean-centred double quantisation costs against the plain scheme,
+    per kernel family (median device times, L2 flushed before each call):
+    quantise and dequantise a 22016x8192 weight, the few-token forward (16
+    tokens) on it, and the 4096x4096 forward + backward at 4096 tokens."""
+    import statistics
+
+    def med(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e3
+
+    out = {}
+    w = synth.weight_bf16(22016, 8192, seed=99, device=dev)
+    Wp = lib.quantize_weight(w)
+    Wc = lib.quantize_weight_centered(w)
+    ws = torch.empty(lib.nf4_centered_workspace_size(w.numel()), dtype=torch.uint8, device=dev)
+    dq = torch.empty(w.numel(), dtype=torch.bfloat16, device=dev)
+    out["quantize_us"] = {"plain": med(lambda: lib.nf4_quantize(w.reshape(-1), Wp.codes, Wp.c8, Wp.s2)),
+                          "centered": med(lambda: lib.nf4_quantize_centered(w.reshape(-1), Wc.codes, Wc.c8, Wc.s2,
+                                                                            Wc.mean, ws=ws))}
+    out["dequantize_us"] = {"plain": med(lambda: lib.nf4_dequantize(Wp.codes, Wp.c8, Wp.s2, w.numel(), out=dq)),
+                            "centered": med(lambda: lib.nf4_dequantize_centered(Wc.codes, Wc.c8, Wc.s2, Wc.mean,
+                                                                                w.numel(), out=dq))}
+    del dq, ws
+    X = synth.normal_bf16((16, 8192), 1.0, seed=5, device=dev)
+    A = synth.normal_bf16((64, 8192), 1.0 / 8192, seed=6, device=dev)
+    B = synth.normal_bf16((22016, 64), synth.B_STD, seed=7, device=dev)
+    Y = torch.empty((16, 22016), dtype=torch.bfloat16, device=dev)
+    U = torch.empty((16, 64), dtype=torch.float32, device=dev)
+    out["fwd_16_tokens_us"] = {k: med(lambda W=W: lib.qlora_linear_fwd(X, W, A, B, 0.25, Y=Y, U=U))
+                               for k, W in (("plain", Wp), ("centered", Wc))}
+    del w, Wp, Wc, X, A, B, Y, U
+    d = {k: v.to(dev) for k, v in synth.linear_inputs(synth.Linear("c2", 4096, 4096), 4096, 64, 0).items()}
+    Wp = lib.quantize_weight(d["W"])
+    Wc = lib.quantize_weight_centered(d["W"])
+
+    def fb(W):
+        _, U2 = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.25)
+        lib.qlora_linear_bwd(d["dY"], d["X"], U2, W, d["A"], d["B"], 0.25)
+    out["fwd_bwd_4096_us"] = {k: med(lambda W=W: fb(W)) for k, W in (("plain", Wp), ("centered", Wc))}
+    for k in list(out):
+        out[k]["overhead"] = out[k]["centered"] / out[k]["plain"] - 1.0
+    out["workload"] = ("22016x8192 weight (quantise, dequantise, 16-token forward); 4096x4096 forward + backward "
+                       "at 4096 tokens, r=64")
+    return out
+
+
 def c1_graph_timing(lib, synth, torch, dev, reps=200):
     """c1 step (quantize + fwd + bwd, 512x512, 64 tokens, r=16) eager vs one CUDA graph.
 
@@ -785,16 +842,25 @@ def run_ours(args, rank, world):
 
     extras = {}
     if rank == 0 and not args.no_sweep and grouped:
-        # The same step with every linear its own call (no grouping).
+        # Grouped against per-linear calls, timed in alternation (rounds of a
+        # few steps each) so that both see the same clocks and power state.
         flat = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=False)
+        again = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=True)
         for _ in range(3):
             flat.step()
-        ts = time_steps(torch, flat.step, stream, args.steps, flush)
-        fms = float(np.mean(ts))
-        extras["per_linear_step"] = {"ms_per_step": fms, "tflops": fl / (fms * 1e-3) / 1e12,
-                                     "grouped_ms_per_step": ms, "grouped_speedup": fms / ms}
+            again.step()
+        tg, tf = [], []
+        for _ in range(4):
+            tg += time_steps(torch, again.step, stream, max(2, args.steps // 4), flush)
+            tf += time_steps(torch, flat.step, stream, max(2, args.steps // 4), flush)
+        gms, fms = float(np.mean(tg)), float(np.mean(tf))
+        extras["grouping_ab"] = {"per_linear_ms_per_step": fms, "per_linear_tflops": fl / (fms * 1e-3) / 1e12,
+                                 "grouped_ms_per_step": gms, "grouped_tflops": fl / (gms * 1e-3) / 1e12,
+                                 "grouped_speedup": fms / gms,
+                                 "timing": "4 alternating rounds of K/4 steps each, L2 flushed before every step"}
         flat.close()
-        del flat
+        again.close()
+        del flat, again
     if rank == 0 and not args.no_sweep:
         quant_gbs, dequant_gbs = nf4_stream_timing(lib, synth, torch, dev, flush)
         extras["nf4_quantize_gbs"] = quant_gbs
@@ -808,6 +874,7 @@ def run_ours(args, rank, world):
         extras["c5_quantize_sweep"] = c5_quantize_sweep(lib, synth, torch, dev)
         extras["c5_quantize_sweep"]["hbm_frac"] = extras["c5_quantize_sweep"]["quantize_gbs"] / peaks["hbm_gbs"]
         extras["c1_graph"] = c1_graph_timing(lib, synth, torch, dev)
+        extras["centered_dq"] = centered_cost(lib, synth, torch, dev, flush)
 
     value = world * fl / (ms * 1e-3) / 1e12
     cpu = None

@@ -48,7 +48,7 @@ class QloraError(RuntimeError):
 
 class _NF4Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("c8", ctypes.c_void_p), ("s2", ctypes.c_void_p),
-                ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64)]
+                ("n_out", ctypes.c_int64), ("k_in", ctypes.c_int64), ("mean", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -88,7 +88,9 @@ EXPORTED = ("nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_
             "qlora_fwd_workspace_size", "qlora_bwd_workspace_size", "nf4_levels", "qlora_strerror",
             "qlora_profile_enable", "qlora_profile_collect", "qlora_kernel_name", "qlora_linear_fwd_noalloc")
 
-NF4Weight = namedtuple("NF4Weight", "codes c8 s2 n_out k_in")
+# mean: None for the plain double quantisation, or the 1-element fp32 device
+# tensor of a weight quantised with nf4_quantize_centered.
+NF4Weight = namedtuple("NF4Weight", "codes c8 s2 n_out k_in mean", defaults=(None,))
 
 
 def qlora_strerror(code):
@@ -125,7 +127,9 @@ def _check(code, where):
 
 
 def _weight(W):
-    return _NF4Weight(W.codes.data_ptr(), W.c8.data_ptr(), W.s2.data_ptr(), int(W.n_out), int(W.k_in))
+    mean = getattr(W, "mean", None)
+    return _NF4Weight(W.codes.data_ptr(), W.c8.data_ptr(), W.s2.data_ptr(), int(W.n_out), int(W.k_in),
+                      None if mean is None else mean.data_ptr())
 
 
 def nf4_sizes(numel):
@@ -492,3 +496,52 @@ def qlora_group_bwd(dY, X, U, W, n_member, A, B, s, dx_dtype=DTYPE_BF16, dX=None
                                 _ptr(status), _stream(stream)),
            "qlora_group_bwd")
     return dX, dA, dB
+
+
+# ------------------------------------------ mean-centred double quantisation
+
+_lib.nf4_centered_workspace_size.argtypes = [_I64]
+_lib.nf4_centered_workspace_size.restype = _SZ
+_lib.nf4_quantize_centered.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P]
+_lib.nf4_quantize_centered.restype = ctypes.c_int
+_lib.nf4_dequantize_centered.argtypes = [_P, _P, _P, _P, _I64, _P, _P]
+_lib.nf4_dequantize_centered.restype = ctypes.c_int
+
+EXPORTED = EXPORTED + ("nf4_centered_workspace_size", "nf4_quantize_centered", "nf4_dequantize_centered")
+
+
+def nf4_centered_workspace_size(numel):
+    return int(_lib.nf4_centered_workspace_size(numel))
+
+
+def nf4_quantize_centered(w, codes=None, c8=None, s2=None, mean=None, ws=None, status=None, stream=None):
+    """Quantise a bf16 CUDA tensor with mean-centred constants; returns
+    ``(codes, c8, s2, mean)`` (allocated if not given; mean is fp32 [1])."""
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.is_contiguous()
+    numel = w.numel()
+    nc, nb, ns = nf4_sizes(numel)
+    dev = w.device
+    codes = torch.empty(nc, dtype=torch.uint8, device=dev) if codes is None else codes
+    c8 = torch.empty(nb, dtype=torch.uint8, device=dev) if c8 is None else c8
+    s2 = torch.empty(ns, dtype=torch.float32, device=dev) if s2 is None else s2
+    mean = torch.empty(4, dtype=torch.float32, device=dev)[:1] if mean is None else mean
+    if ws is None:
+        ws = torch.empty(max(nf4_centered_workspace_size(numel), 16), dtype=torch.uint8, device=dev)
+    _check(_lib.nf4_quantize_centered(_ptr(w), numel, _ptr(codes), _ptr(c8), _ptr(s2), _ptr(mean), _ptr(ws),
+                                      ws.numel(), _ptr(status), _stream(stream)), "nf4_quantize_centered")
+    return codes, c8, s2, mean
+
+
+def quantize_weight_centered(w, stream=None):
+    """NF4-quantise a bf16 weight [n_out, k_in] with mean-centred constants;
+    returns an :class:`NF4Weight` whose ``mean`` is set."""
+    codes, c8, s2, mean = nf4_quantize_centered(w, stream=stream)
+    return NF4Weight(codes, c8, s2, w.shape[0], w.shape[1], mean)
+
+
+def nf4_dequantize_centered(codes, c8, s2, mean, numel, out=None, stream=None):
+    """bf16 tensor of ``numel`` values dequantised with mean-centred constants."""
+    out = torch.empty(numel, dtype=torch.bfloat16, device=codes.device) if out is None else out
+    _check(_lib.nf4_dequantize_centered(_ptr(codes), _ptr(c8), _ptr(s2), _ptr(mean), numel, _ptr(out),
+                                        _stream(stream)), "nf4_dequantize_centered")
+    return out

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqlora_nf4.so")
-SOURCES = ["api.cu", "quant.cu", "fused.cu", "fused_pair.cu", "skinny.cu", "lowm.cu", "noalloc.cu", "optim.cu", "dropout.cu"]
+SOURCES = ["api.cu", "quant.cu", "fused.cu", "fused_pair.cu", "fused_pair_fwd.cu", "skinny.cu", "lowm.cu", "noalloc.cu", "optim.cu", "dropout.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

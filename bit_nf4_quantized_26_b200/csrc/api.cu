@@ -160,6 +160,17 @@ bool use_pair(int64_t rows) {
   return enabled && rows % 256 == 0;
 }
 
+// QLORA_TMEM_A=1 selects the CTA-pair forward that keeps the dequantised
+// tile in tensor memory (exact, but measured slower than the shared-memory
+// kernel, which stays the default).
+bool use_tmem_a() {
+  static const bool enabled = [] {
+    const char* e = getenv("QLORA_TMEM_A");
+    return e && e[0] == '1';
+  }();
+  return enabled;
+}
+
 // ------------------------------------------------------------ checks
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -192,7 +203,8 @@ qlora_status check_linear_shape(int64_t M, const nf4_weight& W, int32_t r) {
 
 qlora_status check_weight_ptrs(const nf4_weight& W) {
   if (!W.codes || !W.c8 || !W.s2) return QLORA_ERR_NULL;
-  if (!aligned16(W.codes) || !aligned16(W.c8) || !aligned16(W.s2)) return QLORA_ERR_ALIGN;
+  if (!aligned16(W.codes) || !aligned16(W.c8) || !aligned16(W.s2) || (W.mean && !aligned16(W.mean)))
+    return QLORA_ERR_ALIGN;
   return QLORA_OK;
 }
 
@@ -353,25 +365,34 @@ struct FwdPlan {
   int s_down, per_down;
   int bn, s_fwd, per_fwd;
   bool low;                  // few-token path (lowm.cu)
-  int low_tiles, low_atiles, low_kc, low_ctas, low_mpad;
-  size_t off_ucat, off_pfwd, total;
+  int low_tiles, low_kc, low_ctas, low_mpad;
+  size_t off_ucat, off_pfwd, off_cnt, total;
 };
 
-// Few tokens: persistent CTAs (two per SM, and at least one per row tile so
-// that no CTA's range spans more than two tiles) over (tiles + atiles) * kc
-// units.  G members: the rows of A are the G members' adapters stacked.
+// Few tokens: U = X A^T by the rank-r kernel (one 128-token tile per member,
+// the contraction split over a cluster), then persistent CTAs (two per SM,
+// and at least one per row tile so that no CTA's range spans more than two
+// tiles) over tiles * kc units of W.
 FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   FwdPlan p{};
   p.low = true;
+  split_plan(G, K / 64, 4, 2 * kSms, p.s_down, p.per_down);
   p.low_mpad = M <= 8 ? 8 : (M <= 16 ? 16 : 32);
   p.low_tiles = static_cast<int>(cdiv(N, kLowmRows));
-  p.low_atiles = static_cast<int>(cdiv(static_cast<int64_t>(G) * r, kLowmARows));
   p.low_kc = static_cast<int>(cdiv(K / 64, 4));
-  const int64_t all_tiles = p.low_tiles + p.low_atiles;
-  const int64_t units = all_tiles * p.low_kc;
-  p.low_ctas = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(2 * kSms, all_tiles)));
-  p.off_pfwd = 0;
-  p.total = align256(static_cast<size_t>(p.low_ctas) * 2 * kLowmRows * p.low_mpad * 4);
+  const int64_t units = static_cast<int64_t>(p.low_tiles) * p.low_kc;
+  // Two CTAs per SM, less the slots the rank-r kernel's CTAs hold while it
+  // runs beside this one (so that no persistent CTA starts late).
+  const int64_t slots = 2 * kSms - static_cast<int64_t>(p.s_down) * G;
+  p.low_ctas = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(slots, p.low_tiles)));
+  size_t off = 0;
+  p.off_pfwd = off;
+  off += align256(static_cast<size_t>(p.low_ctas) * 2 * kLowmRows * p.low_mpad * 4);
+  p.off_cnt = off;
+  off += align256(static_cast<size_t>(p.low_tiles) * 4);
+  p.off_ucat = off;
+  off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
+  p.total = off;
   return p;
 }
 
@@ -392,10 +413,10 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
   if (M <= 256) {
     // The weight streams through once: spread it over several waves of CTAs
-    // (balanced SMs) while keeping the fp32 partials of Y under a quarter of
-    // the NF4 bytes (S * M * N * 4 <= N * K / 8).
+    // (balanced SMs), at most 8 slices of the contraction (a cluster, reduced
+    // in distributed shared memory) of at least 8 stages each.
     int64_t s = cdiv(4 * kSms, tiles);
-    s = std::min<int64_t>(s, std::max<int64_t>(1, K / (8 * M)));
+    s = std::min<int64_t>(s, kMaxCluster);
     s = std::min<int64_t>(s, std::max<int64_t>(1, kst / 8));
     s = std::max<int64_t>(s, 1);
     p.per_fwd = static_cast<int>(cdiv(kst, s));
@@ -408,7 +429,6 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   p.off_ucat = off;
   off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
   p.off_pfwd = off;
-  if (p.s_fwd > 1) off += align256(static_cast<size_t>(p.s_fwd) * M * N * 4);
   p.total = off;
   return p;
 }
@@ -588,7 +608,48 @@ qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float
   CUtensorMap tm_out;
   if (nfull > 0 && !map_bf16(&tm_out, w_bf16, nfull, 64, 64, 32, 128)) return QLORA_ERR_CUDA;
   ProfScope ps(kKDequantize, static_cast<cudaStream_t>(stream));
-  return from_cuda(launch_nf4_dequantize(codes, c8, s2, numel, w_bf16, nfull > 0 ? &tm_out : nullptr, tables(),
+  return from_cuda(launch_nf4_dequantize(codes, c8, s2, nullptr, numel, w_bf16, nfull > 0 ? &tm_out : nullptr,
+                                         tables(), static_cast<cudaStream_t>(stream)));
+}
+
+size_t nf4_centered_workspace_size(int64_t numel) {
+  if (numel <= 0) return 0;
+  const int64_t nblocks = cdiv(numel, 64), ngroups = cdiv(numel, 16384);
+  return align256(static_cast<size_t>(nblocks) * 4) + align256(static_cast<size_t>(ngroups) * 8);
+}
+
+qlora_status nf4_quantize_centered(const uint16_t* w_bf16, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                                   float* mean, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (numel < 0 || numel >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  if (numel == 0) return QLORA_OK;
+  if (!w_bf16 || !codes || !c8 || !s2 || !mean) return QLORA_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(c8) || !aligned16(s2) || !aligned16(mean) ||
+      (d_status && !aligned16(d_status)))
+    return QLORA_ERR_ALIGN;
+  if (!ws || ws_bytes < nf4_centered_workspace_size(numel)) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QLORA_ERR_ALIGN;
+  if (qlora_status st = check_device()) return st;
+  float* cbuf = static_cast<float*>(ws);
+  double* gsum = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(cdiv(numel, 64)) * 4));
+  ProfScope ps(kKQuantize, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_nf4_quantize_centered(w_bf16, numel, codes, c8, s2, mean, cbuf, gsum, d_status, tables(),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+qlora_status nf4_dequantize_centered(const uint8_t* codes, const uint8_t* c8, const float* s2, const float* mean,
+                                     int64_t numel, uint16_t* w_bf16, void* stream) {
+  if (numel < 0 || numel >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  if (numel == 0) return QLORA_OK;
+  if (!w_bf16 || !codes || !c8 || !s2 || !mean) return QLORA_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(codes) || !aligned16(c8) || !aligned16(s2) || !aligned16(mean))
+    return QLORA_ERR_ALIGN;
+  if (numel >= (int64_t(1) << 37)) return QLORA_ERR_SHAPE;
+  if (qlora_status st = check_device()) return st;
+  const int64_t nfull = numel / 64;
+  CUtensorMap tm_out;
+  if (nfull > 0 && !map_bf16(&tm_out, w_bf16, nfull, 64, 64, 32, 128)) return QLORA_ERR_CUDA;
+  ProfScope ps(kKDequantize, static_cast<cudaStream_t>(stream));
+  return from_cuda(launch_nf4_dequantize(codes, c8, s2, mean, numel, w_bf16, nfull > 0 ? &tm_out : nullptr, tables(),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -631,44 +692,6 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   uint16_t* ucat = reinterpret_cast<uint16_t*>(wsb + p.off_ucat);
   float* pfwd = reinterpret_cast<float*>(wsb + p.off_pfwd);
 
-  if (p.low) {
-    LowmArgs la{};
-    la.codes = W.codes;
-    la.c8 = W.c8;
-    la.s2 = W.s2;
-    la.X = X;
-    la.A = A;
-    la.B = B;
-    la.part = pfwd;
-    la.Y = Y;
-    la.y_f32 = y_dtype == QLORA_DTYPE_F32;
-    la.U = U_out;
-    la.s = s;
-    la.M = static_cast<int>(M);
-    la.N = static_cast<int>(N);
-    la.K = static_cast<int>(K);
-    la.r = r;
-    la.tiles = p.low_tiles;
-    la.atiles = p.low_atiles;
-    la.kc = p.low_kc;
-    la.ctas = p.low_ctas;
-    la.mpad = p.low_mpad;
-    la.status = d_status;
-    la.tab = tables();
-    fill_group(grp, &la, r);
-    CUtensorMap lc, la_map, lx, lxa;
-    if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) || !map_bf16(&la_map, A, ra, K, 64, kLowmARows, 128) ||
-        !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128) ||
-        !map_bf16(&lxa, Xa, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
-      return QLORA_ERR_CUDA;
-    {
-      ProfScope ps(kKLowFwd, cs);
-      if (qlora_status st = from_cuda(launch_lowm_fwd(lc, la_map, lx, lxa, la, cs))) return st;
-    }
-    ProfScope ps(kKLowFinish, cs);
-    return from_cuda(launch_lowm_finish(la, cs));
-  }
-
   // U = Xa A^T for every member (contraction split over a cluster), plus the
   // bf16 hi/lo of s*U; the G CTAs of a token tile read the same X rows.
   CUtensorMap mx_down, ma_down;
@@ -685,6 +708,11 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   sa.out_cat = ucat;
   sa.status = d_status;
   fill_group(grp, &sa);
+  uint32_t* tile_count = reinterpret_cast<uint32_t*>(wsb + p.off_cnt);
+  if (p.low) {  // the few-token kernel's tile counters start at zero
+    sa.zero = tile_count;
+    sa.zero_count = p.low_tiles;
+  }
   {
     ProfScope ps(kKDown, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa,
@@ -692,10 +720,45 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
       return st;
   }
 
+  if (p.low) {
+    LowmArgs la{};
+    la.codes = W.codes;
+    la.c8 = W.c8;
+    la.s2 = W.s2;
+    la.mean = W.mean;
+    la.B = B;
+    la.part = pfwd;
+    la.Y = Y;
+    la.y_f32 = y_dtype == QLORA_DTYPE_F32;
+    la.U = U_out;
+    la.tile_count = tile_count;
+    la.s = s;
+    la.M = static_cast<int>(M);
+    la.N = static_cast<int>(N);
+    la.K = static_cast<int>(K);
+    la.r = r;
+    la.tiles = p.low_tiles;
+    la.atiles = 0;
+    la.kc = p.low_kc;
+    la.ctas = p.low_ctas;
+    la.mpad = p.low_mpad;
+    la.status = d_status;
+    la.tab = tables();
+    fill_group(grp, &la, r);
+    CUtensorMap lc, lx;
+    if (!map_u8(&lc, W.codes, N, K / 2, 128, kLowmRows, 128) ||
+        !map_bf16(&lx, X, M, K, 64, static_cast<uint32_t>(p.low_mpad), 128))
+      return QLORA_ERR_CUDA;
+    ProfScope ps(kKLowFwd, cs);
+    return from_cuda(launch_lowm_fwd(lc, lx, la, cs));
+  }
+
+
   // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
   if (M > kWideM) {
     const bool pair = use_pair(N) && group_pairs(grp);
-    const uint32_t tok_box = pair ? 128 : 256;
+    const bool tmem_a = pair && use_tmem_a();
+    const uint32_t tok_box = tmem_a ? 112 : (pair ? 128 : 256);
     CUtensorMap wx, wc, wu, wb;
     if (!map_bf16(&wx, X, M, K, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
         !map_bf16(&wu, ucat, M, 2 * ra, 32, tok_box, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
@@ -703,6 +766,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     FusedArgs fa{};
     fa.c8 = W.c8;
     fa.s2 = W.s2;
+    fa.mean = W.mean;
     fa.out = Y;
     fa.out_f32 = y_dtype == QLORA_DTYPE_F32;
     fa.ld_out = N;
@@ -717,6 +781,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     fa.tab = tables();
     fill_group(grp, &fa);
     ProfScope ps(kKFusedFwd, cs);
+    if (tmem_a) return from_cuda(launch_fused_pair_fwd(wx, wc, wu, wb, fa, cs));
     return from_cuda(pair ? launch_fused_pair(false, wx, wc, wu, wb, fa, cs)
                           : launch_fused2x(false, wx, wc, wu, wb, fa, cs));
   }
@@ -727,10 +792,10 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   FusedArgs fa{};
   fa.c8 = W.c8;
   fa.s2 = W.s2;
-  fa.out = p.s_fwd > 1 ? static_cast<void*>(pfwd) : Y;
+  fa.mean = W.mean;
+  fa.out = Y;
   fa.out_f32 = y_dtype == QLORA_DTYPE_F32;
   fa.ld_out = N;
-  fa.split_stride = p.s_fwd > 1 ? M * N : 0;
   fa.M = static_cast<int>(M);
   fa.rows = static_cast<int>(N);
   fa.n_out = static_cast<int>(N);
@@ -741,15 +806,8 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   fa.status = d_status;
   fa.tab = tables();
   fill_group(grp, &fa);
-  {
-    ProfScope ps(kKFusedFwd, cs);
-    if (qlora_status st = from_cuda(launch_fused_fwd(p.bn, mx, mc, mu, mb, fa, p.s_fwd, cs))) return st;
-  }
-  if (p.s_fwd > 1) {
-    ProfScope ps(kKFinishFwd, cs);
-    return from_cuda(launch_finish_out(pfwd, p.s_fwd, M * N, Y, y_dtype == QLORA_DTYPE_F32, cs));
-  }
-  return QLORA_OK;
+  ProfScope ps(kKFusedFwd, cs);
+  return from_cuda(launch_fused_fwd(p.bn, mx, mc, mu, mb, fa, p.s_fwd, cs));
 }
 
 qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight W, const uint16_t* A, const uint16_t* B,
@@ -841,6 +899,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     FusedArgs fa{};
     fa.c8 = W.c8;
     fa.s2 = W.s2;
+    fa.mean = W.mean;
     fa.out = dx_gemm;
     fa.out_f32 = gemm_f32;
     fa.ld_out = K;
@@ -866,10 +925,10 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     FusedArgs fa{};
     fa.c8 = W.c8;
     fa.s2 = W.s2;
+    fa.mean = W.mean;
     fa.out = dx_gemm;
     fa.out_f32 = gemm_f32;
     fa.ld_out = K;
-    fa.split_stride = 0;
     fa.M = Mi;
     fa.rows = Ki;
     fa.n_out = Ni;

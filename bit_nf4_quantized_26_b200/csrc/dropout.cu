@@ -61,64 +61,89 @@ __global__ void __launch_bounds__(256) dropout_apply_kernel(const uint16_t* __re
 // dX = dX_main + keep * c * (dU A), dX_main fp32 [M, K] from the GEMM without
 // its adapter stages, dU from the bf16 hi/lo pairs of the interleaved layout
 // (column c holds part (c/16)%2 of j = 16 floor(c/32) + c%16), A bf16 [r, K].
-// A CTA computes a 64 x 64 block of (m, k) on the CUDA cores (r <= 64 terms,
-// fp32); each thread a 4 x 4 micro-block whose four k form one mask group.
+// A CTA computes a 64 x 64 block of (m, k): dU A on the tensor cores
+// (register-operand m16n8k16 MMAs, fp32 accumulate, the hi and the lo part of
+// dU each once), then per element the mask and the add.  Warp w takes rows
+// 16 (w % 4) .. + 15 and columns 32 (w / 4) .. + 31 of the block.
 constexpr int kDxTile = 64;
+constexpr int kDxLd = 64 + 8;  // bf16 per shared-memory row: 144 bytes, conflict-free fragment loads
+
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 __global__ void __launch_bounds__(256) dropout_dx_kernel(const float* __restrict__ dx32,
                                                          const uint16_t* __restrict__ ducat,
                                                          const uint16_t* __restrict__ A, void* __restrict__ out,
                                                          int out_f32, int M, int K, int r, const DropoutArgs d) {
-  __shared__ float su[kDxTile][kDxTile + 1];  // [m][j]
-  __shared__ float sa[kDxTile][kDxTile];      // [j][k]
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  __shared__ __align__(16) uint16_t uh[kDxTile][kDxLd];  // [m][j] hi part of dU
+  __shared__ __align__(16) uint16_t ul[kDxTile][kDxLd];  // [m][j] lo part
+  __shared__ __align__(16) uint16_t at[kDxTile][kDxLd];  // [k][j] A transposed
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int m0 = blockIdx.y * kDxTile, k0 = blockIdx.x * kDxTile;
   grid_dependency_wait();
   grid_dependents_launch();
   for (int e = tid; e < kDxTile * kDxTile; e += 256) {
     const int mm = e / kDxTile, j = e % kDxTile;
-    float v = 0.0f;
+    uint16_t hi = 0, lo = 0;
     if (m0 + mm < M && j < r) {
       const uint16_t* row = ducat + static_cast<int64_t>(m0 + mm) * 2 * r;
       const int col = 32 * (j >> 4) + (j & 15);
-      v = __fadd_rn(bf16_bits_to_float(row[col]), bf16_bits_to_float(row[col + 16]));
+      hi = row[col];
+      lo = row[col + 16];
     }
-    su[mm][j] = v;
+    uh[mm][j] = hi;
+    ul[mm][j] = lo;
     const int jj = e / kDxTile, kk = e % kDxTile;
-    sa[jj][kk] = jj < r ? bf16_bits_to_float(A[static_cast<int64_t>(jj) * K + k0 + kk]) : 0.0f;
+    at[kk][jj] = jj < r ? A[static_cast<int64_t>(jj) * K + k0 + kk] : uint16_t(0);
   }
   __syncthreads();
+  const int mr = (warp & 3) * 16, kc = (warp >> 2) * 32;
   float acc[4][4] = {};
-  for (int j = 0; j < r; ++j) {
-    float av[4], uv[4];
+  for (int ks = 0; ks < r; ks += 16) {
+    const int jc = ks + 2 * t;
+    const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc]);
+    const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc]);
+    const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc + 8]);
+    const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc + 8]);
+    const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc]);
+    const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc]);
+    const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc + 8]);
+    const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc + 8]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      av[i] = sa[j][4 * tx + i];
-      uv[i] = su[4 * ty + i][j];
+    for (int nt = 0; nt < 4; ++nt) {
+      const int kk = kc + nt * 8 + g;
+      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&at[kk][jc]);
+      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&at[kk][jc + 8]);
+      mma_16816_bf16(acc[nt], ah0, ah1, ah2, ah3, b0, b1);
+      mma_16816_bf16(acc[nt], al0, al1, al2, al3, b0, b1);
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(uv[a], av[b], acc[a][b]);
   }
-  const int k = k0 + 4 * tx;
+  // acc[nt]: (row g, columns 2t, 2t+1) and (row g + 8, the same columns) of
+  // the 16 x 8 tile nt; the two columns lie in one group of four (one mask word).
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int m = m0 + 4 * ty + a;
-    if (m >= M) continue;
-    const int64_t e = static_cast<int64_t>(m) * K + k;  // a multiple of 4: one mask group
-    const uint32_t keep = keep4(static_cast<uint64_t>(e >> 2), d);
-    const float4 base = *reinterpret_cast<const float4*>(dx32 + e);
-    const float bv[4] = {base.x, base.y, base.z, base.w};
-    float v[4];
+  for (int nt = 0; nt < 4; ++nt) {
+    const int k = k0 + kc + nt * 8 + 2 * t;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) v[b] = (keep >> b) & 1u ? __fadd_rn(bv[b], __fmul_rn(d.c, acc[a][b])) : bv[b];
-    if (out_f32) {
-      *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e) = make_float4(v[0], v[1], v[2], v[3]);
-    } else {
-      const uint32_t lo = static_cast<uint32_t>(bf16_bits(v[0])) | (static_cast<uint32_t>(bf16_bits(v[1])) << 16);
-      const uint32_t hi = static_cast<uint32_t>(bf16_bits(v[2])) | (static_cast<uint32_t>(bf16_bits(v[3])) << 16);
-      *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + e) = make_uint2(lo, hi);
+    for (int h = 0; h < 2; ++h) {
+      const int m = m0 + mr + g + 8 * h;
+      if (m >= M) continue;
+      const int64_t e = static_cast<int64_t>(m) * K + k;
+      const uint32_t keep = keep4(static_cast<uint64_t>(e >> 2), d) >> (e & 3);
+      const float2 base = *reinterpret_cast<const float2*>(dx32 + e);
+      const float v0 = (keep & 1u) ? __fadd_rn(base.x, __fmul_rn(d.c, acc[nt][2 * h])) : base.x;
+      const float v1 = (keep & 2u) ? __fadd_rn(base.y, __fmul_rn(d.c, acc[nt][2 * h + 1])) : base.y;
+      if (out_f32) {
+        *reinterpret_cast<float2*>(reinterpret_cast<float*>(out) + e) = make_float2(v0, v1);
+      } else {
+        *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(out) + e) =
+            static_cast<uint32_t>(bf16_bits(v0)) | (static_cast<uint32_t>(bf16_bits(v1)) << 16);
+      }
     }
   }
 }

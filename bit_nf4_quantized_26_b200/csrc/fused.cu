@@ -36,8 +36,13 @@ struct FusedPlan {
   static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
+  // Split contraction: each CTA of the cluster parks its fp32 tile here (the
+  // idle ring), rows padded by 4 floats so that row-wise stores spread over
+  // the banks.
+  static constexpr uint32_t kPartLd = BN + 4;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kStages >= 3, "pipeline too shallow");
+  static_assert(128 * kPartLd * 4 <= kBarOff, "partial tile must fit in the ring");
 };
 
 template <int BN, bool DX, int DQW>
@@ -183,6 +188,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     // DQW == 4: thread dt owns tile row dt (one whole NF4 block per stage).
     // DQW == 8: threads 2i and 2i+1 share tile row i, half a block each.
     const int dt = threadIdx.x - 64;
+    const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
     const int rl = DQW == 4 ? dt : (dt >> 1);
     const uint32_t half = DQW == 4 ? 0u : static_cast<uint32_t>(dt & 1);
     const int64_t kbpr = a.k_in / 64;  // NF4 blocks per W row
@@ -199,9 +205,11 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         return n < a.n_out && kb < kbpr;
       }
     };
-    // six-deep register prefetch of the block constants (covers a DRAM miss
-    // when the weight streams through once, as for a handful of tokens)
-    constexpr int kPD = 6;
+    // register prefetch of the block constants, six stages ahead for a
+    // handful of tokens (the weight streams through once: cover a DRAM miss),
+    // four for 128 or more (two CTAs of 128 tokens per SM sit at the register
+    // limit; each of their stages takes longer)
+    constexpr int kPD = BN >= 128 ? 4 : 6;
     uint32_t pc[kPD];
     float ps[kPD];
     auto fetch = [&](int t, uint32_t& c, float& sv) {
@@ -243,7 +251,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         dst = st + P::kB + bs * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
         swz = nl & 7;
       }
-      const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
+      const float chat = valid ? nf4_block_scale(c8b, s2v, wmean) : 0.0f;
       if (DQW == 4) {
         if (valid) {
           nf4_block_to_swizzled_row(src, nf4_make_lut(a.tab, chat), dst, swz);
@@ -282,36 +290,108 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       const int orow = row0 + erow;
       const bool rok = orow < a.rows;
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+      if (gridDim.z > 1) {
+        // split contraction: this CTA's fp32 tile goes to its shared memory
+        float* prow = reinterpret_cast<float*>(smem) + erow * P::kPartLd;
 #pragma unroll 1
-      for (int ci = 0; ci < kChunks; ++ci) {
-        const int cb = cgrp * kChunks + ci;
-        if (cb >= kAll) break;  // warp-uniform
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tq + cb * 32, v);
-        tmem_ld_wait();
-        if (rok) {
-          const int mb = m0 + cb * 32;
-          const int nv = min(32, a.M - mb);
-          const int64_t ld = a.ld_out;
-          if (a.split_stride || a.out_f32) {
-            float* o = reinterpret_cast<float*>(a.out) + static_cast<int64_t>(z) * a.split_stride + orow +
-                       static_cast<int64_t>(mb) * ld;
+        for (int ci = 0; ci < kChunks; ++ci) {
+          const int cb = cgrp * kChunks + ci;
+          if (cb >= kAll) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tq + cb * 32, v);
+          tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nv) *o = __uint_as_float(v[j]);
-              o += ld;
-            }
-          } else {
-            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(prow + cb * 32 + j) = make_float4(
+                __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        }
+      } else {
+#pragma unroll 1
+        for (int ci = 0; ci < kChunks; ++ci) {
+          const int cb = cgrp * kChunks + ci;
+          if (cb >= kAll) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tq + cb * 32, v);
+          tmem_ld_wait();
+          if (rok) {
+            const int mb = m0 + cb * 32;
+            const int nv = min(32, a.M - mb);
+            const int64_t ld = a.ld_out;
+            if (a.out_f32) {
+              float* o = reinterpret_cast<float*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nv) *o = bf16_bits(__uint_as_float(v[j]));
-              o += ld;
+              for (int j = 0; j < 32; ++j) {
+                if (j < nv) *o = __uint_as_float(v[j]);
+                o += ld;
+              }
+            } else {
+              uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + orow + static_cast<int64_t>(mb) * ld;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j < nv) *o = bf16_bits(__uint_as_float(v[j]));
+                o += ld;
+              }
             }
           }
         }
       }
     }
+  }
+
+  if (gridDim.z > 1) {
+    // Split contraction: the S CTAs of the cluster (one per slice of the
+    // contraction, cluster rank = blockIdx.z) each sum a slice of the tile's
+    // rows over all S partial tiles through distributed shared memory, in
+    // rank order 0..S-1 (deterministic), and write the outputs.  A thread
+    // takes four tokens of one W-side row and has the S partial loads in
+    // flight together; consecutive threads take consecutive rows, so the
+    // stores of a token's outputs are contiguous.
+    __syncwarp();
+    cluster_sync_all();
+    const int S = static_cast<int>(gridDim.z);
+    const int rows_per = (128 + S - 1) / S;
+    const int r0 = z * rows_per, r1 = min(128, r0 + rows_per);
+    const int nrow = r1 - r0;
+    const float* part = reinterpret_cast<const float*>(smem);
+    const int64_t ld = a.ld_out;
+    constexpr int kC4 = BN / 4;
+    for (int e = threadIdx.x; e < nrow * kC4; e += blockDim.x) {
+      const int row = r0 + e % nrow, c4 = (e / nrow) * 4;
+      const uint32_t off = static_cast<uint32_t>((row * P::kPartLd + c4) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k0 = 0; k0 < 8; k0 += 4) {  // four loads in flight, added in rank order
+        float4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k0 + k < S) v[k] = dsmem_ld_f4(dsmem_addr(part, static_cast<uint32_t>(k0 + k)) + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (k0 + k == 0) {
+            acc = v[0];
+          } else if (k0 + k < S) {
+            acc.x = __fadd_rn(acc.x, v[k].x);
+            acc.y = __fadd_rn(acc.y, v[k].y);
+            acc.z = __fadd_rn(acc.z, v[k].z);
+            acc.w = __fadd_rn(acc.w, v[k].w);
+          }
+        }
+      }
+      const int orow = row0 + row;
+      const float o[4] = {acc.x, acc.y, acc.z, acc.w};
+      if (orow < a.rows) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = m0 + c4 + i;
+          if (m < a.M) {
+            if (a.out_f32) reinterpret_cast<float*>(a.out)[orow + static_cast<int64_t>(m) * ld] = o[i];
+            else reinterpret_cast<uint16_t*>(a.out)[orow + static_cast<int64_t>(m) * ld] = bf16_bits(o[i]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // peers may still be reading this CTA's partial tile
   }
 
   tc_fence_before();
@@ -486,6 +566,7 @@ __global__ void __launch_bounds__(192, 1)
     grid_dependents_launch();
   } else {
     const int dt = threadIdx.x - 64;  // 0..127
+    const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
     const int64_t kbpr = a.k_in / 64;
     if (!DX) {
       // -------------------------------------------------- forward dequant
@@ -511,7 +592,7 @@ __global__ void __launch_bounds__(192, 1)
       Nf4Lut lut{};
       for (int t = 0; t < nmain; ++t) {
         if ((t & 1) == 0) {
-          const float chat = valid ? nf4_block_scale(pc[0], ps[0]) : 0.0f;
+          const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
 #pragma unroll
           for (int i = 0; i + 1 < kPD; ++i) {
             pc[i] = pc[i + 1];
@@ -571,7 +652,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
         const bool valid = kok && (t * 32 + nl) < a.n_out;
-        const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
+        const float chat = valid ? nf4_block_scale(c8b, s2v, wmean) : 0.0f;
         const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (!mbar_wait_all(&full[s], u & 1, wc)) break;
@@ -669,23 +750,25 @@ static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  if (splits < 1 || splits > 8) return cudaErrorInvalidValue;
   dim3 grid((a.rows + 127) / 128, (a.M + BN - 1) / BN, splits);
-  return launch_kernel(fused_kernel<BN, DX, DQW>, grid, dim3(64 + 32 * DQW), P::kSmem, stream, dim3(1, 1, 1), m0, m1,
-                       m2, m3, a);
+  // A split contraction runs as a cluster of its slices (reduced in-cluster).
+  return launch_kernel(fused_kernel<BN, DX, DQW>, grid, dim3(64 + 32 * DQW), P::kSmem, stream,
+                       dim3(1, 1, static_cast<unsigned>(splits)), m0, m1, m2, m3, a);
 }
 
-// Dequantiser warps per CTA.  With 128 or more tokens per tile the MMA work
-// hides the lookups and the integer pipe's throughput is the limit, so four
-// warps (no duplicated table work) are best; with a handful of tokens the
-// kernel is a pure weight stream whose lookups must hide their own latency,
-// so eight.  QLORA_DEQUANT_WARPS=4 or 8 overrides.
+// Dequantiser warps per CTA: four (one whole NF4 block per thread and stage,
+// no duplicated table work) measured faster than eight (half blocks, tables
+// built in pairs) at every tile width this kernel runs (64, 128 and 256
+// tokens: 95 / 114 / 206 us against 108 / 128 / 222 us on a 22016 x 8192
+// weight).  QLORA_DEQUANT_WARPS=8 selects eight.
 static int dequant_warps(int bn) {
   static int forced = [] {
     const char* e = getenv("QLORA_DEQUANT_WARPS");
     return e ? atoi(e) : 0;
   }();
-  if (forced == 4 || forced == 8) return forced;
-  return bn <= 64 ? 8 : 4;
+  (void)bn;
+  return forced == 8 ? 8 : 4;
 }
 
 template <int BN, bool DX>

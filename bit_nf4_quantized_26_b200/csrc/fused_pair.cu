@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(192, 1)
     grid_dependents_launch();
   } else {
     const int dt = threadIdx.x - 64;  // 0..127
+    const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
     const int64_t kbpr = a.k_in / 64;
     if (!DX) {
       // -------------------------------------------------- forward dequant
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
       Nf4Lut lut{};
       for (int t = 0; t < nmain; ++t) {
         if ((t & 1) == 0) {
-          const float chat = valid ? nf4_block_scale(pc[0], ps[0]) : 0.0f;
+          const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
 #pragma unroll
           for (int i = 0; i + 1 < kPD; ++i) {
             pc[i] = pc[i + 1];
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
         const bool valid = kok && (t * 32 + nl) < a.n_out;
-        const float chat = valid ? nf4_block_scale(c8b, s2v) : 0.0f;
+        const float chat = valid ? nf4_block_scale(c8b, s2v, wmean) : 0.0f;
         const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (!mbar_wait_all(&cfull[s], u & 1, wc)) break;

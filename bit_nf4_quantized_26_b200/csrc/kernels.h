@@ -55,10 +55,10 @@ inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block
 struct FusedArgs {
   const uint8_t* c8;   // FP8 block constants of W [n_out * k_in / 64]
   const float* s2;     // group scales of W
+  const float* mean;   // mean of W's constants (mean-centred scheme) or null
   void* out;           // out[m * ld_out + row]
   int out_f32;         // 1: fp32 output, 0: bf16 output
   int64_t ld_out;      // row stride of out (elements)
-  int64_t split_stride;// elements between split-K partial slices (0: no split)
   int M;               // tokens
   int rows;            // extent of the W-side index (N for fwd, K for dX)
   int n_out, k_in;     // shape of W
@@ -102,6 +102,8 @@ struct SkinnyArgs {
   int32_t* status;
   int groups;           // G (1..4)
   int grp_n[5];         // member offsets along N (grp_n[0] = 0, grp_n[G] = N)
+  uint32_t* zero;       // DOWN: words cleared by the first CTA (the few-token forward's tile counters)
+  int zero_count;
 };
 
 // One CTA waits on an mbarrier nothing completes, with a `limit_ns` bound,
@@ -139,9 +141,15 @@ cudaError_t launch_adamw8(const AdamW8Args& a, cudaStream_t stream);
 
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
                                 int32_t* status, const Nf4Tables& tab, cudaStream_t stream);
-//   tm_out: out viewed as [numel / 64, 64] bf16, box {64, 32} SW128 (null when numel < 64).
-cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
-                                  uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
+// Mean-centred constants: codes plus the fp32 constants (cbuf [nblocks]) and
+// fp64 group sums (gsum [ngroups]); then the mean; then the centred FP8 encoding.
+cudaError_t launch_nf4_quantize_centered(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                                         float* mean, float* cbuf, double* gsum, int32_t* status,
+                                         const Nf4Tables& tab, cudaStream_t stream);
+//   tm_out: out viewed as [numel / 64, 64] bf16, box {64, 32} SW128 (null when numel < 64);
+//   mean: null for the plain scheme.
+cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, const float* mean,
+                                  int64_t numel, uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
                                   cudaStream_t stream);
 
 // Forward: Y[m, n] (+)= sum_k X[m,k] W'[n,k]  (+ LoRA extension in split 0).
@@ -173,6 +181,13 @@ cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMa
                               const CUtensorMap& tm_uc, const CUtensorMap& tm_ext, const FusedArgs& a,
                               cudaStream_t stream);
 
+// Large-M forward on CTA pairs with the dequantised tile in tensor memory:
+// 256 W rows x 448 tokens per cluster of two CTAs.  Needs rows % 256 == 0.
+//   tm_b: X [M, K] box {32, 112} SW64; tm_codes: codes [N, K/2] box {16, 128};
+//   tm_uc: Ucat [M, 2r] box {32, 112} SW64; tm_ext: B [N, r] box {32, 128} SW64.
+cudaError_t launch_fused_pair_fwd(const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
+                                  const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream);
+
 // Skinny LoRA products; the contraction is split over a cluster of `splits`
 // (1..8) CTAs along y and reduced in-cluster.  See skinny.cu for the maps.
 cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& tmB, const SkinnyArgs& a,
@@ -180,29 +195,27 @@ cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& t
 
 // Few-token forward (M <= 32): register-operand MMAs on in-register
 // dequantised tiles, persistent CTAs over (128-row tile, 256-wide K chunk)
-// units; row tiles tiles .. tiles + atiles - 1 hold the rows of A, 32 each.
-// See lowm.cu.
+// units; the last CTA to finish a row tile adds its partials in CTA order and
+// s U B^T (U from the rank-r kernel launched just before).  See lowm.cu.
 constexpr int kLowmThreads = 256;
 constexpr int kLowmRows = 128;
-constexpr int kLowmARows = 32;
-constexpr int kLowmMpad = 32;  // largest partial row stride (tokens, padded to 8)
 constexpr int kLowmMaxM = 32;
 
 struct LowmArgs {
   const uint8_t* codes;  // [N, K/2]
   const uint8_t* c8;     // [N * K / 64]
   const float* s2;
-  const uint16_t* X;     // [M, K] bf16
-  const uint16_t* A;     // [r, K] bf16
+  const float* mean;     // mean of W's constants (mean-centred scheme) or null
   const uint16_t* B;     // [N, r] bf16
   float* part;           // [ctas][2][128][mpad] fp32 partials
   void* Y;               // [M, N]
   int y_f32;
-  float* U;              // [M, r] fp32
+  const float* U;        // [M, ra] fp32, from the rank-r kernel launched before
+  uint32_t* tile_count;  // [tiles] partials counted in, cleared by that kernel
   float s;
   int M, N, K, r;
   int tiles;             // ceil(N / 128)
-  int atiles;            // ra / 32 rounded up
+  int atiles;            // 0 (U comes from the rank-r kernel)
   int kc;                // ceil(K / 256)
   int ctas;              // CTAs of the main kernel (>= tiles + atiles)
   int mpad;              // tokens per partial row: 8 * n8 token tiles (8, 16 or 32)
@@ -215,15 +228,9 @@ struct LowmArgs {
   int grp_end[3];
 };
 
-//   tm_codes: codes [N, K/2] u8 box {128, 128} SW128; tm_a: A [r, K] bf16
-//   box {64, 32} SW128; tm_x: X [M, K] bf16 box {64, mpad} SW128; tm_xa: the
-//   adapter's input (X, or X after dropout) with the same box.
-cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                            const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream);
-cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream);
-
-// Fixed-order sum of the small-M forward's split-K partials of Y.
-cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32,
-                              cudaStream_t stream);
+//   tm_codes: codes [N, K/2] u8 box {128, 128} SW128; tm_x: X [M, K] bf16
+//   box {64, mpad} SW128.
+cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_x, const LowmArgs& a,
+                            cudaStream_t stream);
 
 }  // namespace qnf4

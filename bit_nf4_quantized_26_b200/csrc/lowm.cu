@@ -45,7 +45,6 @@ namespace {
 constexpr int kLowmWarps = kLowmThreads / 32;
 constexpr int kLowmAhead = 2;                     // units in flight ahead of the one computed
 constexpr uint32_t kLowmCodes = kLowmRows * 128;  // 16 KB: 128 rows x 256 codes, or 32 A rows x 256 bf16
-constexpr uint32_t kLowmABox = kLowmARows * 128;  // {64 features, 32 rows} bf16
 
 template <int NT>
 struct LowmPlan {
@@ -79,11 +78,10 @@ __device__ __forceinline__ int64_t lowm_units(const LowmArgs& a) {
   return static_cast<int64_t>(a.tiles + a.atiles) * a.kc;
 }
 
-// Whether this warp has rows in `tile`: all 16 rows of its slice exist (N and
-// the rows of A are multiples of 16).  A tiles use warps 0 and 1 only.
+// Whether this warp has rows in `tile`: all 16 rows of its slice exist (N is
+// a multiple of 64).
 __device__ __forceinline__ bool warp_rows_valid(const LowmArgs& a, int tile, int warp) {
-  if (tile < a.tiles) return tile * kLowmRows + warp * 16 + 16 <= a.N;
-  return warp < 2 && (tile - a.tiles) * kLowmARows + warp * 16 + 16 <= a.ra;
+  return tile * kLowmRows + warp * 16 + 16 <= a.N;
 }
 
 // Block constants of rows g and g + 8 of this warp's slice, block t of the
@@ -110,9 +108,7 @@ __device__ __forceinline__ void load_consts(const LowmArgs& a, int tile, int kci
 // Lane 0 of warp 0: issue the copies of unit `i` of this CTA's range into
 // stage i % kStages once the eight warps have released its previous use.
 template <int NT>
-__device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_a,
-                                           const CUtensorMap* tm_x, const CUtensorMap* tm_xa, const LowmArgs& a,
-                                           uint8_t* smem,
+__device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CUtensorMap* tm_x, uint8_t* smem,
                                            uint64_t* full, uint64_t* empty, int i, int tile, int kci,
                                            const WaitCtx& wc) {
   using P = LowmPlan<NT>;
@@ -120,24 +116,78 @@ __device__ __forceinline__ bool lowm_issue(const CUtensorMap* tm_codes, const CU
   if (i >= P::kStages && !mbar_wait(&empty[s], ((i / P::kStages) & 1) ^ 1, wc)) return false;
   uint8_t* st = smem + s * P::kStage;
   mbar_arrive_expect_tx(&full[s], kLowmCodes + 4 * P::kXBox);
-  if (tile < a.tiles) {
-    tma_load_2d(st, tm_codes, &full[s], kci * 128, tile * kLowmRows);
-  } else {
+  tma_load_2d(st, tm_codes, &full[s], kci * 128, tile * kLowmRows);
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
-      tma_load_2d(st + b * kLowmABox, tm_a, &full[s], kci * 256 + b * 64, (tile - a.tiles) * kLowmARows);
-  }
-  // W tiles multiply X; the adapter's A tiles multiply its input (X, or X after dropout).
-  const CUtensorMap* tx = tile < a.tiles ? tm_x : tm_xa;
-#pragma unroll
-  for (int b = 0; b < 4; ++b) tma_load_2d(st + kLowmCodes + b * P::kXBox, tx, &full[s], kci * 256 + b * 64, 0);
+  for (int b = 0; b < 4; ++b) tma_load_2d(st + kLowmCodes + b * P::kXBox, tm_x, &full[s], kci * 256 + b * 64, 0);
   return true;
+}
+
+// The CTAs whose ranges hold units of row tile `tile`: c0 .. c1.
+__device__ __forceinline__ void tile_ctas(const LowmArgs& a, int tile, int& c0, int& c1) {
+  const int64_t units = lowm_units(a);
+  c0 = cta_of_unit(static_cast<int64_t>(tile) * a.kc, units, a.ctas);
+  c1 = cta_of_unit(static_cast<int64_t>(tile + 1) * a.kc - 1, units, a.ctas);
+}
+
+// Y rows of `tile` = the sum of its partials in CTA order + s U B^T (fp32,
+// one rounding), by the CTA that wrote the tile's last partial.  Thread:
+// row = tid % 128, tokens (tid / 128) * mpad/2 ..; su holds U's columns of the
+// tile's group member for the M tokens.
+template <int NT>
+__device__ void finish_tile(const LowmArgs& a, int tile, const float* su) {
+  constexpr int kMpad = 8 * NT;
+  constexpr int kHalf = kMpad / 2;
+  const int row = threadIdx.x & (kLowmRows - 1);
+  const int m0 = (threadIdx.x >> 7) * kHalf;
+  const int n = tile * kLowmRows + row;
+  if (n >= a.N || m0 >= a.M) return;
+  int c0, c1;
+  tile_ctas(a, tile, c0, c1);
+  const int64_t units = lowm_units(a);
+  float y[kHalf];
+#pragma unroll
+  for (int e = 0; e < kHalf; ++e) y[e] = 0.0f;
+  for (int c = c0; c <= c1; ++c) {
+    const int first = static_cast<int>(unit_start(c, units, a.ctas) / a.kc);
+    const float* src = a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * kMpad + m0;
+#pragma unroll
+    for (int e = 0; e < kHalf; e += 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(src + e));
+      y[e] = __fadd_rn(y[e], v.x);
+      y[e + 1] = __fadd_rn(y[e + 1], v.y);
+      y[e + 2] = __fadd_rn(y[e + 2], v.z);
+      y[e + 3] = __fadd_rn(y[e + 3], v.w);
+    }
+  }
+  float lo[kHalf];
+#pragma unroll
+  for (int e = 0; e < kHalf; ++e) lo[e] = 0.0f;
+  const uint4* br = reinterpret_cast<const uint4*>(a.B + static_cast<int64_t>(n) * a.r);
+  for (int j8 = 0; j8 < a.r / 8; ++j8) {
+    const uint4 bv = __ldg(br + j8);
+    const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float b = __uint_as_float(e & 1 ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+#pragma unroll
+      for (int mm = 0; mm < kHalf; ++mm) lo[mm] = fmaf(su[(m0 + mm) * 64 + 8 * j8 + e], b, lo[mm]);
+    }
+  }
+#pragma unroll
+  for (int mm = 0; mm < kHalf; ++mm) {
+    const int m = m0 + mm;
+    if (m < a.M) {
+      const float v = y[mm] + a.s * lo[mm];
+      const int64_t o = static_cast<int64_t>(m) * a.N + n;
+      if (a.y_f32) reinterpret_cast<float*>(a.Y)[o] = v;
+      else reinterpret_cast<uint16_t*>(a.Y)[o] = bf16_bits(v);
+    }
+  }
 }
 
 template <int NT>
 __global__ void __launch_bounds__(kLowmThreads, 2)
-    lowm_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_a,
-                    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xa,
+    lowm_fwd_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                     const LowmArgs a) {
   using P = LowmPlan<NT>;
   extern __shared__ uint8_t smem_raw[];
@@ -145,6 +195,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
   uint64_t* empty = full + P::kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + P::kStages);
+  int* last_flag = const_cast<int*>(abort_flag) + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool issuer = threadIdx.x == 0;
 
@@ -162,21 +213,22 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_codes);
-    tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_xa);
   }
   __syncthreads();
   const WaitCtx wc{abort_flag, a.status};
-  grid_dependency_wait();
-  grid_dependents_launch();
-  if (count <= 0) return;
+  // Programmatic dependent launch: the kernel launched just before this one
+  // computes U (and clears the tile counters); the codes, constants and X
+  // come from earlier kernels, complete when it let this one start.  So the
+  // main loop runs beside it, and the wait comes before U and the counters
+  // are touched (and before this kernel lets its own dependents start).
+  const Nf4Mean wmean = nf4_load_mean(a.mean);
 
   // Copy issue state (lane 0 of warp 0 only).
   int issued = 0, itile = tile0, ikci = kci0;
   bool ok = true;
   auto issue_next = [&]() {
-    ok = lowm_issue<NT>(&tm_codes, &tm_a, &tm_x, &tm_xa, a, smem, full, empty, issued, itile, ikci, wc);
+    ok = lowm_issue<NT>(&tm_codes, &tm_x, smem, full, empty, issued, itile, ikci, wc);
     if (ok) {
       ++issued;
       if (++ikci == a.kc) {
@@ -192,7 +244,7 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   const int g = lane >> 2, t = lane & 3;
   const uint32_t ct = (5u * static_cast<uint32_t>(t)) & 7u;
   // Byte offsets, within a 128-byte swizzled row of phase g, of codes word
-  // (j ^ ct) of block t (XOR j << 2 for step j), and of X / A chunk (j ^ ct)
+  // (j ^ ct) of block t (XOR j << 2 for step j), and of X chunk (j ^ ct)
   // (XOR j << 4 for step j).
   const uint32_t code_off = ((static_cast<uint32_t>(2 * t) ^ static_cast<uint32_t>(g)) << 4) ^ (ct << 2);
   const uint32_t chunk_off = (ct ^ static_cast<uint32_t>(g)) << 4;
@@ -217,52 +269,35 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     const uint8_t* st = smem + s * P::kStage;
     // X box of this lane's block; token row 8n + g has phase g.
     const uint8_t* xs = st + kLowmCodes + t * P::kXBox + g * 128;
-    const bool nf4_unit = tile < a.tiles && warp_rows_valid(a, tile, warp);
-    if (!nf4_unit && more) load_consts(a, ntile, nkci, warp, g, t, cur);
     if (warp_rows_valid(a, tile, warp)) {
-      if (tile < a.tiles) {
-        const Nf4Lut la = nf4_make_lut(a.tab, nf4_block_scale(cur.ca, cur.sa));
-        const Nf4Lut lb = nf4_make_lut(a.tab, nf4_block_scale(cur.cb, cur.sb));
-        // The next unit's constants load into `cur` (dead from here on) and
-        // have a whole unit of work to arrive.
-        if (more) load_consts(a, ntile, nkci, warp, g, t, cur);
-        // rows warp*16 + g and + 8, both of phase g
-        const uint8_t* ra = st + (warp * 16 + g) * 128;
-        uint32_t wa[8], wb[8];
+      const Nf4Lut la = nf4_make_lut(a.tab, nf4_block_scale(cur.ca, cur.sa, wmean));
+      const Nf4Lut lb = nf4_make_lut(a.tab, nf4_block_scale(cur.cb, cur.sb, wmean));
+      // The next unit's constants load into `cur` (dead from here on) and
+      // have a whole unit of work to arrive.
+      if (more) load_consts(a, ntile, nkci, warp, g, t, cur);
+      // rows warp*16 + g and + 8, both of phase g
+      const uint8_t* ra = st + (warp * 16 + g) * 128;
+      uint32_t wa[8], wb[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t o = code_off ^ (static_cast<uint32_t>(j) << 2);
-          wa[j] = lds32(ra + o);
-          wb[j] = lds32(ra + 1024 + o);
-        }
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t o = code_off ^ (static_cast<uint32_t>(j) << 2);
+        wa[j] = lds32(ra + o);
+        wb[j] = lds32(ra + 1024 + o);
+      }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 oa = nf4_lookup8(wa[j], la);
-          const uint4 ob = nf4_lookup8(wb[j], lb);
-          const uint32_t xo = chunk_off ^ (static_cast<uint32_t>(j) << 4);
+      for (int j = 0; j < 8; ++j) {
+        const uint4 oa = nf4_lookup8(wa[j], la);
+        const uint4 ob = nf4_lookup8(wb[j], lb);
+        const uint32_t xo = chunk_off ^ (static_cast<uint32_t>(j) << 4);
 #pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint4 xv = lds128(xs + n * 1024 + xo);
-            mma_16816(acc[n], oa.x, ob.x, oa.y, ob.y, xv.x, xv.y);
-            mma_16816(acc[n], oa.z, ob.z, oa.w, ob.w, xv.z, xv.w);
-          }
-        }
-      } else {
-        // Rows of A (bf16, box t holds block t's 64 features of 32 rows).
-        const uint8_t* ra = st + t * kLowmABox + (warp * 16 + g) * 128;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t xo = chunk_off ^ (static_cast<uint32_t>(j) << 4);
-          const uint4 oa = lds128(ra + xo);
-          const uint4 ob = lds128(ra + 1024 + xo);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint4 xv = lds128(xs + n * 1024 + xo);
-            mma_16816(acc[n], oa.x, ob.x, oa.y, ob.y, xv.x, xv.y);
-            mma_16816(acc[n], oa.z, ob.z, oa.w, ob.w, xv.z, xv.w);
-          }
+        for (int n = 0; n < NT; ++n) {
+          const uint4 xv = lds128(xs + n * 1024 + xo);
+          mma_16816(acc[n], oa.x, ob.x, oa.y, ob.y, xv.x, xv.y);
+          mma_16816(acc[n], oa.z, ob.z, oa.w, ob.w, xv.z, xv.w);
         }
       }
+    } else if (more) {
+      load_consts(a, ntile, nkci, warp, g, t, cur);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -288,117 +323,42 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     for (int i = max(0, issued - P::kStages); i < issued; ++i)
       mbar_drain(&full[i % P::kStages], (i / P::kStages) & 1, a.status);
   }
-}
 
-// Finisher layout: 64 rows x mpad/4 token quads (128, 256 or 512 threads);
-// CTA b covers rows [64 b, 64 b + 64) of the output (half of row tile b / 2).
-constexpr int kFinRows = 64;
-
-// Sum over the CTAs that touched `tile`, in CTA order, of the partial of
-// `row` for tokens 4 q .. 4 q + 3.  Loads are issued four contributors at a
-// time so their latencies overlap; the additions keep the CTA order.
-__device__ __forceinline__ float4 sum_tile_partials(const LowmArgs& a, int tile, int row, int q) {
-  const int64_t units = lowm_units(a);
-  const int c0 = cta_of_unit(static_cast<int64_t>(tile) * a.kc, units, a.ctas);
-  const int c1 = cta_of_unit(static_cast<int64_t>(tile + 1) * a.kc - 1, units, a.ctas);
-  float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  for (int cb = c0; cb <= c1; cb += 4) {
-    float4 v[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = cb + j;
-      v[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      if (c <= c1) {
-        const int first = static_cast<int>(unit_start(c, units, a.ctas) / a.kc);
-        v[j] = *reinterpret_cast<const float4*>(
-            a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * a.mpad + 4 * q);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (cb + j <= c1) {
-        y.x += v[j].x;
-        y.y += v[j].y;
-        y.z += v[j].z;
-        y.w += v[j].w;
-      }
-    }
-  }
-  return y;
-}
-
-// Y[m, n] = sum of the row tile's partials + s * sum_j U[m, j] B[n, j], with
-// U = the A tiles' partials summed (every CTA forms the U of its rows' member;
-// the first CTA of each member stores it).  The row of B is read before the
-// wait for the main kernel (B is not one of its outputs).
-__global__ void __launch_bounds__(512) lowm_finish_kernel(const LowmArgs a) {
-  __shared__ float su[kLowmMpad][64];
-  const int tid = threadIdx.x;
-  const int rl = tid & (kFinRows - 1), q = tid >> 6;
-  const int n0 = blockIdx.x * kFinRows;
-  const int mem = group_member(a.grp_end, a.groups, n0);  // 64-row blocks lie in one member
-  const bool mem_first = mem == 0 ? n0 == 0 : n0 == a.grp_end[mem - 1];
-  const int n = n0 + rl;
-  const bool active = n < a.N && 4 * q < a.M;
-  uint4 bv[8];
-  const uint4* br = reinterpret_cast<const uint4*>(a.B + static_cast<int64_t>(n < a.N ? n : 0) * a.r);
-#pragma unroll
-  for (int j8 = 0; j8 < 8; ++j8) bv[j8] = j8 < a.r / 8 ? __ldg(br + j8) : make_uint4(0u, 0u, 0u, 0u);
-  grid_dependency_wait();
+  grid_dependency_wait();  // U and the cleared tile counters are complete and visible
   grid_dependents_launch();
+  if (count <= 0) return;
 
-  float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (active) y = sum_tile_partials(a, blockIdx.x >> 1, (blockIdx.x & 1) * kFinRows + rl, q);
-  // U: thread (j = tid & 63, quad q) sums row j of the A tiles for its tokens.
-  {
-    const int j = tid & 63;
-    const int ja = mem * a.r + j;  // row of the stacked A
-    if (j < a.r && 4 * q < a.M) {
-      const float4 u = sum_tile_partials(a, a.tiles + ja / kLowmARows, ja % kLowmARows, q);
-      const float uv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int m = 4 * q + e;
-        if (m < a.M) {
-          su[m][j] = uv[e];
-          if (mem_first) a.U[static_cast<int64_t>(m) * a.ra + ja] = uv[e];
-        }
-      }
-    }
-  }
+  // Each row tile this CTA wrote a partial of (at most two): count the
+  // partial in; the CTA that counts the tile's last one finishes the tile.
+  __threadfence();  // this thread's partial stores, before the count
   __syncthreads();
-  if (!active) return;
-  float lo[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-  for (int j8 = 0; j8 < 8; ++j8) {
-    if (j8 < a.r / 8) {
-      const uint32_t w[4] = {bv[j8].x, bv[j8].y, bv[j8].z, bv[j8].w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float b = __uint_as_float(e & 1 ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-#pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          if (4 * q + mm < a.M) lo[mm] = fmaf(su[4 * q + mm][8 * j8 + e], b, lo[mm]);
-        }
+  float* su = reinterpret_cast<float*>(smem);  // the ring is idle now: U of the member, [mpad][64]
+  const int tile_last = static_cast<int>((u_beg + count - 1) / a.kc);
+  for (int tl = tile0; tl <= tile_last; ++tl) {
+    if (threadIdx.x == 0) {
+      int c0, c1;
+      tile_ctas(a, tl, c0, c1);
+      const unsigned prev = atomicAdd(a.tile_count + tl, 1u);
+      *last_flag = prev == static_cast<unsigned>(c1 - c0) ? 1 : 0;
+      __threadfence();  // the other CTAs' partials, before this CTA reads them
+    }
+    __syncthreads();
+    if (*last_flag) {
+      const int mem = group_member(a.grp_end, a.groups, tl * kLowmRows);
+      for (int e = threadIdx.x; e < 8 * NT * 64; e += blockDim.x) {
+        const int m = e >> 6, jj = e & 63;
+        su[e] = (m < a.M && jj < a.r) ? __ldcg(a.U + static_cast<int64_t>(m) * a.ra + mem * a.r + jj) : 0.0f;
       }
+      __syncthreads();
+      finish_tile<NT>(a, tl, su);
     }
-  }
-  const float yv[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-  for (int mm = 0; mm < 4; ++mm) {
-    const int m = 4 * q + mm;
-    if (m < a.M) {
-      const float v = yv[mm] + a.s * lo[mm];
-      const int64_t o = static_cast<int64_t>(m) * a.N + n;
-      if (a.y_f32) reinterpret_cast<float*>(a.Y)[o] = v;
-      else reinterpret_cast<uint16_t*>(a.Y)[o] = bf16_bits(v);
-    }
+    __syncthreads();
   }
 }
 
 template <int NT>
-static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                                    const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream) {
+static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorMap& tm_x, const LowmArgs& a,
+                                    cudaStream_t stream) {
   static bool attr_set = false;  // benign race: setting the same value twice is harmless
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(lowm_fwd_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -407,24 +367,19 @@ static cudaError_t launch_lowm_impl(const CUtensorMap& tm_codes, const CUtensorM
     attr_set = true;
   }
   return launch_kernel(lowm_fwd_kernel<NT>, dim3(a.ctas), dim3(kLowmThreads), LowmPlan<NT>::kSmem, stream,
-                       dim3(1, 1, 1), tm_codes, tm_a, tm_x, tm_xa, a);
+                       dim3(1, 1, 1), tm_codes, tm_x, a);
 }
 
 }  // namespace
 
-cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_a, const CUtensorMap& tm_x,
-                            const CUtensorMap& tm_xa, const LowmArgs& a, cudaStream_t stream) {
+cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_x, const LowmArgs& a,
+                            cudaStream_t stream) {
   switch (a.mpad) {
-    case 8: return launch_lowm_impl<1>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
-    case 16: return launch_lowm_impl<2>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
-    case 32: return launch_lowm_impl<4>(tm_codes, tm_a, tm_x, tm_xa, a, stream);
+    case 8: return launch_lowm_impl<1>(tm_codes, tm_x, a, stream);
+    case 16: return launch_lowm_impl<2>(tm_codes, tm_x, a, stream);
+    case 32: return launch_lowm_impl<4>(tm_codes, tm_x, a, stream);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_lowm_finish(const LowmArgs& a, cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>((a.N + kFinRows - 1) / kFinRows);
-  return launch_kernel(lowm_finish_kernel, dim3(grid), dim3(kFinRows * (a.mpad / 4)), 0, stream, dim3(1, 1, 1), a);
 }
 
 }  // namespace qnf4

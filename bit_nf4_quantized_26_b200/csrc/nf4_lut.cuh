@@ -38,6 +38,22 @@ __device__ __forceinline__ float nf4_block_scale(uint32_t c8_byte, float s2) {
   return __fmul_rn(e4m3_to_float(c8_byte), s2);
 }
 
+// Mean of the constants of a mean-centred weight (0 and unused otherwise):
+// chat = RN32(RN32(e4m3(c8) * s2) + mean).
+struct Nf4Mean {
+  bool centered;
+  float value;
+};
+
+__device__ __forceinline__ Nf4Mean nf4_load_mean(const float* mean) {
+  return Nf4Mean{mean != nullptr, mean != nullptr ? __ldg(mean) : 0.0f};
+}
+
+__device__ __forceinline__ float nf4_block_scale(uint32_t c8_byte, float s2, const Nf4Mean& m) {
+  const float c = nf4_block_scale(c8_byte, s2);
+  return m.centered ? __fadd_rn(c, m.value) : c;
+}
+
 // The 16 dequantised values of one block, as byte planes.  Two separate
 // roundings per value: RN32 product, then RNE to bf16.
 __device__ __forceinline__ Nf4Lut nf4_make_lut(const Nf4Tables& tab, float chat) {

@@ -9,18 +9,19 @@ namespace qnf4 {
 // ------------------------------------------------------------------ quantize
 //
 // One CTA (256 threads) owns one double-quantisation group: 256 blocks of 64
-// elements = 32 KB of bf16 input.  Eight threads share a block (8 elements,
-// 16 bytes each), so a warp reads 512 contiguous bytes per pass and writes
-// 128 contiguous bytes of codes; 8 passes cover the group.  All 8 loads of a
-// thread are issued before any arithmetic; five CTAs per SM keep 160 KB of
-// loads in flight.  The block absmax is a max over the bf16 magnitude bits
-// (non-negative floats order like unsigned ints) reduced across the 8 lanes
-// with shuffles.  Per pair of elements the scaling and the bucket fma are one
-// packed two-lane fp32 instruction each; the bucket table is split into
-// float thresholds and byte bases in shared memory (bank conflicts only
-// between buckets 0 and 32); codes are packed with integer multiply-adds on
-// the FMA pipe.  The kernel is issue-bound: 19-21 instructions per element,
-// ~3.5 of 4 per cycle per SM.
+// elements = 32 KB of bf16 input.  Four threads share a block (16 elements,
+// 32 bytes each, two 16-byte loads), so a warp reads 1 KB contiguous per
+// pass and writes 256 contiguous bytes of codes; 4 passes cover the group.
+// All 8 loads of a thread are issued before any arithmetic; five CTAs per SM
+// keep 160 KB of loads in flight.  The block absmax is a max over the bf16
+// magnitude bits (non-negative floats order like unsigned ints) reduced
+// across the 4 lanes with two shuffles; each lane takes the block's
+// reciprocal once for its 16 elements.  Per pair of elements the scaling and
+// the bucket fma are one packed two-lane fp32 instruction each; the nearest
+// code then costs one mask, a 4-byte threshold load and a 1-byte base load
+// from shared memory (the 33 buckets' thresholds sit in distinct banks but
+// for buckets 0 and 32, and all bases in 9 words, so a warp's loads rarely
+// conflict), one compare and the nibble placement.
 
 constexpr int kQuantThreads = 256;
 
@@ -31,16 +32,10 @@ __device__ __forceinline__ uint32_t max_abs_bits(uint4 v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
-// Nearest-level code of x: bucket b = RNE(16 x + 16) is the low 6 bits of t
-// (t = fma(x, 16, 1.5 * 2^23 + 16), exact offset, one rounding), then
-// base[b] + (x > thr[b]).
-__device__ __forceinline__ uint32_t quant_code(float x, float t, const float* thr, const uint8_t* base) {
-  const uint32_t b = __float_as_uint(t) & 63u;
-  return static_cast<uint32_t>(base[b]) + (x > thr[b] ? 1u : 0u);
-}
-
 // x = RN32(e * rc) and t = RN32(16 x + C) for both elements of a bf16 pair,
 // with packed two-lane fp32 instructions (each lane rounds as the scalar op).
+// C = 1.5 * 2^23 + 16, so t's bits are 0x4B400000 + RNE(16 x + 16): the low
+// six bits are the bucket b (b = 0..32 for |x| <= 1).
 __device__ __forceinline__ void scale_pair(uint32_t word, uint64_t rc2, float& x0, float& x1, float& t0,
                                            float& t1) {
   uint64_t e2, x2, t2;
@@ -53,11 +48,16 @@ __device__ __forceinline__ void scale_pair(uint32_t word, uint64_t rc2, float& x
   asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t2));
 }
 
-// Packed codes of the 8 elements of v (element i in nibble i); the nibbles
-// are placed with integer multiply-adds, which run on the FMA pipe.
-__device__ __forceinline__ uint32_t codes8(uint4 v, float rc, const float* thr, const uint8_t* base) {
-  uint64_t rc2;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
+// Nearest-level code of x from its bucket: code = base[b] + (x > thr[b]).  The
+// mask keeps the bucket inside the 64-entry tables whatever x is (a
+// non-finite input gives an unspecified code, never a stray address).
+__device__ __forceinline__ uint32_t quant_code(float x, float t, const float* thr, const uint8_t* base) {
+  const uint32_t b = __float_as_uint(t) & 63u;
+  return static_cast<uint32_t>(base[b]) + (x > thr[b] ? 1u : 0u);
+}
+
+// Packed codes of the 8 elements of v (element i in nibble i).
+__device__ __forceinline__ uint32_t codes8(uint4 v, uint64_t rc2, const float* thr, const uint8_t* base) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
@@ -87,18 +87,23 @@ __device__ __forceinline__ uint32_t codes_degenerate(uint4 v) {
   return out;
 }
 
+// CENTERED: instead of the FP8 step, the group's fp32 constants go to cbuf and
+// their fp64 sum (sequential, in block order) to gsum[group]; the mean and the
+// centred encoding follow in two more kernels.
+template <bool CENTERED>
 __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const uint16_t* __restrict__ w,
                                                                          int64_t numel, uint8_t* __restrict__ codes,
                                                                          uint8_t* __restrict__ c8,
                                                                          float* __restrict__ s2, int32_t* status,
-                                                                         Nf4Tables tab) {
+                                                                         Nf4Tables tab, float* __restrict__ cbuf,
+                                                                         double* __restrict__ gsum) {
   __shared__ float thr[64];
   __shared__ uint8_t base[64];
   __shared__ uint32_t cblk[256];
   __shared__ uint32_t wmax[kQuantThreads / 32];
 
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, sub = lane & 7;
+  const int warp = tid >> 5, lane = tid & 31, sub = lane & 3;
   if (tid < 64) {
     thr[tid] = tab.thr[tid];
     base[tid] = static_cast<uint8_t>(tab.base[tid]);
@@ -110,44 +115,63 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const ui
   const int64_t blk0 = static_cast<int64_t>(blockIdx.x) * 256;
   const bool full_group = (blk0 + 256) * 64 <= numel;
 
-  uint4 v[8];
+  // Pass p, lane: block p*64 + warp*8 + lane/4, elements sub*16 .. sub*16+15.
+  uint4 v[4][2];
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int64_t e0 = (blk0 + p * 32 + warp * 4 + (lane >> 3)) * 64 + sub * 8;
-    if (full_group) {
-      v[p] = __ldg(reinterpret_cast<const uint4*>(w + e0));
-    } else {
-      uint32_t t[4] = {0, 0, 0, 0};
+  for (int p = 0; p < 4; ++p) {
+    const int64_t e0 = (blk0 + p * 64 + warp * 8 + (lane >> 2)) * 64 + sub * 16;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (e0 + i < numel) t[i >> 1] |= static_cast<uint32_t>(w[e0 + i]) << (16 * (i & 1));
+    for (int h = 0; h < 2; ++h) {
+      if (full_group) {
+        v[p][h] = __ldg(reinterpret_cast<const uint4*>(w + e0 + 8 * h));
+      } else {
+        uint32_t t[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int64_t e = e0 + 8 * h + i;
+          if (e < numel) t[i >> 1] |= static_cast<uint32_t>(w[e]) << (16 * (i & 1));
+        }
+        v[p][h] = make_uint4(t[0], t[1], t[2], t[3]);
       }
-      v[p] = make_uint4(t[0], t[1], t[2], t[3]);
     }
   }
-  __syncthreads();  // lut ready
+  __syncthreads();  // bucket tables ready
 
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int lb = p * 32 + warp * 4 + (lane >> 3);
-    uint32_t m = max_abs_bits(v[p]);
+  for (int p = 0; p < 4; ++p) {
+    const int lb = p * 64 + warp * 8 + (lane >> 2);
+    uint32_t m = max(max_abs_bits(v[p][0]), max_abs_bits(v[p][1]));
     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
     if (m > 0x7F7Fu && sub == 0 && status) atomicOr(status, QLORA_DEV_NONFINITE);
     const float c = __uint_as_float(m << 16);
     const float rc = __frcp_rn(c);
-    uint32_t out;
+    uint2 out;
     if (rc < __int_as_float(0x7F800000)) {
-      out = codes8(v[p], rc, thr, base);
+      uint64_t rc2;
+      asm("mov.b64 %0, {%1, %1};" : "=l"(rc2) : "f"(rc));
+      out.x = codes8(v[p][0], rc2, thr, base);
+      out.y = codes8(v[p][1], rc2, thr, base);
     } else {
-      out = codes_degenerate(v[p]);
+      out.x = codes_degenerate(v[p][0]);
+      out.y = codes_degenerate(v[p][1]);
     }
     const int64_t b = blk0 + lb;
-    if (b < nblocks) *reinterpret_cast<uint32_t*>(codes + b * 32 + sub * 4) = out;
+    if (b < nblocks) *reinterpret_cast<uint2*>(codes + b * 32 + sub * 8) = out;
     if (sub == 0) cblk[lb] = m << 16;  // c as fp32 bits (0 for padding blocks)
   }
   __syncthreads();
+
+  if (CENTERED) {
+    const int64_t b = blk0 + tid;
+    if (b < nblocks) cbuf[b] = __uint_as_float(cblk[tid]);
+    if (tid == 0) {
+      double acc = 0.0;  // padding blocks add +0
+      for (int i = 0; i < 256; ++i) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(cblk[i])));
+      gsum[blockIdx.x] = acc;
+    }
+    return;
+  }
 
   // Double quantisation of the 256 constants of this group.
   const uint32_t cbits = cblk[tid];
@@ -160,6 +184,52 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const ui
   const float scale = __fdiv_rn(__uint_as_float(amax), 448.0f);
   const float y = scale > 0.0f ? __fdiv_rn(__uint_as_float(cbits), scale) : 0.0f;
   const int64_t b = blk0 + tid;
+  if (b < nblocks) c8[b] = static_cast<uint8_t>(float_to_e4m3_satfinite(y));
+  if (tid == 0) s2[blockIdx.x] = scale;
+}
+
+// ------------------------------------------------ mean-centred constants
+//
+// The tensor mean of the block constants: the group sums added sequentially
+// in fp64, divided by the number of blocks, rounded once to fp32.  One
+// thread: the order of the additions is fixed.  The other lanes stage the
+// group sums through shared memory ahead of the additions.
+__global__ void nf4_mean_kernel(const double* __restrict__ gsum, int64_t ngroups, int64_t nblocks, float* mean) {
+  __shared__ double chunk[1024];
+  grid_dependency_wait();
+  grid_dependents_launch();
+  double total = 0.0;
+  for (int64_t g0 = 0; g0 < ngroups; g0 += 1024) {
+    const int n = static_cast<int>(ngroups - g0 < 1024 ? ngroups - g0 : 1024);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) chunk[i] = gsum[g0 + i];
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int i = 0; i < n; ++i) total = __dadd_rn(total, chunk[i]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *mean = __double2float_rn(__ddiv_rn(total, static_cast<double>(nblocks)));
+}
+
+// Per group of 256 constants: c' = RN32(c - mean) (0 for padding blocks);
+// s2 = RN32(max|c'| / 448); c8 = E4M3(RN32(c' / s2)), 0 when s2 = 0.
+__global__ void __launch_bounds__(256) nf4_encode_centered_kernel(const float* __restrict__ cbuf, int64_t nblocks,
+                                                                  const float* __restrict__ mean,
+                                                                  uint8_t* __restrict__ c8, float* __restrict__ s2) {
+  __shared__ uint32_t wmax[8];
+  grid_dependency_wait();
+  grid_dependents_launch();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + tid;
+  const float cc = b < nblocks ? __fsub_rn(cbuf[b], *mean) : 0.0f;
+  // |c'| as bits: non-negative floats order like unsigned ints
+  uint32_t amax = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(cc) & 0x7FFFFFFFu);
+  if (lane == 0) wmax[warp] = amax;
+  __syncthreads();
+  amax = wmax[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = max(amax, wmax[i]);
+  const float scale = __fdiv_rn(__uint_as_float(amax), 448.0f);
+  const float y = scale > 0.0f ? __fdiv_rn(cc, scale) : 0.0f;
   if (b < nblocks) c8[b] = static_cast<uint8_t>(float_to_e4m3_satfinite(y));
   if (tid == 0) s2[blockIdx.x] = scale;
 }
@@ -182,6 +252,7 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const _
                                                                           const uint8_t* __restrict__ codes,
                                                                           const uint8_t* __restrict__ c8,
                                                                           const float* __restrict__ s2,
+                                                                          const float* __restrict__ mean,
                                                                           int64_t numel, uint16_t* __restrict__ out,
                                                                           Nf4Tables tab) {
   __shared__ __align__(1024) uint8_t stage[kDequantThreads * 128];
@@ -191,7 +262,8 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const _
   const int64_t b = static_cast<int64_t>(blockIdx.x) * kDequantThreads + tid;
   const int64_t nblocks = (numel + 63) / 64, nfull = numel / 64;
   const bool valid = b < nblocks;
-  const float chat = valid ? nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8))) : 0.0f;
+  const Nf4Mean wmean = nf4_load_mean(mean);
+  const float chat = valid ? nf4_block_scale(__ldg(c8 + b), __ldg(s2 + (b >> 8)), wmean) : 0.0f;
   const Nf4Lut lut = nf4_make_lut(tab, chat);
   uint4 c0 = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u), c1 = c0;  // code 7 = +0
   if (valid) {
@@ -225,18 +297,35 @@ __global__ void __launch_bounds__(kDequantThreads) nf4_dequantize_kernel(const _
 cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
                                 int32_t* status, const Nf4Tables& tab, cudaStream_t stream) {
   const int64_t ngroups = (numel + 16383) / 16384;
-  return launch_kernel(nf4_quantize_kernel, dim3(static_cast<unsigned>(ngroups)), dim3(kQuantThreads), 0, stream,
-                       dim3(1, 1, 1), w, numel, codes, c8, s2, status, tab);
+  return launch_kernel(nf4_quantize_kernel<false>, dim3(static_cast<unsigned>(ngroups)), dim3(kQuantThreads), 0,
+                       stream, dim3(1, 1, 1), w, numel, codes, c8, s2, status, tab, static_cast<float*>(nullptr),
+                       static_cast<double*>(nullptr));
 }
 
-cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, int64_t numel,
-                                  uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
+cudaError_t launch_nf4_quantize_centered(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
+                                         float* mean, float* cbuf, double* gsum, int32_t* status,
+                                         const Nf4Tables& tab, cudaStream_t stream) {
+  const int64_t nblocks = (numel + 63) / 64;
+  const int64_t ngroups = (numel + 16383) / 16384;
+  const dim3 one(1, 1, 1);
+  cudaError_t e = launch_kernel(nf4_quantize_kernel<true>, dim3(static_cast<unsigned>(ngroups)), dim3(kQuantThreads),
+                                0, stream, one, w, numel, codes, c8, s2, status, tab, cbuf, gsum);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(nf4_mean_kernel, one, dim3(256), 0, stream, one, static_cast<const double*>(gsum), ngroups,
+                    nblocks, mean);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(nf4_encode_centered_kernel, dim3(static_cast<unsigned>(ngroups)), dim3(256), 0, stream, one,
+                       static_cast<const float*>(cbuf), nblocks, static_cast<const float*>(mean), c8, s2);
+}
+
+cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, const float* mean,
+                                  int64_t numel, uint16_t* out, const CUtensorMap* tm_out, const Nf4Tables& tab,
                                   cudaStream_t stream) {
   const int64_t nblocks = (numel + 63) / 64;
   const int64_t grid = (nblocks + kDequantThreads - 1) / kDequantThreads;
   CUtensorMap none{};
   return launch_kernel(nf4_dequantize_kernel, dim3(static_cast<unsigned>(grid)), dim3(kDequantThreads), 0, stream,
-                       dim3(1, 1, 1), tm_out ? *tm_out : none, tm_out ? 1 : 0, codes, c8, s2, numel, out, tab);
+                       dim3(1, 1, 1), tm_out ? *tm_out : none, tm_out ? 1 : 0, codes, c8, s2, mean, numel, out, tab);
 }
 
 // ------------------------------------------------------- bounded-wait self-test
@@ -258,10 +347,9 @@ __global__ void selftest_timeout_kernel(int32_t* status, uint64_t limit_ns) {
     fence_barrier_init();
   }
   __syncthreads();
-  WaitCtx wc{&abort_flag, status};
-  wc.limit_ns = limit_ns;
+  const WaitCtx wc{&abort_flag, status};
   const int warp = threadIdx.x >> 5;
-  const bool ok = warp == 0 ? mbar_wait_warp(&bar, 0, wc) : mbar_wait_all(&bar, 0, wc);
+  const bool ok = warp == 0 ? mbar_wait_warp(&bar, 0, wc, limit_ns) : mbar_wait_all(&bar, 0, wc, limit_ns);
   if ((threadIdx.x & 31) == 0 && !ok) atomicAdd(status + 1, 1);
 }
 

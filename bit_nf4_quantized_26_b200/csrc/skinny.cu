@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   const WaitCtx wc{abort_flag, a.status};
   grid_dependency_wait();  // inputs of earlier kernels are complete and visible
   grid_dependents_launch();
+  if (MODE == kSkDown && a.zero && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < a.zero_count; i += blockDim.x) a.zero[i] = 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -336,56 +338,6 @@ cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& t
     case kSkDA: return launch_skinny_impl<kSkDA>(tmA, tmB, a, grid_rows, splits, stream);
     default: return cudaErrorInvalidValue;
   }
-}
-
-// ------------------------------------------------------------------ finishers
-
-// Sum of the S split partials of four consecutive elements i..i+3, in split
-// order.  The loads of up to eight partials are issued before the first add
-// so their latencies overlap; the additions stay in the fixed order
-// 0, 1, ..., S-1 for every element.
-__device__ __forceinline__ float4 sum_partials4(const float* __restrict__ P, int S, int64_t n, int64_t i) {
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int z0 = 0; z0 < S; z0 += 8) {
-    float4 v[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      v[k] = (z0 + k < S) ? __ldg(reinterpret_cast<const float4*>(P + (z0 + k) * n + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (z0 + k < S) {
-        acc.x = __fadd_rn(acc.x, v[k].x);
-        acc.y = __fadd_rn(acc.y, v[k].y);
-        acc.z = __fadd_rn(acc.z, v[k].z);
-        acc.w = __fadd_rn(acc.w, v[k].w);
-      }
-    }
-  }
-  return acc;
-}
-
-// One thread per four consecutive outputs (n is a multiple of 4: N % 64 == 0).
-__global__ void finish_out_kernel(const float* __restrict__ P, int S, int64_t n, void* __restrict__ out,
-                                  int out_f32) {
-  const int64_t i = 4 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
-  grid_dependency_wait();
-  grid_dependents_launch();
-  if (i >= n) return;
-  const float4 acc = sum_partials4(P, S, n, i);
-  if (out_f32) {
-    *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + i) = acc;
-  } else {
-    const uint32_t lo = static_cast<uint32_t>(bf16_bits(acc.x)) | (static_cast<uint32_t>(bf16_bits(acc.y)) << 16);
-    const uint32_t hi = static_cast<uint32_t>(bf16_bits(acc.z)) | (static_cast<uint32_t>(bf16_bits(acc.w)) << 16);
-    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + i) = make_uint2(lo, hi);
-  }
-}
-
-cudaError_t launch_finish_out(const float* P, int S, int64_t count, void* out, int out_f32, cudaStream_t stream) {
-  if (count % 4 != 0) return cudaErrorInvalidValue;
-  const int64_t threads = count / 4;
-  return launch_kernel(finish_out_kernel, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, stream,
-                       dim3(1, 1, 1), P, S, count, out, out_f32);
 }
 
 }  // namespace qnf4

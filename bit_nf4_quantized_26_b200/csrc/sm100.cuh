@@ -61,19 +61,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // timeout the waiter records QLORA_DEV_TIMEOUT, raises the CTA's abort flag so
 // the other roles stop waiting too, and returns false.
 struct WaitCtx {
-  volatile int* abort_flag;              // shared memory
-  int32_t* status;                       // global memory, may be null
-  uint64_t limit_ns = kWaitTimeoutNs;    // give up after this long
+  volatile int* abort_flag;  // shared memory
+  int32_t* status;           // global memory, may be null
 };
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+// limit_ns: the kernels use the default; the self-test passes a short one.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > w.limit_ns) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *w.abort_flag = 1;
         if (w.status) atomicOr(w.status, QLORA_DEV_TIMEOUT);
         return false;
@@ -101,16 +102,18 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32
 // Warp-uniform wait: lane 0 polls, the outcome is broadcast, so the whole warp
 // takes the same branch (needed before .sync.aligned tcgen05 ops and before
 // a per-warp elected arrival).
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                               uint64_t limit_ns = kWaitTimeoutNs) {
   uint32_t ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w) ? 1u : 0u;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, limit_ns) ? 1u : 0u;
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
 // Every lane polls (all wake as soon as the phase completes); a vote makes
 // the outcome warp-uniform.
-__device__ __forceinline__ bool mbar_wait_all(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  const bool ok = mbar_wait(bar, parity, w);
+__device__ __forceinline__ bool mbar_wait_all(uint64_t* bar, uint32_t parity, const WaitCtx& w,
+                                              uint64_t limit_ns = kWaitTimeoutNs) {
+  const bool ok = mbar_wait(bar, parity, w, limit_ns);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
@@ -273,6 +276,12 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank)
   return out;
 }
 
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -308,7 +317,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > w.limit_ns) {
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
         *w.abort_flag = 1;
         if (w.status) atomicOr(w.status, QLORA_DEV_TIMEOUT);
         return false;

@@ -1,8 +1,8 @@
 """Double quantisation with mean centring (a variant of the constants'
 encoding, for an error ablation against the plain scheme).
 
-TEST INFRASTRUCTURE ONLY (see the package header).  No CUDA path uses it
-yet; this module fixes what one must compute.
+TEST INFRASTRUCTURE ONLY (see the package header).  This module fixes what
+the library's mean-centred quantiser and dequantisers must compute.
 
 The pages describe double quantisation as "the quantisation constants are
 themselves quantised to FP8 in blocks of 256" ("QLoRA" encyclopedia entry,
@@ -19,7 +19,8 @@ its sign.  Readings taken here:
   c8 = E4M3_RNE_satfinite(RN32(c' / s2)) (0 when s2 = 0);
 * dequantised constant: c_hat = RN32(RN32(e4m3(c8) * s2) + mean).
 
-The 4-bit codes are unchanged (they come from the exact constants).
+The 4-bit codes are unchanged (they come from the exact constants), and the
+dequantised weight is w' = bf16(RN32(q[code] * c_hat)) as in the plain scheme.
 
 Parity status: pinned (constant constants reconstruct exactly; the fixed-
 order mean against an exact rational mean within one fp32 rounding; the
@@ -29,8 +30,8 @@ scheme's error bound recovered when the mean is forced to zero).
 
 import numpy as np
 
-from .nf4 import GROUP, FP8_MAX
-from .numerics import e4m3_decode, e4m3_encode
+from .nf4 import BLOCK, GROUP, FP8_MAX, absmax_constants, codebook, encode_codes, pack_codes, unpack_codes
+from .numerics import e4m3_decode, e4m3_encode, f32_to_bf16_bits
 
 
 def constants_mean(c):
@@ -73,3 +74,25 @@ def dequantized_constants_centered(c8, s2, mean):
     s2 = np.asarray(s2, dtype=np.float32)
     g = np.arange(c8.size) // GROUP
     return ((e4m3_decode(c8) * s2[g]).astype(np.float32) + np.float32(mean)).astype(np.float32)
+
+
+def quantize_centered(w_bits, numel=None):
+    """NF4 quantisation with mean-centred double quantisation of a bf16
+    tensor (flattened row-major): ``(codes_packed, c8, s2, mean)``.  The codes
+    are those of the plain scheme; only the constants' encoding differs."""
+    w_bits = np.asarray(w_bits, dtype=np.uint16).reshape(-1)
+    numel = w_bits.size if numel is None else numel
+    c = absmax_constants(w_bits, numel)
+    codes = encode_codes(w_bits, numel, c)
+    c8, s2, mean = double_quantize_centered(c)
+    return pack_codes(codes), c8, s2, mean
+
+
+def dequantize_centered(codes_packed, c8, s2, mean, numel):
+    """bf16 bit patterns of w' = bf16(RN32(q[code] * c_hat)), c_hat from
+    :func:`dequantized_constants_centered` (two roundings there, two here)."""
+    nblocks = -(-numel // BLOCK)
+    codes = unpack_codes(codes_packed, nblocks * BLOCK).reshape(nblocks, BLOCK)
+    chat = dequantized_constants_centered(c8, s2, mean)
+    vals = (codebook()[codes] * chat[:, None]).astype(np.float32)
+    return f32_to_bf16_bits(vals).reshape(-1)[:numel]

@@ -79,6 +79,11 @@ int main(void) {
         QLORA_ERR_WORKSPACE);
   CHECK(qlora_linear_fwd_noalloc(p, 64, w, p, p, 8, 0.25f, p, QLORA_DTYPE_BF16, p, NULL, NULL) == QLORA_ERR_SHAPE);
   CHECK(qlora_linear_fwd_noalloc(p, 0, w, p, p, 16, 0.25f, p, 7, p, NULL, NULL) == QLORA_ERR_DTYPE);
+  /* Mean-centred double quantisation: argument checks. */
+  CHECK(nf4_centered_workspace_size(0) == 0);
+  CHECK(nf4_quantize_centered(p, 64, p, p, p, NULL, p, 1u << 20, NULL, NULL) == QLORA_ERR_NULL);
+  CHECK(nf4_quantize_centered(p, 64, p, p, p, p, p, 16, NULL, NULL) == QLORA_ERR_WORKSPACE);
+  CHECK(nf4_dequantize_centered(p, p, p, NULL, 64, p, NULL) == QLORA_ERR_NULL);
   /* Bounded-wait self-test: argument checks only (no device here). */
   CHECK(qlora_selftest_timeout(NULL, 5000000, NULL) == QLORA_ERR_NULL);
   CHECK(qlora_selftest_timeout(p, 10, NULL) == QLORA_ERR_SHAPE);

@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 24
+    assert len(names) == 27
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -144,6 +144,21 @@ def test_group_argument_errors():
                                                                                                     4096, 64)
     assert q.qlora_group_bwd_workspace_size(4096, 12288, 4096, 3, 64) > q.qlora_bwd_workspace_size(4096, 12288,
                                                                                                    4096, 64)
+
+
+def test_centred_quantize_argument_errors():
+    lib = q.raw()
+    assert q.nf4_centered_workspace_size(0) == 0
+    assert q.nf4_centered_workspace_size(16384 * 3) == 256 * 3 * 4 + 256
+    assert lib.nf4_quantize_centered(FAKE, 64, FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None, None) == NULL  # mean
+    assert lib.nf4_quantize_centered(FAKE, 64, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 1 << 20, None, None) == ALIGN
+    assert lib.nf4_quantize_centered(FAKE, 64, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None, None) == WS
+    assert lib.nf4_quantize_centered(FAKE, -1, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None, None) == SHAPE
+    assert lib.nf4_quantize_centered(None, 0, None, None, None, None, None, 0, None, None) == OK
+    assert lib.nf4_dequantize_centered(FAKE, FAKE, FAKE, None, 64, FAKE, None) == NULL
+    w = q._NF4Weight(FAKE, FAKE, FAKE, 4096, 4096, FAKE + 8)   # misaligned mean pointer
+    assert q.raw().qlora_linear_fwd(FAKE, 64, w, FAKE, FAKE, 64, 0.25, FAKE, 0, FAKE, FAKE, 1 << 40, None,
+                                    None) == ALIGN
 
 
 def test_bwd_argument_errors():

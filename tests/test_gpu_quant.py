@@ -136,3 +136,55 @@ def test_nonfinite_input_sets_status():
     lib.nf4_quantize(w, status=status)
     torch.cuda.synchronize()
     assert int(status[0].item()) & lib.DEV_NONFINITE
+
+
+def test_nan_input_sets_status_and_other_groups_stay_exact():
+    """A NaN makes its block's codes unspecified (never a stray table access);
+    the other groups of the call are still exact."""
+    lib = _lib()
+    w = synth.normal_bf16((16384 * 4,), 0.02, seed=4)
+    w[16384 * 2 + 100] = float("nan")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    codes, c8, s2 = lib.nf4_quantize(w.cuda(), status=status)
+    torch.cuda.synchronize()
+    assert int(status[0].item()) & lib.DEV_NONFINITE
+    flat = bits(w)
+    for g in (0, 1, 3):
+        p, c, s = nf4.quantize(flat[g * 16384:(g + 1) * 16384])
+        assert np.array_equal(np_u8(codes)[g * 8192:(g + 1) * 8192], p)
+        assert np.array_equal(np_u8(c8)[g * 256:(g + 1) * 256], c)
+
+
+def test_c5_quantize_sweep_all_layers_sampled_groups():
+    """The 65B-shaped sweep: every linear weight of 80 layers (hidden 8192,
+    intermediate 22016; 64.76 G parameters) drawn on the device, quantised,
+    and dropped, keeping only the 33.4 GB of NF4 resident.  Then the weights
+    of the first, the last and three random layers are drawn again from the
+    same seeds and 6 random double-quantisation groups of each matrix (plus
+    its first and last) are checked bit for bit against the oracle."""
+    lib = _lib()
+    kept = []
+    for layer in range(synth.C5_LAYERS):
+        for j, lin in enumerate(synth.c5_layer_linears()):
+            w = synth.weight_bf16(lin.n_out, lin.k_in, seed=650000 + 10 * layer + j, device="cuda")
+            kept.append(lib.nf4_quantize(w.reshape(-1)))
+            del w
+    torch.cuda.synchronize()
+    resident = sum(c.numel() + c8.numel() + 4 * s2.numel() for c, c8, s2 in kept)
+    assert resident == 33407713280
+    rng = np.random.default_rng(80)
+    layers = sorted({0, synth.C5_LAYERS - 1, *rng.integers(1, synth.C5_LAYERS - 1, 3).tolist()})
+    for layer in layers:
+        for j, lin in enumerate(synth.c5_layer_linears()):
+            codes, c8, s2 = kept[layer * 7 + j]
+            w = synth.weight_bf16(lin.n_out, lin.k_in, seed=650000 + 10 * layer + j, device="cuda").reshape(-1)
+            ngroups = s2.numel()
+            picks = sorted({0, ngroups - 1, *rng.integers(0, ngroups, 6).tolist()})
+            for g in picks:
+                seg = bits(w[g * 16384:(g + 1) * 16384])
+                p, c, s = nf4.quantize(seg)
+                assert np.array_equal(np_u8(codes[g * 8192:(g + 1) * 8192]), p), (layer, j, g)
+                assert np.array_equal(np_u8(c8[g * 256:(g + 1) * 256]), c), (layer, j, g)
+                assert s2[g].item() == float(s[0]), (layer, j, g)
+            del w
+    del kept

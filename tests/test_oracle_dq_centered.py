@@ -69,3 +69,41 @@ def test_centring_lowers_the_constant_error_on_normal_weights():
     e_plain = np.sqrt(np.mean(((plain - c) / c) ** 2))
     e_cent = np.sqrt(np.mean(((cent - c) / c) ** 2))
     assert e_cent < e_plain
+
+
+def test_full_centred_quantize_keeps_the_plain_codes():
+    """Centring changes only the constants' encoding: the packed codes equal
+    the plain scheme's, and c8 / s2 / mean are double_quantize_centered of
+    the exact block constants."""
+    w = synth.bf16_bits(synth.weight_bf16(64, 1024, seed=7)).reshape(-1)
+    codes, c8, s2, mean = dqc.quantize_centered(w)
+    pcodes, _, _ = nf4.quantize(w)
+    assert np.array_equal(codes, pcodes)
+    r8, rs2, rmean = dqc.double_quantize_centered(nf4.absmax_constants(w, w.size))
+    assert np.array_equal(c8, r8) and np.array_equal(s2.view(np.uint32), rs2.view(np.uint32)) and mean == rmean
+
+
+def test_centred_dequantize_reduces_to_plain_with_zero_mean():
+    """With the mean forced to 0 the centred encoding is the plain one, and
+    the centred dequantisation (c_hat = RN32(RN32(e4m3 * s2) + 0)) gives the
+    plain dequantised weights bit for bit."""
+    w = synth.bf16_bits(synth.weight_bf16(32, 2048, seed=8)).reshape(-1)
+    pcodes, p8, ps2 = nf4.quantize(w)
+    got = dqc.dequantize_centered(pcodes, p8, ps2, np.float32(0.0), w.size)
+    assert np.array_equal(got, nf4.dequantize(pcodes, p8, ps2, w.size))
+
+
+def test_centred_dequantize_closed_form_per_element():
+    """Elementwise: w'[i] = bf16(RN32(q[code_i] * c_hat[block(i)])) with c_hat
+    = RN32(RN32(e4m3(c8) * s2) + mean), written out with Python floats and the
+    fp32 / bf16 roundings of oracle.numerics, on a few hundred elements."""
+    w = synth.bf16_bits(synth.weight_bf16(4, 256, seed=9, outliers=True)).reshape(-1)
+    codes, c8, s2, mean = dqc.quantize_centered(w)
+    got = dqc.dequantize_centered(codes, c8, s2, mean, w.size)
+    q = nf4.codebook()
+    flat_codes = nf4.unpack_codes(codes, w.size)
+    for i in range(0, w.size, 7):
+        b = i // 64
+        chat = np.float32(np.float32(nm.e4m3_decode(np.array([c8[b]], dtype=np.uint8))[0] * s2[b // 256]) + mean)
+        want = nm.f32_to_bf16_bits(np.array([np.float32(q[flat_codes[i]] * chat)], dtype=np.float32))[0]
+        assert got[i] == want, i
