@@ -2,6 +2,7 @@
 // workspace planning, TMA descriptor creation and kernel launches.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -169,6 +170,16 @@ bool use_tmem_a() {
     return e && e[0] == '1';
   }();
   return enabled;
+}
+
+// A slots of that kernel: QLORA_TMEM_A_SLOTS = 4 (448-token tiles, the
+// default) or 8 (384-token tiles).
+int tmem_a_slots() {
+  static const int v = [] {
+    const char* e = getenv("QLORA_TMEM_A_SLOTS");
+    return (e && atoi(e) == 8) ? 8 : 4;
+  }();
+  return v;
 }
 
 // ------------------------------------------------------------ checks
@@ -758,7 +769,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   if (M > kWideM) {
     const bool pair = use_pair(N) && group_pairs(grp);
     const bool tmem_a = pair && use_tmem_a();
-    const uint32_t tok_box = tmem_a ? 112 : (pair ? 128 : 256);
+    const uint32_t tok_box = tmem_a ? static_cast<uint32_t>(pair_fwd_tokens(tmem_a_slots()) / 4) : (pair ? 128 : 256);
     CUtensorMap wx, wc, wu, wb;
     if (!map_bf16(&wx, X, M, K, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
         !map_bf16(&wu, ucat, M, 2 * ra, 32, tok_box, 64) || !map_bf16(&wb, B, N, r, 32, 128, 64))
@@ -781,7 +792,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
     fa.tab = tables();
     fill_group(grp, &fa);
     ProfScope ps(kKFusedFwd, cs);
-    if (tmem_a) return from_cuda(launch_fused_pair_fwd(wx, wc, wu, wb, fa, cs));
+    if (tmem_a) return from_cuda(launch_fused_pair_fwd(wx, wc, wu, wb, fa, tmem_a_slots(), cs));
     return from_cuda(pair ? launch_fused_pair(false, wx, wc, wu, wb, fa, cs)
                           : launch_fused2x(false, wx, wc, wu, wb, fa, cs));
   }

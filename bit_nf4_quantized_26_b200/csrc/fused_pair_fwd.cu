@@ -17,7 +17,8 @@
 //   cfull[s]  this CTA's packed codes landed (local TMA)
 //   full[s]   leader only: both CTAs' token / LoRA tiles landed (paired TMA)
 //   wfull[s]  leader only: both CTAs' A rows stored in tensor memory (one
-//             release arrival per dequantiser warp after tcgen05.wait::st)
+//             arrival per dequantiser warp after tcgen05.wait::st and the
+//             tcgen05 fence before the thread synchronisation)
 //   empty[s]  both CTAs: the pair's MMAs of the stage finished (multicast
 //             commit); the dequantisers also wait on it before reusing an A slot
 //   accf      both CTAs: the accumulators are final (multicast commit)
@@ -29,15 +30,16 @@ namespace qnf4 {
 
 namespace {
 
+template <int ASLOTS>
 struct PlanPairT {
-  static constexpr int kN = 224;                 // tokens per accumulator (MMA N)
+  static constexpr int kN = (512 - 16 * ASLOTS) / 2;  // tokens per accumulator (MMA N)
   static constexpr uint32_t kBq = (kN / 2) * 64; // one accumulator's token rows in one CTA: 112 x 32 bf16
   static constexpr uint32_t kB = 2 * kBq;        // 14 KB
   static constexpr uint32_t kC = 2048;           // packed codes of a main stage (128 rows x 16 B)
   static constexpr uint32_t kExt = 8192;         // rows of B in an adapter stage (128 x 32 bf16)
   static constexpr uint32_t kStage = 23552;      // kB + kExt rounded up to 1 KB
   static constexpr uint32_t kStages = 8;
-  static constexpr int kASlots = 4;
+  static constexpr int kASlots = ASLOTS;
   static constexpr uint32_t kACol = 2 * kN;      // first tensor-memory column of the A ring
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 512;
@@ -70,18 +72,17 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Arrive with release at cluster scope on a barrier of either CTA of the pair.
-__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 }  // namespace
 
+// The dequantisers publish their rows with a plain remote arrival (release at
+// CTA scope, as for any cross-CTA pair barrier); a cluster-scope release costs
+// a memory barrier per warp and stage and measured 2.3-2.7x slower.
+template <int ASLOTS>
 __global__ void __launch_bounds__(192, 1)
     fused_pair_fwd_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
                           const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
                           const FusedArgs a) {
-  using P = PlanPairT;
+  using P = PlanPairT<ASLOTS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
@@ -183,7 +184,10 @@ __global__ void __launch_bounds__(192, 1)
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait_cluster(&wfull[s], u & 1, wc)) { aborted = true; break; }
+        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) {
+          aborted = true;
+          break;
+        }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint64_t b0 = sdesc_sw64(sb, 16, 512), b1 = sdesc_sw64(sb + P::kBq, 16, 512);
@@ -251,8 +255,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       const uint32_t s = t % P::kStages, u = t / P::kStages;
       if (!mbar_wait_all(&cfull[s], u & 1, wc)) break;
-      // The A slot of stage t was last read by the MMAs of stage t - kASlots.
-      if (t >= P::kASlots) {
+      // The A slot of stage t was last read by the MMAs of stage t - kASlots
+      // (with as many slots as stages, the codes of stage t landing already
+      // imply it: they were loaded after that stage's MMAs finished).
+      if (P::kASlots < static_cast<int>(P::kStages) && t >= P::kASlots) {
         const int tp = t - P::kASlots;
         if (!mbar_wait_all(&empty[tp % P::kStages], (tp / P::kStages) & 1, wc)) break;
       }
@@ -276,7 +282,7 @@ __global__ void __launch_bounds__(192, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote_release(dsmem_addr(&wfull[s], 0));
+      if (lane == 0) mbar_arrive_remote(dsmem_addr(&wfull[s], 0));
     }
 
     grid_dependency_wait();
@@ -328,18 +334,30 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-cudaError_t launch_fused_pair_fwd(const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
-                                  const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream) {
+template <int ASLOTS>
+static cudaError_t launch_pair_fwd_impl(const CUtensorMap& tm_b, const CUtensorMap& tm_codes,
+                                        const CUtensorMap& tm_uc, const CUtensorMap& tm_ext, const FusedArgs& a,
+                                        cudaStream_t stream) {
+  using P = PlanPairT<ASLOTS>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fused_pair_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(PlanPairT::kSmem));
+    cudaError_t e = cudaFuncSetAttribute(fused_pair_fwd_kernel<ASLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(P::kSmem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int tok = 2 * PlanPairT::kN;
-  return launch_kernel(fused_pair_fwd_kernel, dim3(2 * ((a.rows + 255) / 256), (a.M + tok - 1) / tok, 1), dim3(192),
-                       PlanPairT::kSmem, stream, dim3(2, 1, 1), tm_b, tm_codes, tm_uc, tm_ext, a);
+  const int tok = 2 * P::kN;
+  return launch_kernel(fused_pair_fwd_kernel<ASLOTS>, dim3(2 * ((a.rows + 255) / 256), (a.M + tok - 1) / tok, 1),
+                       dim3(192), P::kSmem, stream, dim3(2, 1, 1), tm_b, tm_codes, tm_uc, tm_ext, a);
+}
+
+int pair_fwd_tokens(int slots) { return 512 - 16 * slots; }
+
+cudaError_t launch_fused_pair_fwd(const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
+                                  const CUtensorMap& tm_ext, const FusedArgs& a, int slots,
+                                  cudaStream_t stream) {
+  return slots == 8 ? launch_pair_fwd_impl<8>(tm_b, tm_codes, tm_uc, tm_ext, a, stream)
+                    : launch_pair_fwd_impl<4>(tm_b, tm_codes, tm_uc, tm_ext, a, stream);
 }
 
 }  // namespace qnf4

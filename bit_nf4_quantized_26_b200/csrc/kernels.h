@@ -182,11 +182,14 @@ cudaError_t launch_fused_pair(bool dx, const CUtensorMap& tm_b, const CUtensorMa
                               cudaStream_t stream);
 
 // Large-M forward on CTA pairs with the dequantised tile in tensor memory:
-// 256 W rows x 448 tokens per cluster of two CTAs.  Needs rows % 256 == 0.
-//   tm_b: X [M, K] box {32, 112} SW64; tm_codes: codes [N, K/2] box {16, 128};
-//   tm_uc: Ucat [M, 2r] box {32, 112} SW64; tm_ext: B [N, r] box {32, 128} SW64.
+// 256 W rows x pair_fwd_tokens(slots) tokens per cluster of two CTAs (`slots`
+// A slots of 16 columns: 4 or 8).  Needs rows % 256 == 0.
+//   tm_b: X [M, K] box {32, tokens/4} SW64; tm_codes: codes [N, K/2] box {16, 128};
+//   tm_uc: Ucat [M, 2r] box {32, tokens/4} SW64; tm_ext: B [N, r] box {32, 128} SW64.
+int pair_fwd_tokens(int slots);
 cudaError_t launch_fused_pair_fwd(const CUtensorMap& tm_b, const CUtensorMap& tm_codes, const CUtensorMap& tm_uc,
-                                  const CUtensorMap& tm_ext, const FusedArgs& a, cudaStream_t stream);
+                                  const CUtensorMap& tm_ext, const FusedArgs& a, int slots,
+                                  cudaStream_t stream);
 
 // Skinny LoRA products; the contraction is split over a cluster of `splits`
 // (1..8) CTAs along y and reduced in-cluster.  See skinny.cu for the maps.

@@ -297,35 +297,6 @@ __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t cluster_addr) {
 // the leader's (rank 0) shared memory, rows 128-255 from the peer's, B split
 // the same way along N; each CTA's TMEM holds its 128 rows of D.
 
-// Wait with acquire at cluster scope (arrivals may come from the peer CTA).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 31u) == 0) {
-      if (*w.abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
-        *w.abort_flag = 1;
-        if (w.status) atomicOr(w.status, QLORA_DEV_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
 // Arrive on a barrier given by its shared::cluster address (default
 // semantics, as cluster pipelines do; the data it publishes lives in the
 // arriving CTA's own shared memory and was fenced for the async proxy).
