@@ -921,7 +921,8 @@ def run_case(args):
     """Profiler driver: time one entry point on one shape (no JSON contract).
 
     --case fwd:M:N:K or bwd:M:N:K (r=64, alpha=16), quant:N:K / dequant:N:K (NF4
-    quantisation / dequantisation of an N x K weight), adamw8:n (one 8-bit AdamW
+    quantisation / dequantisation of an N x K weight), cquant:N:K (the same with
+    mean-centred double quantisation), adamw8:n (one 8-bit AdamW
     step over n parameters), or layer:M (the decoder-layer step with M tokens);
     --steps calls after 2 warm-up calls.
     """
@@ -962,6 +963,14 @@ def run_case(args):
         torch.cuda.synchronize()
         print(json.dumps({"case": args.case, "ok": True}))
         return
+    if args.case.startswith("cquant:"):
+        _, N, K = args.case.split(":")
+        w = synth.weight_bf16(int(N), int(K), seed=1, device="cuda")
+        for _ in range(2 + args.steps):
+            lib.nf4_quantize_centered(w.view(-1))
+        torch.cuda.synchronize()
+        print(json.dumps({"case": args.case, "ok": True}))
+        return
     if args.case.startswith("quant:"):
         _, N, K = args.case.split(":")
         w = synth.weight_bf16(int(N), int(K), seed=1, device="cuda")
@@ -998,7 +1007,7 @@ def main():
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (for profiler captures): no e2e, no extras, no CPU baseline")
     ap.add_argument("--case", default=None,
-                    help="profiler driver: fwd:M:N:K, bwd:M:N:K, quant:N:K, dequant:N:K, adamw8:n or layer:M")
+                    help="profiler driver: fwd:M:N:K, bwd:M:N:K, quant:N:K, cquant:N:K, dequant:N:K, adamw8:n or layer:M")
     args = ap.parse_args()
     if args.case:
         run_case(args)
