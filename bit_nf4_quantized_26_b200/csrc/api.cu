@@ -626,7 +626,9 @@ qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float
 size_t nf4_centered_workspace_size(int64_t numel) {
   if (numel <= 0) return 0;
   const int64_t nblocks = cdiv(numel, 64), ngroups = cdiv(numel, 16384);
-  return align256(static_cast<size_t>(nblocks) * 4) + align256(static_cast<size_t>(ngroups) * 8);
+  // fp32 constants, fp64 group sums, two buffers for the pairwise passes
+  return align256(static_cast<size_t>(nblocks) * 4) + align256(static_cast<size_t>(ngroups) * 8) +
+         2 * align256(static_cast<size_t>(cdiv(ngroups, 2048)) * 8);
 }
 
 qlora_status nf4_quantize_centered(const uint16_t* w_bf16, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
@@ -641,10 +643,14 @@ qlora_status nf4_quantize_centered(const uint16_t* w_bf16, int64_t numel, uint8_
   if (!aligned16(ws)) return QLORA_ERR_ALIGN;
   if (qlora_status st = check_device()) return st;
   float* cbuf = static_cast<float*>(ws);
-  double* gsum = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(cdiv(numel, 64)) * 4));
+  uint8_t* wp = static_cast<uint8_t*>(ws) + align256(static_cast<size_t>(cdiv(numel, 64)) * 4);
+  double* gsum = reinterpret_cast<double*>(wp);
+  wp += align256(static_cast<size_t>(cdiv(numel, 16384)) * 8);
+  double* lvl0 = reinterpret_cast<double*>(wp);
+  double* lvl1 = reinterpret_cast<double*>(wp + align256(static_cast<size_t>(cdiv(cdiv(numel, 16384), 2048)) * 8));
   ProfScope ps(kKQuantize, static_cast<cudaStream_t>(stream));
-  return from_cuda(launch_nf4_quantize_centered(w_bf16, numel, codes, c8, s2, mean, cbuf, gsum, d_status, tables(),
-                                                static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_nf4_quantize_centered(w_bf16, numel, codes, c8, s2, mean, cbuf, gsum, lvl0, lvl1, d_status,
+                                                tables(), static_cast<cudaStream_t>(stream)));
 }
 
 qlora_status nf4_dequantize_centered(const uint8_t* codes, const uint8_t* c8, const float* s2, const float* mean,

@@ -144,8 +144,8 @@ cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes
 // Mean-centred constants: codes plus the fp32 constants (cbuf [nblocks]) and
 // fp64 group sums (gsum [ngroups]); then the mean; then the centred FP8 encoding.
 cudaError_t launch_nf4_quantize_centered(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
-                                         float* mean, float* cbuf, double* gsum, int32_t* status,
-                                         const Nf4Tables& tab, cudaStream_t stream);
+                                         float* mean, float* cbuf, double* gsum, double* lvl0, double* lvl1,
+                                         int32_t* status, const Nf4Tables& tab, cudaStream_t stream);
 //   tm_out: out viewed as [numel / 64, 64] bf16, box {64, 32} SW128 (null when numel < 64);
 //   mean: null for the plain scheme.
 cudaError_t launch_nf4_dequantize(const uint8_t* codes, const uint8_t* c8, const float* s2, const float* mean,

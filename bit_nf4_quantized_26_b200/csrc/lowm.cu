@@ -20,22 +20,22 @@
 // shared-memory read conflict-free: the 8 lanes of each quarter warp (two
 // rows g, four blocks t) hit 8 different 16-byte bank groups.
 //
-// Rows of A (the LoRA down-projection, bf16) form ceil(r/32) more row tiles
-// of 32 rows (two warps) whose operands are copied as they are instead of
-// dequantised, so U = X A^T comes out of the same pass at little cost.
+// U = X A^T (fp32) comes from the rank-r kernel launched just before this one
+// (programmatic dependent launch: the main loop below runs beside it).
 //
-// Lane 0 of warp 0 streams each unit's codes (one 128 x 128-byte TMA box; for
-// an A tile four 32 x 64-feature boxes) and its X slice (four 64-feature
-// boxes; rows past M and features past K arrive as zeros) into a shared-memory
-// ring (four stages, three for 32 tokens), two units ahead of the unit being
-// computed.  No warp is
-// set aside for the copies, so every warp has the full register budget.
+// Lane 0 of warp 0 streams each unit's codes (one 128 x 128-byte TMA box) and
+// its X slice (four 64-feature boxes; rows past M and features past K arrive
+// as zeros) into a shared-memory ring (four stages, three for 32 tokens), two
+// units ahead of the unit being computed.  No warp is set aside for the
+// copies, so every warp has the full register budget.
 //
 // The units (row tile major, K chunk minor) are cut into equal contiguous
 // ranges, one per persistent CTA.  A range spans at most two row tiles (the
 // CTA count is at least the tile count); the CTA writes one fp32 partial per
-// tile it touches.  The finisher adds a tile's partials in CTA order (a fixed
-// order: results are deterministic), adds s U B^T in fp32 and rounds once.
+// tile it touches and counts it in on the tile's counter.  The CTA that counts
+// a tile's last partial finishes the tile: it adds the partials in CTA order
+// (a fixed order: results are deterministic), adds s U B^T in fp32 and rounds
+// once.
 #include "kernels.h"
 
 namespace qnf4 {
@@ -129,12 +129,17 @@ __device__ __forceinline__ void tile_ctas(const LowmArgs& a, int tile, int& c0, 
   c1 = cta_of_unit(static_cast<int64_t>(tile + 1) * a.kc - 1, units, a.ctas);
 }
 
+// Row stride of the staged B tile in shared memory: 128 bytes of a row (r <=
+// 64 bf16) plus 16 of padding, so the 16-byte reads of the eight lanes of a
+// quarter warp (eight consecutive rows) fall in different bank groups.
+constexpr int kSbStride = 144;
+
 // Y rows of `tile` = the sum of its partials in CTA order + s U B^T (fp32,
 // one rounding), by the CTA that wrote the tile's last partial.  Thread:
 // row = tid % 128, tokens (tid / 128) * mpad/2 ..; su holds U's columns of the
-// tile's group member for the M tokens.
+// tile's group member for the M tokens, sb the tile's rows of B.
 template <int NT>
-__device__ void finish_tile(const LowmArgs& a, int tile, const float* su) {
+__device__ void finish_tile(const LowmArgs& a, int tile, const float* su, const uint8_t* sb) {
   constexpr int kMpad = 8 * NT;
   constexpr int kHalf = kMpad / 2;
   const int row = threadIdx.x & (kLowmRows - 1);
@@ -147,6 +152,7 @@ __device__ void finish_tile(const LowmArgs& a, int tile, const float* su) {
   float y[kHalf];
 #pragma unroll
   for (int e = 0; e < kHalf; ++e) y[e] = 0.0f;
+#pragma unroll 2
   for (int c = c0; c <= c1; ++c) {
     const int first = static_cast<int>(unit_start(c, units, a.ctas) / a.kc);
     const float* src = a.part + ((static_cast<int64_t>(c) * 2 + (tile == first ? 0 : 1)) * kLowmRows + row) * kMpad + m0;
@@ -162,9 +168,9 @@ __device__ void finish_tile(const LowmArgs& a, int tile, const float* su) {
   float lo[kHalf];
 #pragma unroll
   for (int e = 0; e < kHalf; ++e) lo[e] = 0.0f;
-  const uint4* br = reinterpret_cast<const uint4*>(a.B + static_cast<int64_t>(n) * a.r);
+  const uint8_t* brow = sb + row * kSbStride;
   for (int j8 = 0; j8 < a.r / 8; ++j8) {
-    const uint4 bv = __ldg(br + j8);
+    const uint4 bv = *reinterpret_cast<const uint4*>(brow + j8 * 16);
     const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -332,7 +338,10 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
   // partial in; the CTA that counts the tile's last one finishes the tile.
   __threadfence();  // this thread's partial stores, before the count
   __syncthreads();
-  float* su = reinterpret_cast<float*>(smem);  // the ring is idle now: U of the member, [mpad][64]
+  // The ring is idle now: U of the member, [mpad][64] fp32, then the tile's
+  // rows of B, [128][kSbStride bytes].
+  float* su = reinterpret_cast<float*>(smem);
+  uint8_t* sb = smem + 8 * NT * 64 * 4;
   const int tile_last = static_cast<int>((u_beg + count - 1) / a.kc);
   for (int tl = tile0; tl <= tile_last; ++tl) {
     if (threadIdx.x == 0) {
@@ -344,13 +353,43 @@ __global__ void __launch_bounds__(kLowmThreads, 2)
     }
     __syncthreads();
     if (*last_flag) {
+      // U of the member and the tile's rows of B into shared memory, 16-byte
+      // loads (rows of U and the member's column offset are multiples of 16
+      // floats; rows of B are r <= 64 bf16), all of a thread's in flight
+      // before any is stored.
       const int mem = group_member(a.grp_end, a.groups, tl * kLowmRows);
-      for (int e = threadIdx.x; e < 8 * NT * 64; e += blockDim.x) {
-        const int m = e >> 6, jj = e & 63;
-        su[e] = (m < a.M && jj < a.r) ? __ldcg(a.U + static_cast<int64_t>(m) * a.ra + mem * a.r + jj) : 0.0f;
+      constexpr int kUq = 8 * NT * 16, kBq = kLowmRows * 8;
+      constexpr int kUn = (kUq + kLowmThreads - 1) / kLowmThreads, kBn = kBq / kLowmThreads;
+      float4 uv[kUn];
+      uint4 bq[kBn];
+#pragma unroll
+      for (int q = 0; q < kUn; ++q) {
+        const int e4 = static_cast<int>(threadIdx.x) + q * kLowmThreads;
+        const int m = e4 >> 4, jj = (e4 & 15) * 4;
+        uv[q] = (e4 < kUq && m < a.M && jj < a.r)
+                    ? __ldcg(reinterpret_cast<const float4*>(a.U + static_cast<int64_t>(m) * a.ra + mem * a.r + jj))
+                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+#pragma unroll
+      for (int q = 0; q < kBn; ++q) {
+        const int e8 = static_cast<int>(threadIdx.x) + q * kLowmThreads;
+        const int rw = e8 >> 3, j8 = e8 & 7;
+        const int64_t n = static_cast<int64_t>(tl) * kLowmRows + rw;
+        bq[q] = (n < a.N && j8 < a.r / 8) ? __ldg(reinterpret_cast<const uint4*>(a.B + n * a.r) + j8)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int q = 0; q < kUn; ++q) {
+        const int e4 = static_cast<int>(threadIdx.x) + q * kLowmThreads;
+        if (e4 < kUq) reinterpret_cast<float4*>(su)[e4] = uv[q];
+      }
+#pragma unroll
+      for (int q = 0; q < kBn; ++q) {
+        const int e8 = static_cast<int>(threadIdx.x) + q * kLowmThreads;
+        *reinterpret_cast<uint4*>(sb + (e8 >> 3) * kSbStride + (e8 & 7) * 16) = bq[q];
       }
       __syncthreads();
-      finish_tile<NT>(a, tl, su);
+      finish_tile<NT>(a, tl, su, sb);
     }
     __syncthreads();
   }

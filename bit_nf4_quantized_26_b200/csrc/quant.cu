@@ -88,8 +88,8 @@ __device__ __forceinline__ uint32_t codes_degenerate(uint4 v) {
 }
 
 // CENTERED: instead of the FP8 step, the group's fp32 constants go to cbuf and
-// their fp64 sum (sequential, in block order) to gsum[group]; the mean and the
-// centred encoding follow in two more kernels.
+// their fp64 pairwise sum to gsum[group]; the mean and the centred encoding
+// follow in more kernels.
 template <bool CENTERED>
 __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const uint16_t* __restrict__ w,
                                                                          int64_t numel, uint8_t* __restrict__ codes,
@@ -165,10 +165,19 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const ui
   if (CENTERED) {
     const int64_t b = blk0 + tid;
     if (b < nblocks) cbuf[b] = __uint_as_float(cblk[tid]);
+    // Pairwise sum of the group's 256 constants (padding blocks are +0):
+    // neighbours by xor-shuffles within each warp (IEEE addition commutes, so
+    // lane l and lane l ^ k form the same sum), then the 8 warp sums.
+    double v = static_cast<double>(__uint_as_float(cblk[tid]));
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, k));
+    __shared__ double wsum[kQuantThreads / 32];
+    if (lane == 0) wsum[warp] = v;
+    __syncthreads();
     if (tid == 0) {
-      double acc = 0.0;  // padding blocks add +0
-      for (int i = 0; i < 256; ++i) acc = __dadd_rn(acc, static_cast<double>(__uint_as_float(cblk[i])));
-      gsum[blockIdx.x] = acc;
+      const double q0 = __dadd_rn(__dadd_rn(wsum[0], wsum[1]), __dadd_rn(wsum[2], wsum[3]));
+      const double q1 = __dadd_rn(__dadd_rn(wsum[4], wsum[5]), __dadd_rn(wsum[6], wsum[7]));
+      gsum[blockIdx.x] = __dadd_rn(q0, q1);
     }
     return;
   }
@@ -190,24 +199,39 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const ui
 
 // ------------------------------------------------ mean-centred constants
 //
-// The tensor mean of the block constants: the group sums added sequentially
-// in fp64, divided by the number of blocks, rounded once to fp32.  One
-// thread: the order of the additions is fixed.  The other lanes stage the
-// group sums through shared memory ahead of the additions.
-__global__ void nf4_mean_kernel(const double* __restrict__ gsum, int64_t ngroups, int64_t nblocks, float* mean) {
-  __shared__ double chunk[1024];
+// The tensor mean of the block constants: their fp64 pairwise sum (zero-padded
+// to a power of two, neighbours added level by level), divided by the number
+// of blocks in fp64 and rounded once to fp32.  The group sums are the tree's
+// nodes 256 constants up; each CTA of this kernel turns an aligned chunk of
+// 2048 of the values below into their pairwise sum (values past `len` are
+// +0, the padding), so repeated passes over 2048x fewer values reach the
+// root, and the pass that runs as a single CTA writes the mean.
+constexpr int kSumThreads = 1024;
+
+__global__ void __launch_bounds__(kSumThreads) nf4_pairwise_kernel(const double* __restrict__ in, int64_t len,
+                                                                   double* __restrict__ out, int64_t nblocks,
+                                                                   float* mean) {
+  __shared__ double wsum[32];
   grid_dependency_wait();
   grid_dependents_launch();
-  double total = 0.0;
-  for (int64_t g0 = 0; g0 < ngroups; g0 += 1024) {
-    const int n = static_cast<int>(ngroups - g0 < 1024 ? ngroups - g0 : 1024);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) chunk[i] = gsum[g0 + i];
-    __syncthreads();
-    if (threadIdx.x == 0)
-      for (int i = 0; i < n; ++i) total = __dadd_rn(total, chunk[i]);
-    __syncthreads();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * (2 * kSumThreads) + 2 * tid;
+  const double x0 = i0 < len ? in[i0] : 0.0;
+  const double x1 = i0 + 1 < len ? in[i0 + 1] : 0.0;
+  double v = __dadd_rn(x0, x1);
+#pragma unroll
+  for (int k = 1; k < 32; k <<= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, k));
+  if (lane == 0) wsum[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = wsum[lane];
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, k));
+    if (lane == 0) {
+      if (gridDim.x == 1) *mean = __double2float_rn(__ddiv_rn(v, static_cast<double>(nblocks)));
+      else out[blockIdx.x] = v;
+    }
   }
-  if (threadIdx.x == 0) *mean = __double2float_rn(__ddiv_rn(total, static_cast<double>(nblocks)));
 }
 
 // Per group of 256 constants: c' = RN32(c - mean) (0 for padding blocks);
@@ -303,16 +327,26 @@ cudaError_t launch_nf4_quantize(const uint16_t* w, int64_t numel, uint8_t* codes
 }
 
 cudaError_t launch_nf4_quantize_centered(const uint16_t* w, int64_t numel, uint8_t* codes, uint8_t* c8, float* s2,
-                                         float* mean, float* cbuf, double* gsum, int32_t* status,
-                                         const Nf4Tables& tab, cudaStream_t stream) {
+                                         float* mean, float* cbuf, double* gsum, double* lvl0, double* lvl1,
+                                         int32_t* status, const Nf4Tables& tab, cudaStream_t stream) {
   const int64_t nblocks = (numel + 63) / 64;
   const int64_t ngroups = (numel + 16383) / 16384;
   const dim3 one(1, 1, 1);
   cudaError_t e = launch_kernel(nf4_quantize_kernel<true>, dim3(static_cast<unsigned>(ngroups)), dim3(kQuantThreads),
                                 0, stream, one, w, numel, codes, c8, s2, status, tab, cbuf, gsum);
   if (e != cudaSuccess) return e;
-  e = launch_kernel(nf4_mean_kernel, one, dim3(256), 0, stream, one, static_cast<const double*>(gsum), ngroups,
-                    nblocks, mean);
+  // Pairwise passes: gsum -> lvl0 -> lvl1 -> lvl0 ... until one CTA is left.
+  const double* in = gsum;
+  int64_t len = ngroups;
+  for (int pass = 0;; ++pass) {
+    const int64_t ctas = (len + 2 * kSumThreads - 1) / (2 * kSumThreads);
+    double* out = (pass & 1) ? lvl1 : lvl0;
+    e = launch_kernel(nf4_pairwise_kernel, dim3(static_cast<unsigned>(ctas)), dim3(kSumThreads), 0, stream, one, in,
+                      len, out, nblocks, mean);
+    if (e != cudaSuccess || ctas == 1) break;
+    in = out;
+    len = ctas;
+  }
   if (e != cudaSuccess) return e;
   return launch_kernel(nf4_encode_centered_kernel, dim3(static_cast<unsigned>(ngroups)), dim3(256), 0, stream, one,
                        static_cast<const float*>(cbuf), nblocks, static_cast<const float*>(mean), c8, s2);

@@ -141,16 +141,18 @@ QLORA_API qlora_status nf4_dequantize(const uint8_t* codes, const uint8_t* c8, c
  * sign bit on them and cuts the constants' error (about 2.8% -> 0.4% RMS on
  * N(0, 0.02) weights):
  *
- *   mean = fp32(S / nblocks), S = fp64 sum of the block constants c taken
- *          sequentially within each group of 256, then over the group sums;
+ *   mean = fp32(S / nblocks), S = fp64 pairwise sum of the block constants
+ *          c (zero-padded to a power of two, neighbouring pairs added level
+ *          by level until one value is left);
  *   per group: c' = RN32(c - mean); s2 = RN32(max|c'| / 448);
  *          c8 = E4M3 round-to-nearest-even, saturating (RN32(c' / s2));
  *   dequantised constant: c_hat = RN32(RN32(e4m3(c8) * s2) + mean).
  *
  * nf4_quantize_centered writes codes, c8, s2 as nf4_quantize does plus the
- * fp32 `mean` (device float[1]); it runs three kernels (codes and constants;
- * the mean; the centred FP8 encoding) and needs a device workspace of
- * nf4_centered_workspace_size(numel) bytes (4 per block + 8 per group).
+ * fp32 `mean` (device float[1]); it runs the codes-and-constants kernel,
+ * one or more pairwise-sum passes (one per factor of 2048 groups) and the
+ * centred FP8 encoding, and needs a device workspace of
+ * nf4_centered_workspace_size(numel) bytes (about 4 per block + 8 per group).
  * nf4_dequantize_centered is nf4_dequantize with c_hat as above.  Pass the
  * mean in nf4_weight.mean to run the GEMMs on such a weight.  Bit-exact with
  * the CPU oracle.  Other conventions as for nf4_quantize / nf4_dequantize.

@@ -12,9 +12,10 @@ first, because they are all positive and a symmetric FP8 grid would waste
 its sign.  Readings taken here:
 
 * one mean per tensor: mean = fp32(S / n) for the n block constants c_i,
-  where S is summed in fp64 in a fixed order — sequentially within each group
-  of 256 constants, then sequentially over the group sums — so a parallel
-  implementation can reproduce it exactly;
+  where S is their pairwise sum in fp64: the constants, padded with zeros to
+  a power of two, are added in neighbouring pairs, level by level, until one
+  value is left.  The order is fixed, so a parallel implementation reproduces
+  it exactly, and its rounding error grows with log2(n), not n;
 * per group: c' = RN32(c - mean); s2 = RN32(max|c'| / 448);
   c8 = E4M3_RNE_satfinite(RN32(c' / s2)) (0 when s2 = 0);
 * dequantised constant: c_hat = RN32(RN32(e4m3(c8) * s2) + mean).
@@ -22,8 +23,10 @@ its sign.  Readings taken here:
 The 4-bit codes are unchanged (they come from the exact constants), and the
 dequantised weight is w' = bf16(RN32(q[code] * c_hat)) as in the plain scheme.
 
-Parity status: pinned (constant constants reconstruct exactly; the fixed-
-order mean against an exact rational mean within one fp32 rounding; the
+Parity status: pinned (constant constants reconstruct exactly; the pairwise
+sum's tree shape on inputs where other orders round differently, and its
+textbook error bound; the mean against an exact rational mean within one
+fp32 rounding; the
 reconstruction error within the E4M3 half-step bound per group; the plain
 scheme's error bound recovered when the mean is forced to zero).
 """
@@ -34,17 +37,26 @@ from .nf4 import BLOCK, GROUP, FP8_MAX, absmax_constants, codebook, encode_codes
 from .numerics import e4m3_decode, e4m3_encode, f32_to_bf16_bits
 
 
+def pairwise_sum(x):
+    """fp64 pairwise sum: zero-pad to a power of two, then replace the array
+    by the sums of its neighbouring pairs (x[0] + x[1], x[2] + x[3], ...)
+    until one value is left."""
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    p = 1
+    while p < x.size:
+        p *= 2
+    level = np.zeros(p, dtype=np.float64)
+    level[: x.size] = x
+    while level.size > 1:
+        level = level[0::2] + level[1::2]
+    return level[0]
+
+
 def constants_mean(c):
-    """fp32 mean of the block constants, summed in fp64 in the fixed order
-    (sequential within groups of 256, then sequential over the groups)."""
-    c = np.asarray(c, dtype=np.float32).astype(np.float64)
-    n = c.size
-    ng = -(-n // GROUP)
-    pad = np.zeros(ng * GROUP, dtype=np.float64)
-    pad[:n] = c
-    group_sums = np.cumsum(pad.reshape(ng, GROUP), axis=1)[:, -1]   # sequential within a group
-    total = np.cumsum(group_sums)[-1]                                # sequential over groups
-    return np.float32(total / n)
+    """fp32 mean of the block constants: their fp64 pairwise sum divided by
+    their count in fp64, rounded once to fp32."""
+    c = np.asarray(c, dtype=np.float32)
+    return np.float32(pairwise_sum(c.astype(np.float64)) / np.float64(c.size))
 
 
 def double_quantize_centered(c, mean=None):

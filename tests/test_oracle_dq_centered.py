@@ -25,8 +25,37 @@ def test_constant_constants_reconstruct_exactly():
     assert np.array_equal(dqc.dequantized_constants_centered(c8, s2, mean), c)
 
 
+def test_pairwise_sum_tree_shape():
+    """Inputs on which the summation orders round differently fix the tree:
+    neighbours first, then the pair sums, zero padding on the right.
+    [1, 0, u, u] with u = 2^-53 (half an fp64 ulp of 1): the pairs give
+    1 and 2u, and 1 + 2u is exact, while a running sum loses each u to the
+    tie rule.  [1, u, u]: the pairs are (1 + u) -> 1 and (u + 0), and 1 + u
+    ties to 1 again, while adding the last two first would keep 2u."""
+    u = 2.0 ** -53
+    assert dqc.pairwise_sum([1.0, 0.0, u, u]) == 1.0 + 2 * u
+    assert dqc.pairwise_sum([1.0, u, u]) == 1.0
+    assert dqc.pairwise_sum([u, u, 1.0]) == 1.0 + 2 * u
+    # eight leaves: ((1 + 0) + (u + u)) + ((u + u) + (u + u)) = 1 + 2u + 4u
+    assert dqc.pairwise_sum([1.0, 0.0] + [u] * 6) == 1.0 + 6 * u
+    assert dqc.pairwise_sum([]) == 0.0 and dqc.pairwise_sum([3.5]) == 3.5
+
+
+def test_pairwise_sum_error_bound():
+    """Textbook bound for pairwise summation of n values:
+    |S - sum| <= ceil(log2 n) * 2^-53 * sum|x| (to first order), against the
+    exact sum (math.fsum), on sizes that are not powers of two."""
+    import math
+    rng = np.random.default_rng(9)
+    for n in (3, 1000, 4097, 100003):
+        x = rng.standard_normal(n) * rng.uniform(0.5, 2.0, n) * 10.0 ** rng.integers(-3, 4, n)
+        exact = math.fsum(x)
+        bound = math.ceil(math.log2(n)) * 2.0 ** -53 * float(np.sum(np.abs(x))) * 1.001
+        assert abs(dqc.pairwise_sum(x) - exact) <= bound, n
+
+
 def test_mean_is_the_exact_mean_within_one_rounding():
-    """The fixed-order fp64 sum of a few thousand fp32 constants is exact
+    """The pairwise fp64 sum of a few thousand fp32 constants is exact
     enough that the fp32 mean is the exact rational mean rounded once (or
     its neighbour when the exact mean lies within fp64 noise of a tie)."""
     c = _constants(64, 4096, 3)
