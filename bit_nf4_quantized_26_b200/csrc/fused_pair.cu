@@ -40,8 +40,14 @@ struct PlanPair {
 
 }  // namespace
 
+// Warp 0: copies; warp 1: MMAs (leader CTA); warps 2..9: two groups of four
+// dequantiser warps taking alternate stages (two independent instruction
+// streams per SM sub-partition: one warp per stage is latency-bound), which
+// also split the epilogue's columns between them.
+constexpr int kPairThreads = 320;
+
 template <bool DX>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     fused_pair_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
                       const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
                       const FusedArgs a) {
@@ -155,43 +161,51 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA (leader)
-    if (lane == 0 && rank == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptors); the
+    // elected lane issues the MMAs and the commits.
+    if (rank == 0) {
       const uint32_t idesc = idesc_bf16_f32(256, 256, DX ? 1 : 0, 0);
       const uint32_t a_step = DX ? (2048u >> 4) : (32u >> 4);
       bool aborted = false;
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) { aborted = true; break; }
+        if (!mbar_wait_all(&full[s], u & 1, wc)) { aborted = true; break; }
+        if (t < nmain && !mbar_wait_all(&wfull[s], u & 1, wc)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint32_t sa = sb + P::kB;
         const uint64_t b0 = sdesc_sw64(sb, 16, 512), b1 = sdesc_sw64(sb + P::kBq, 16, 512);
         const uint64_t ad = DX ? sdesc_sw128(sa, 4096, 1024) : sdesc_sw64(sa, 16, 512);
-        if (t < nmain) {
+        if (elect_one()) {
+          if (t < nmain) {
 #pragma unroll
-          for (uint32_t kk = 0; kk < 2; ++kk) {
-            const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
-            umma_bf16_pair(tmem_d, ad + kk * a_step, b0 + kk * 2, idesc, acc);
-            umma_bf16_pair(tmem_d + 256, ad + kk * a_step, b1 + kk * 2, idesc, acc);
-          }
-        } else {
+            for (uint32_t kk = 0; kk < 2; ++kk) {
+              const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
+              umma_bf16_pair(tmem_d, ad + kk * a_step, b0 + kk * 2, idesc, acc);
+              umma_bf16_pair(tmem_d + 256, ad + kk * a_step, b1 + kk * 2, idesc, acc);
+            }
+          } else {
 #pragma unroll
-          for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
-            umma_bf16_pair(tmem_d, ad, b0 + part * 2, idesc, 1u);
-            umma_bf16_pair(tmem_d + 256, ad, b1 + part * 2, idesc, 1u);
+            for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
+              umma_bf16_pair(tmem_d, ad, b0 + part * 2, idesc, 1u);
+              umma_bf16_pair(tmem_d + 256, ad, b1 + part * 2, idesc, 1u);
+            }
           }
+          umma_commit_pair(&empty[s], 0x3);
         }
-        umma_commit_pair(&empty[s], 0x3);
+        __syncwarp();
       }
-      umma_commit_pair(accf, 0x3);
-      if (aborted) mbar_drain(accf, 0, a.status);
+      if (elect_one()) {
+        umma_commit_pair(accf, 0x3);
+        if (aborted) mbar_drain(accf, 0, a.status);
+      }
     }
     __syncwarp();
     grid_dependency_wait();
     grid_dependents_launch();
   } else {
-    const int dt = threadIdx.x - 64;  // 0..127
+    const int dt = (threadIdx.x - 64) & 127;  // 0..127 within the group
+    const int grp = (threadIdx.x - 64) >> 7;  // stages t with t % 2 == grp
     const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
     const int64_t kbpr = a.k_in / 64;
     if (!DX) {
@@ -215,18 +229,17 @@ __global__ void __launch_bounds__(192, 1)
       };
 #pragma unroll
       for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
-      Nf4Lut lut{};
-      for (int t = 0; t < nmain; ++t) {
-        if ((t & 1) == 0) {
-          const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
+      // Stage t covers half of block t / 2: each group builds that block's
+      // table itself.
+      for (int t = grp; t < nmain; t += 2) {
+        const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
 #pragma unroll
-          for (int i = 0; i + 1 < kPD; ++i) {
-            pc[i] = pc[i + 1];
-            ps[i] = ps[i + 1];
-          }
-          fetch(t / 2 + kPD, pc[kPD - 1], ps[kPD - 1]);
-          lut = nf4_make_lut(a.tab, chat);
+        for (int i = 0; i + 1 < kPD; ++i) {
+          pc[i] = pc[i + 1];
+          ps[i] = ps[i + 1];
         }
+        fetch(t / 2 + kPD, pc[kPD - 1], ps[kPD - 1]);
+        const Nf4Lut lut = nf4_make_lut(a.tab, chat);
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (!mbar_wait_all(&cfull[s], u & 1, wc)) break;
         uint8_t* st = smem + s * P::kStage;
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(192, 1)
       const int nl = p & 31, bs = p >> 5;
       const int kb = row0 / 64 + bs;
       const bool kok = kb < kbpr;
-      constexpr int kPD = 6;
+      constexpr int kPD = 4;  // stages of prefetch (this group's: every other stage)
       uint32_t pc[kPD];
       float ps[kPD];
       auto fetch = [&](int t, uint32_t& c, float& sv) {
@@ -267,8 +280,8 @@ __global__ void __launch_bounds__(192, 1)
         }
       };
 #pragma unroll
-      for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
-      for (int t = 0; t < nmain; ++t) {
+      for (int i = 0; i < kPD; ++i) fetch(grp + 2 * i, pc[i], ps[i]);
+      for (int t = grp; t < nmain; t += 2) {
         const uint32_t c8b = pc[0];
         const float s2v = ps[0];
 #pragma unroll
@@ -276,7 +289,7 @@ __global__ void __launch_bounds__(192, 1)
           pc[i] = pc[i + 1];
           ps[i] = ps[i + 1];
         }
-        fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
+        fetch(t + 2 * kPD, pc[kPD - 1], ps[kPD - 1]);
         const bool valid = kok && (t * 32 + nl) < a.n_out;
         const float chat = valid ? nf4_block_scale(c8b, s2v, wmean) : 0.0f;
         const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes
@@ -304,12 +317,14 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ epilogue
     if (mbar_wait_warp(accf, 0, wc)) {
       tc_fence_after();
+      // Warp w reads TMEM lanes 32 (w % 4) ..; the two groups take half of
+      // the 16 column blocks each.
       const int q = warp & 3;
       const int orow = row0 + q * 32 + lane;
       const bool rok = orow < a.rows;
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int cb = 0; cb < 16; ++cb) {
+      for (int cb = 8 * grp; cb < 8 * grp + 8; ++cb) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tq + cb * 32, v);
         tmem_ld_wait();
@@ -356,7 +371,7 @@ static cudaError_t launch_pair_impl(const CUtensorMap& m0, const CUtensorMap& m1
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_kernel(fused_pair_kernel<DX>, dim3(2 * ((a.rows + 255) / 256), (a.M + 511) / 512, 1), dim3(192),
+  return launch_kernel(fused_pair_kernel<DX>, dim3(2 * ((a.rows + 255) / 256), (a.M + 511) / 512, 1), dim3(kPairThreads),
                        PlanPair::kSmem, stream, dim3(2, 1, 1), m0, m1, m2, m3, a);
 }
 

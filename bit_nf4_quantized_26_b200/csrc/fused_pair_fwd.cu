@@ -8,10 +8,12 @@
 // the bf16 tile straight into tensor memory (tcgen05.st) and the MMA takes its
 // A operand from there.  The weight tile then never passes through shared
 // memory: shared memory carries only the token tiles (TMA in, MMA out) and
-// the packed codes, about half the bytes per stage of the shared-memory
-// design, whose stage period was set by that traffic beside the MMAs.  Tensor
-// memory holds two 128 x 224 fp32 accumulators (448 tokens per pair) and a
-// ring of four 16-column A slots (one 32-deep stage each).
+// the packed codes, so a stage is 16 KB instead of 26 and the ring holds 12
+// stages instead of 8 (the adapter stages' rows of B have buffers of their
+// own).  The main loop is bound by the latency of the copies the ring must
+// hide, so its depth in time is what counts.  Tensor memory holds two
+// 128 x 224 fp32 accumulators (448 tokens per pair) and a ring of four
+// 16-column A slots (one 32-deep stage each).
 //
 // Barriers (all bounded waits):
 //   cfull[s]  this CTA's packed codes landed (local TMA)
@@ -33,19 +35,24 @@ namespace {
 template <int ASLOTS>
 struct PlanPairT {
   static constexpr int kN = (512 - 16 * ASLOTS) / 2;  // tokens per accumulator (MMA N)
-  static constexpr uint32_t kBq = (kN / 2) * 64; // one accumulator's token rows in one CTA: 112 x 32 bf16
-  static constexpr uint32_t kB = 2 * kBq;        // 14 KB
+  static constexpr uint32_t kBq = (kN / 2) * 64; // one accumulator's token rows in one CTA: kN/2 x 32 bf16
+  static constexpr uint32_t kB = 2 * kBq;
   static constexpr uint32_t kC = 2048;           // packed codes of a main stage (128 rows x 16 B)
+  static constexpr uint32_t kStage = (kB + kC + 1023) / 1024 * 1024;
   static constexpr uint32_t kExt = 8192;         // rows of B in an adapter stage (128 x 32 bf16)
-  static constexpr uint32_t kStage = 23552;      // kB + kExt rounded up to 1 KB
-  static constexpr uint32_t kStages = 8;
+  static constexpr uint32_t kExtBufs = 4;        // one per adapter stage: r / 16 <= 4
   static constexpr int kASlots = ASLOTS;
   static constexpr uint32_t kACol = 2 * kN;      // first tensor-memory column of the A ring
-  static constexpr uint32_t kBarOff = kStages * kStage;
+  // As many stages as shared memory holds beside the adapter buffers: the
+  // ring's depth in time is what hides the copies' latency.
+  static constexpr uint32_t kStages = (232448u - 1024u - 512u - kExtBufs * kExt) / kStage;
+  static constexpr uint32_t kExtOff = kStages * kStage;
+  static constexpr uint32_t kBarOff = kExtOff + kExtBufs * kExt;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 512;
-  static_assert(kStage % 1024 == 0 && kStage >= kB + kExt, "stage layout");
+  static_assert(kStage % 1024 == 0 && kStage >= kB + kC, "stage layout");
   static_assert(kBq % 512 == 0, "64-byte swizzle atoms");
   static_assert(kACol + 16 * kASlots <= 512, "tensor memory");
+  static_assert(kStages >= 8 && kStages <= 16, "ring depth");
   static_assert(kSmem <= 232448u, "too much shared memory");
 };
 
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(192, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (P::kB + P::kExt));
           tma_load_2d_pair(st, &tm_uc, full0, uc0 + 32 * e, mt);
           tma_load_2d_pair(st + P::kBq, &tm_uc, full0, uc0 + 32 * e, mt + P::kN);
-          tma_load_2d_pair(st + P::kB, &tm_ext, full0, 16 * e, row0);  // B_lora [128 n x 32 j]
+          tma_load_2d_pair(smem + P::kExtOff + e * P::kExt, &tm_ext, full0, 16 * e, row0);  // B_lora [128 n x 32 j]
         }
         issued = t + 1;
       }
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
             umma_bf16_pair_ta(tmem_d + P::kN, at + kk * 8, b1 + kk * 2, idesc, acc);
           }
         } else {
-          const uint64_t ad = sdesc_sw64(sb + P::kB, 16, 512);
+          const uint64_t ad = sdesc_sw64(smem_u32(smem + P::kExtOff + (t - nmain) * P::kExt), 16, 512);
 #pragma unroll
           for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
             umma_bf16_pair(tmem_d, ad, b0 + part * 2, idesc, 1u);
@@ -339,6 +346,7 @@ static cudaError_t launch_pair_fwd_impl(const CUtensorMap& tm_b, const CUtensorM
                                         const CUtensorMap& tm_uc, const CUtensorMap& tm_ext, const FusedArgs& a,
                                         cudaStream_t stream) {
   using P = PlanPairT<ASLOTS>;
+  if (a.r / 16 > static_cast<int>(P::kExtBufs)) return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(fused_pair_fwd_kernel<ASLOTS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
