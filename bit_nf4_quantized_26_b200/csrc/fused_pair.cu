@@ -14,8 +14,9 @@
 // Barriers (all bounded waits):
 //   cfull[s]  this CTA's packed codes landed (local TMA)
 //   full[s]   leader only: both CTAs' token / LoRA tiles landed (paired TMA)
-//   wfull[s]  leader only: both CTAs' dequantised W tiles written (one arrival
-//             per dequantiser warp after each lane fenced its writes)
+//             and both CTAs' dequantised W tiles are written (one arrival per
+//             dequantiser warp of the stage's group, after each lane fenced
+//             its writes): one barrier, so the MMA warp checks one per stage
 //   empty[s]  both CTAs: the pair's MMAs of the stage finished (multicast commit)
 //   accf      both CTAs: the accumulators are final (multicast commit)
 // No TMA multicast is used.
@@ -56,8 +57,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
   uint64_t* cfull = full + P::kStages;
-  uint64_t* wfull = cfull + P::kStages;
-  uint64_t* empty = wfull + P::kStages;
+  uint64_t* empty = cfull + P::kStages;
   uint64_t* accf = empty + P::kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -73,9 +73,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 8);  // the producer's expect-tx arrival + 4 dequantiser warps per CTA
       mbar_init(&cfull[s], 1);
-      mbar_init(&wfull[s], 8);  // one elected arrival per dequantiser warp, 4 per CTA
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -149,9 +148,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       // Leave nothing in flight into this CTA's shared memory: codes land on the
       // local barrier; the leader also waits for the pair's tiles.
+      // The full barriers also count the dequantisers' arrivals, which may
+      // never come after an abort, so the drain then takes a short limit (the
+      // copies themselves land in microseconds).
+      const uint64_t lim = *abort_flag ? 1000000ull : kWaitTimeoutNs;
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t) {
-        if (t < nmain) mbar_drain(&cfull[t % P::kStages], (t / P::kStages) & 1, a.status);
-        if (rank == 0) mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
+        if (t < nmain) mbar_drain(&cfull[t % P::kStages], (t / P::kStages) & 1, a.status, lim);
+        if (rank == 0) mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status, lim);
       }
     }
     __syncwarp();  // the other lanes pass the wait only after lane 0 is through its loop
@@ -170,7 +173,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (!mbar_wait_all(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait_all(&wfull[s], u & 1, wc)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint32_t sa = sb + P::kB;
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         fence_proxy_async_smem();  // this lane's tile writes -> async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(dsmem_addr(&wfull[s], 0));
+        if (lane == 0) mbar_arrive_remote(dsmem_addr(&full[s], 0));
       }
     } else {
       // -------------------------------------------------- dX dequant
@@ -307,8 +309,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         fence_proxy_async_smem();  // this lane's tile writes -> async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(dsmem_addr(&wfull[s], 0));
+        if (lane == 0) mbar_arrive_remote(dsmem_addr(&full[s], 0));
       }
+    }
+    // Adapter stages: nothing to dequantise, but the stage's group still
+    // arrives on full[s].  It first waits until the slot's previous stage
+    // (t - kStages, a main stage of this group) is retired, so the arrival
+    // falls in the stage's own phase.
+    for (int t = nmain + ((grp - nmain) & 1); t < T; t += 2) {
+      const uint32_t s = t % P::kStages;
+      if (t >= static_cast<int>(P::kStages) && !mbar_wait_all(&empty[s], ((t / P::kStages) - 1) & 1, wc)) break;
+      if (lane == 0) mbar_arrive_remote(dsmem_addr(&full[s], 0));
     }
 
     grid_dependency_wait();

@@ -45,6 +45,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Non-blocking check of the same condition (the fast path of every wait:
+// in a pipeline that keeps up, the phase has completed already).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -68,7 +82,7 @@ struct WaitCtx {
 // limit_ns: the kernels use the default; the self-test passes a short one.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w,
                                           uint64_t limit_ns = kWaitTimeoutNs) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test(bar, parity) || mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -88,10 +102,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 // abort flag.  A drain that runs out records QLORA_DEV_TIMEOUT and returns
 // false; the state of the memory those operations write is then unknown, but
 // the CTA still releases its TMEM, which it must do before it exits.
-__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32_t* status) {
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32_t* status,
+                                           uint64_t limit_ns = kWaitTimeoutNs) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       if (status) atomicOr(status, QLORA_DEV_TIMEOUT);
       return false;
     }
