@@ -151,34 +151,41 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptors); the
+    // elected lane issues the MMAs and the commits.
+    {
       const uint32_t idesc = idesc_bf16_f32(128, BN, DX ? 1 : 0, 0);
       const uint32_t a_step = DX ? (2048u >> 4) : (32u >> 4);  // one K=16 step, descriptor units
       bool aborted = false;
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) { aborted = true; break; }
+        if (!mbar_wait_all(&full[s], u & 1, wc)) { aborted = true; break; }
+        if (t < nmain && !mbar_wait_all(&wfull[s], u & 1, wc)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint32_t sa = sb + P::kB;
         const uint64_t bdesc = sdesc_sw128(sb, 16, 1024);
         const uint64_t adesc = DX ? sdesc_sw128(sa, 8192, 1024) : sdesc_sw128(sa, 16, 1024);
-        if (t < nmain) {
+        if (elect_one()) {
+          if (t < nmain) {
 #pragma unroll
-          for (uint32_t kk = 0; kk < 4; ++kk)
-            umma_bf16(tmem_d, adesc + kk * a_step, bdesc + kk * 2, idesc, (t | kk) != 0 ? 1u : 0u);
-        } else {
-          const int e = t - nmain;
-          const int nkk = min(64, 2 * a.r - 64 * e) / 16;
-          for (int kk = 0; kk < nkk; ++kk)
-            umma_bf16(tmem_d, adesc + static_cast<uint32_t>(kk >> 1) * a_step, bdesc + static_cast<uint32_t>(kk) * 2,
-                      idesc, 1u);
+            for (uint32_t kk = 0; kk < 4; ++kk)
+              umma_bf16(tmem_d, adesc + kk * a_step, bdesc + kk * 2, idesc, (t | kk) != 0 ? 1u : 0u);
+          } else {
+            const int e = t - nmain;
+            const int nkk = min(64, 2 * a.r - 64 * e) / 16;
+            for (int kk = 0; kk < nkk; ++kk)
+              umma_bf16(tmem_d, adesc + static_cast<uint32_t>(kk >> 1) * a_step, bdesc + static_cast<uint32_t>(kk) * 2,
+                        idesc, 1u);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        __syncwarp();
       }
-      umma_commit(accf);
-      if (aborted) mbar_drain(accf, 0, a.status);
+      if (elect_one()) {
+        umma_commit(accf);
+        if (aborted) mbar_drain(accf, 0, a.status);
+      }
     }
     __syncwarp();
     grid_dependency_wait();
@@ -529,37 +536,44 @@ __global__ void __launch_bounds__(192, 1)
       grid_dependents_launch();
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptors); the
+    // elected lane issues the MMAs and the commits.
+    {
       const uint32_t idesc = idesc_bf16_f32(128, 256, DX ? 1 : 0, 0);
       const uint32_t a_step = DX ? (2048u >> 4) : (32u >> 4);
       bool aborted = false;
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) { aborted = true; break; }
+        if (!mbar_wait_all(&full[s], u & 1, wc)) { aborted = true; break; }
+        if (t < nmain && !mbar_wait_all(&wfull[s], u & 1, wc)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint32_t sa = sb + P::kB;
         const uint64_t b0 = sdesc_sw64(sb, 16, 512), b1 = sdesc_sw64(sb + P::kBh, 16, 512);
         const uint64_t ad = DX ? sdesc_sw128(sa, 4096, 1024) : sdesc_sw64(sa, 16, 512);
-        if (t < nmain) {
+        if (elect_one()) {
+          if (t < nmain) {
 #pragma unroll
-          for (uint32_t kk = 0; kk < 2; ++kk) {
-            const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
-            umma_bf16(tmem_d, ad + kk * a_step, b0 + kk * 2, idesc, acc);
-            umma_bf16(tmem_d + 256, ad + kk * a_step, b1 + kk * 2, idesc, acc);
-          }
-        } else {
+            for (uint32_t kk = 0; kk < 2; ++kk) {
+              const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
+              umma_bf16(tmem_d, ad + kk * a_step, b0 + kk * 2, idesc, acc);
+              umma_bf16(tmem_d + 256, ad + kk * a_step, b1 + kk * 2, idesc, acc);
+            }
+          } else {
 #pragma unroll
-          for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
-            umma_bf16(tmem_d, ad, b0 + part * 2, idesc, 1u);
-            umma_bf16(tmem_d + 256, ad, b1 + part * 2, idesc, 1u);
+            for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
+              umma_bf16(tmem_d, ad, b0 + part * 2, idesc, 1u);
+              umma_bf16(tmem_d + 256, ad, b1 + part * 2, idesc, 1u);
+            }
           }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        __syncwarp();
       }
-      umma_commit(accf);
-      if (aborted) mbar_drain(accf, 0, a.status);
+      if (elect_one()) {
+        umma_commit(accf);
+        if (aborted) mbar_drain(accf, 0, a.status);
+      }
     }
     __syncwarp();
     grid_dependency_wait();
