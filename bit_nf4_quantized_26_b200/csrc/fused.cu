@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&wfull[s], DQW);  // one elected arrival per dequantiser warp
+      mbar_init(&wfull[s], 4);  // one elected arrival per dequantiser warp of the stage
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -192,12 +192,14 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     grid_dependents_launch();
   } else {
     // ------------------------------------------------------------ dequantisers
-    // DQW == 4: thread dt owns tile row dt (one whole NF4 block per stage).
-    // DQW == 8: threads 2i and 2i+1 share tile row i, half a block each.
+    // Thread dt owns tile row dt % 128 (one whole NF4 block per stage).
+    // DQW == 8: two groups of four warps take alternate stages (two
+    // independent instruction streams per SM sub-partition).
     const int dt = threadIdx.x - 64;
     const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
-    const int rl = DQW == 4 ? dt : (dt >> 1);
-    const uint32_t half = DQW == 4 ? 0u : static_cast<uint32_t>(dt & 1);
+    const int rl = dt & 127;
+    constexpr int kStep = DQW / 4;  // stages between two of this group's
+    const int grp = dt >> 7;
     const int64_t kbpr = a.k_in / 64;  // NF4 blocks per W row
     auto block_of = [&](int t, int64_t& b) -> bool {
       const int kt = kt0 + t;
@@ -230,8 +232,8 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       }
     };
 #pragma unroll
-    for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
-    for (int t = 0; t < nmain; ++t) {
+    for (int i = 0; i < kPD; ++i) fetch(grp + kStep * i, pc[i], ps[i]);
+    for (int t = grp; t < nmain; t += kStep) {
       const uint32_t c8b = pc[0];
       const float s2v = ps[0];
 #pragma unroll
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         pc[i] = pc[i + 1];
         ps[i] = ps[i + 1];
       }
-      fetch(t + kPD, pc[kPD - 1], ps[kPD - 1]);
+      fetch(t + kStep * kPD, pc[kPD - 1], ps[kPD - 1]);
       int64_t bdummy;
       const bool valid = block_of(t, bdummy);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
@@ -259,22 +261,11 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         swz = nl & 7;
       }
       const float chat = valid ? nf4_block_scale(c8b, s2v, wmean) : 0.0f;
-      if (DQW == 4) {
-        if (valid) {
-          nf4_block_to_swizzled_row(src, nf4_make_lut(a.tab, chat), dst, swz);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
-        }
+      if (valid) {
+        nf4_block_to_swizzled_row(src, nf4_make_lut(a.tab, chat), dst, swz);
       } else {
-        const Nf4Lut lut = nf4_make_lut_pair(a.tab, chat, half);  // all lanes: full-mask shuffle
-        if (valid) {
-          nf4_half_block_to_swizzled_row(src + 16 * half, lut, dst, swz, half);
-        } else {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(dst + (4 * half + j) * 16) = make_uint4(0, 0, 0, 0);
-        }
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(dst + j * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();  // this lane's tile writes -> async proxy
       __syncwarp();
@@ -771,18 +762,19 @@ static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m
                        dim3(1, 1, static_cast<unsigned>(splits)), m0, m1, m2, m3, a);
 }
 
-// Dequantiser warps per CTA: four (one whole NF4 block per thread and stage,
-// no duplicated table work) measured faster than eight (half blocks, tables
-// built in pairs) at every tile width this kernel runs (64, 128 and 256
-// tokens: 95 / 114 / 206 us against 108 / 128 / 222 us on a 22016 x 8192
-// weight).  QLORA_DEQUANT_WARPS=8 selects eight.
+// Dequantiser warps per CTA: eight (two groups of four taking alternate
+// stages) measured 3-6% faster than four at 64 to 256 tokens on 22016 x 8192
+// and 8192 x 22016 weights (200 tokens: 196 against 208 us); each stage's
+// dequantisation is a chain of dependent byte permutes, and two groups give
+// each SM sub-partition two of them to interleave.  QLORA_DEQUANT_WARPS=4
+// selects four.
 static int dequant_warps(int bn) {
   static int forced = [] {
     const char* e = getenv("QLORA_DEQUANT_WARPS");
     return e ? atoi(e) : 0;
   }();
   (void)bn;
-  return forced == 8 ? 8 : 4;
+  return forced == 4 ? 4 : 8;
 }
 
 template <int BN, bool DX>
