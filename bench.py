@@ -47,13 +47,16 @@ WORKLOAD_NAME = ("LLaMA-7B-shaped decoder layer, all 7 linears (q,k,v,o 4096x409
 M_TOKENS = 8 * 2048
 RANK_R = 64
 ALPHA = 16.0
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# Earlier measurements on this GPU type, used when no measured-peaks file is
+# present: copy bandwidth, cuBLAS bf16 as a burst, and the same GEMM held for
+# seconds under the power cap (about 1.3 GHz).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NF4_BYTES_PER_PARAM = 2 + 0.5 + 1 / 64 + 4 / 16384
 # Per-launch DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # CTA-pair GEMMs in the grouped layer step (mean over the step's 4 launches of
 # each), from one ncu capture of the current kernels (the decoder-layer-step
 # summary under profiles/); emptied whenever those kernels change.
-NCU_TRAFFIC_BYTES = {"fused_fwd": 708.1e6, "fused_dx": 724.1e6}
+NCU_TRAFFIC_BYTES = {"fused_fwd": 705.5e6, "fused_dx": 722.1e6}
 
 
 def flops_fwd_bwd(M, N, K, r):
@@ -67,7 +70,7 @@ def load_peaks():
         return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
                 "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                 "source": "measured"}
-    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"], source="fallback")
+    return dict(FALLBACK_PEAKS, source="fallback")
 
 
 # ------------------------------------------------------------------ clocks
@@ -793,9 +796,14 @@ def run_ours(args, rank, world):
         for n in tc:
             kern[n]["tflops"] = layer.kernel_flops(n) / (kern[n]["ms_per_step"] * 1e-3) / 1e12
         ach = kern[dom]["tflops"]
-        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": NCU_TRAFFIC_BYTES.get(dom),
-                    "peak_source": f"{peaks['source']} bf16 burst",
+        # The kernel is timed inside a step of about 12 ms repeated back to
+        # back, under the power cap: the sustained GEMM figure is its peak; the
+        # fraction of the burst figure is reported beside it.
+        pk = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": pk,
+                    "unit": "TFLOP/s", "frac": ach / pk, "traffic": NCU_TRAFFIC_BYTES.get(dom),
+                    "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside the step)",
+                    "frac_of_burst": ach / peaks["bf16_tflops"], "burst_peak": peaks["bf16_tflops"],
                     "launches_per_step": kern[dom]["launches"] // args.steps,
                     "achieved_from": "algorithmic FLOPs of the kernel's launches in a step / their summed "
                                      "event time per step (phase B)"}
