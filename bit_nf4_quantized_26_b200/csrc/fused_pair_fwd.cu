@@ -18,12 +18,16 @@
 // Barriers (all bounded waits):
 //   cfull[s]  this CTA's packed codes landed (local TMA)
 //   full[s]   leader only: both CTAs' token / LoRA tiles landed (paired TMA)
-//   wfull[s]  leader only: both CTAs' A rows stored in tensor memory (one
-//             arrival per dequantiser warp after tcgen05.wait::st and the
-//             tcgen05 fence before the thread synchronisation)
+//             and both CTAs' A rows are stored in tensor memory (one arrival
+//             per dequantiser warp of the stage's group, after
+//             tcgen05.wait::st and the tcgen05 fence before the thread
+//             synchronisation): one barrier per stage for the MMA warp
 //   empty[s]  both CTAs: the pair's MMAs of the stage finished (multicast
 //             commit); the dequantisers also wait on it before reusing an A slot
 //   accf      both CTAs: the accumulators are final (multicast commit)
+// Warp 0 copies, warp 1 issues the MMAs (the whole warp runs the loop, an
+// elected lane issues), warps 2..9 are two groups of four dequantiser warps
+// taking alternate stages.
 // The adapter stages (r/16 of them) take their A operand (the rows of B) from
 // shared memory as in fused_pair.cu.  No TMA multicast is used.
 #include "kernels.h"
@@ -85,7 +89,7 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 // CTA scope, as for any cross-CTA pair barrier); a cluster-scope release costs
 // a memory barrier per warp and stage and measured 2.3-2.7x slower.
 template <int ASLOTS>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fused_pair_fwd_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_codes,
                           const __grid_constant__ CUtensorMap tm_uc, const __grid_constant__ CUtensorMap tm_ext,
                           const FusedArgs a) {
@@ -94,8 +98,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P::kBarOff);
   uint64_t* cfull = full + P::kStages;
-  uint64_t* wfull = cfull + P::kStages;
-  uint64_t* empty = wfull + P::kStages;
+  uint64_t* empty = cfull + P::kStages;
   uint64_t* accf = empty + P::kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -111,9 +114,8 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 8);  // the producer's expect-tx arrival + 4 dequantiser warps per CTA
       mbar_init(&cfull[s], 1);
-      mbar_init(&wfull[s], 8);  // one arrival per dequantiser warp, 4 per CTA
       mbar_init(&empty[s], 1);
     }
     mbar_init(accf, 1);
@@ -173,9 +175,12 @@ __global__ void __launch_bounds__(192, 1)
         issued = t + 1;
       }
       // Leave nothing in flight into this CTA's shared memory.
+      // The full barriers also count the dequantisers' arrivals, which may
+      // never come after an abort, so the drain then takes a short limit.
+      const uint64_t lim = *abort_flag ? 1000000ull : kWaitTimeoutNs;
       for (int t = max(0, issued - static_cast<int>(P::kStages)); t < issued; ++t) {
-        if (t < nmain) mbar_drain(&cfull[t % P::kStages], (t / P::kStages) & 1, a.status);
-        if (rank == 0) mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status);
+        if (t < nmain) mbar_drain(&cfull[t % P::kStages], (t / P::kStages) & 1, a.status, lim);
+        if (rank == 0) mbar_drain(&full[t % P::kStages], (t / P::kStages) & 1, a.status, lim);
       }
     }
     __syncwarp();
@@ -185,39 +190,42 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA (leader)
-    if (lane == 0 && rank == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptors); the
+    // elected lane issues the MMAs and the commits.
+    if (rank == 0) {
       const uint32_t idesc = idesc_bf16_f32(256, P::kN, 0, 0);
       bool aborted = false;
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
-        if (!mbar_wait(&full[s], u & 1, wc)) { aborted = true; break; }
-        if (t < nmain && !mbar_wait(&wfull[s], u & 1, wc)) {
-          aborted = true;
-          break;
-        }
+        if (!mbar_wait_all(&full[s], u & 1, wc)) { aborted = true; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + s * P::kStage);
         const uint64_t b0 = sdesc_sw64(sb, 16, 512), b1 = sdesc_sw64(sb + P::kBq, 16, 512);
-        if (t < nmain) {
-          const uint32_t at = tmem_d + P::kACol + static_cast<uint32_t>(t % P::kASlots) * 16;
+        const uint32_t at = tmem_d + P::kACol + static_cast<uint32_t>(t % P::kASlots) * 16;
+        const uint64_t ad = sdesc_sw64(smem_u32(smem + P::kExtOff + (t >= nmain ? t - nmain : 0) * P::kExt), 16, 512);
+        if (elect_one()) {
+          if (t < nmain) {
 #pragma unroll
-          for (uint32_t kk = 0; kk < 2; ++kk) {
-            const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
-            umma_bf16_pair_ta(tmem_d, at + kk * 8, b0 + kk * 2, idesc, acc);
-            umma_bf16_pair_ta(tmem_d + P::kN, at + kk * 8, b1 + kk * 2, idesc, acc);
-          }
-        } else {
-          const uint64_t ad = sdesc_sw64(smem_u32(smem + P::kExtOff + (t - nmain) * P::kExt), 16, 512);
+            for (uint32_t kk = 0; kk < 2; ++kk) {
+              const uint32_t acc = (t | kk) != 0 ? 1u : 0u;
+              umma_bf16_pair_ta(tmem_d, at + kk * 8, b0 + kk * 2, idesc, acc);
+              umma_bf16_pair_ta(tmem_d + P::kN, at + kk * 8, b1 + kk * 2, idesc, acc);
+            }
+          } else {
 #pragma unroll
-          for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
-            umma_bf16_pair(tmem_d, ad, b0 + part * 2, idesc, 1u);
-            umma_bf16_pair(tmem_d + P::kN, ad, b1 + part * 2, idesc, 1u);
+            for (uint32_t part = 0; part < 2; ++part) {  // hi, lo
+              umma_bf16_pair(tmem_d, ad, b0 + part * 2, idesc, 1u);
+              umma_bf16_pair(tmem_d + P::kN, ad, b1 + part * 2, idesc, 1u);
+            }
           }
+          umma_commit_pair(&empty[s], 0x3);
         }
-        umma_commit_pair(&empty[s], 0x3);
+        __syncwarp();
       }
-      umma_commit_pair(accf, 0x3);
-      if (aborted) mbar_drain(accf, 0, a.status);
+      if (elect_one()) {
+        umma_commit_pair(accf, 0x3);
+        if (aborted) mbar_drain(accf, 0, a.status);
+      }
     }
     __syncwarp();
     grid_dependency_wait();
@@ -226,8 +234,11 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ dequantisers
     // Warp w may access tensor-memory lanes 32 (w % 4) .. + 31 only, so the
     // thread dequantises W row rl = its lane there (A row i = TMEM lane i).
+    // Eight warps in two groups taking alternate stages; group g's four warps
+    // cover the four lane quarters.
     const int q = warp & 3;
     const int rl = q * 32 + lane;
+    const int grp = (threadIdx.x - 64) >> 7;
     const Nf4Mean wmean = nf4_load_mean(a.mean);  // from an earlier kernel: complete (see above)
     const int64_t kbpr = a.k_in / 64;
     const int n = row0 + rl;
@@ -248,18 +259,17 @@ __global__ void __launch_bounds__(192, 1)
     };
 #pragma unroll
     for (int i = 0; i < kPD; ++i) fetch(i, pc[i], ps[i]);
-    Nf4Lut lut{};
-    for (int t = 0; t < nmain; ++t) {
-      if ((t & 1) == 0) {
-        const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
+    // Stage t covers half of block t / 2: each group builds that block's
+    // table itself.
+    for (int t = grp; t < nmain; t += 2) {
+      const float chat = valid ? nf4_block_scale(pc[0], ps[0], wmean) : 0.0f;
 #pragma unroll
-        for (int i = 0; i + 1 < kPD; ++i) {
-          pc[i] = pc[i + 1];
-          ps[i] = ps[i + 1];
-        }
-        fetch(t / 2 + kPD, pc[kPD - 1], ps[kPD - 1]);
-        lut = nf4_make_lut(a.tab, chat);
+      for (int i = 0; i + 1 < kPD; ++i) {
+        pc[i] = pc[i + 1];
+        ps[i] = ps[i + 1];
       }
+      fetch(t / 2 + kPD, pc[kPD - 1], ps[kPD - 1]);
+      const Nf4Lut lut = nf4_make_lut(a.tab, chat);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
       if (!mbar_wait_all(&cfull[s], u & 1, wc)) break;
       // The A slot of stage t was last read by the MMAs of stage t - kASlots
@@ -289,7 +299,15 @@ __global__ void __launch_bounds__(192, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(dsmem_addr(&wfull[s], 0));
+      if (lane == 0) mbar_arrive_remote(dsmem_addr(&full[s], 0));
+    }
+    // Adapter stages: nothing to dequantise, but the stage's group still
+    // arrives on full[s], once the slot's previous stage (t - kStages, a main
+    // stage of this group) is retired, so the arrival falls in its own phase.
+    for (int t = nmain + ((grp - nmain) & 1); t < T; t += 2) {
+      const uint32_t s = t % P::kStages;
+      if (t >= static_cast<int>(P::kStages) && !mbar_wait_all(&empty[s], ((t / P::kStages) - 1) & 1, wc)) break;
+      if (lane == 0) mbar_arrive_remote(dsmem_addr(&full[s], 0));
     }
 
     grid_dependency_wait();
@@ -304,7 +322,9 @@ __global__ void __launch_bounds__(192, 1)
       const bool rok = orow < a.rows;
       const uint32_t tqd = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int cb = 0; cb < (2 * P::kN) / 32; ++cb) {
+      // the two groups take half of the column blocks each
+      constexpr int kCb = (2 * P::kN) / 32;
+      for (int cb = grp * ((kCb + 1) / 2); cb < min(kCb, (grp + 1) * ((kCb + 1) / 2)); ++cb) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tqd + cb * 32, v);
         tmem_ld_wait();
@@ -356,7 +376,7 @@ static cudaError_t launch_pair_fwd_impl(const CUtensorMap& tm_b, const CUtensorM
   }
   const int tok = 2 * P::kN;
   return launch_kernel(fused_pair_fwd_kernel<ASLOTS>, dim3(2 * ((a.rows + 255) / 256), (a.M + tok - 1) / tok, 1),
-                       dim3(192), P::kSmem, stream, dim3(2, 1, 1), tm_b, tm_codes, tm_uc, tm_ext, a);
+                       dim3(320), P::kSmem, stream, dim3(2, 1, 1), tm_b, tm_codes, tm_uc, tm_ext, a);
 }
 
 int pair_fwd_tokens(int slots) { return 512 - 16 * slots; }
