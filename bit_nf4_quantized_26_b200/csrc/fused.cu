@@ -36,13 +36,14 @@ struct FusedPlan {
   static constexpr uint32_t kStages = kFit > 8 ? 8 : kFit;
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 256;
-  // Split contraction: each CTA of the cluster parks its fp32 tile here (the
-  // idle ring), rows padded by 4 floats so that row-wise stores spread over
-  // the banks.
+  // Split contraction: the idle ring receives the slices of the partial tiles
+  // this CTA reduces, rows padded by 4 floats so that row-wise accesses
+  // spread over the banks.
   static constexpr uint32_t kPartLd = BN + 4;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kStages >= 3, "pipeline too shallow");
-  static_assert(128 * kPartLd * 4 <= kBarOff, "partial tile must fit in the ring");
+  // receive slots of a split reduction: S slots of ceil(128 / S) rows, S <= 8
+  static_assert(136 * kPartLd * 4 <= kBarOff, "split-reduction slots must fit in the ring");
 };
 
 template <int BN, bool DX, int DQW>
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
   // extension load; every other role passes the wait after its main loop,
   // before triggering the next kernel.
 
+  bool acc_ok = false;  // dequantiser warps: the accumulators are final
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     bool waited = false;
@@ -278,7 +280,8 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     // ------------------------------------------------------------ epilogue
     // Warp w reads TMEM lane quadrant w % 4; with 8 dequant warps the two
     // warps of a quadrant split the BN accumulator columns in halves.
-    if (mbar_wait_warp(accf, 0, wc)) {
+    acc_ok = mbar_wait_warp(accf, 0, wc);
+    if (acc_ok && gridDim.z == 1) {
       tc_fence_after();
       const int q = warp & 3;
       const int erow = q * 32 + lane;
@@ -288,22 +291,7 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       const int orow = row0 + erow;
       const bool rok = orow < a.rows;
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
-      if (gridDim.z > 1) {
-        // split contraction: this CTA's fp32 tile goes to its shared memory
-        float* prow = reinterpret_cast<float*>(smem) + erow * P::kPartLd;
-#pragma unroll 1
-        for (int ci = 0; ci < kChunks; ++ci) {
-          const int cb = cgrp * kChunks + ci;
-          if (cb >= kAll) break;  // warp-uniform
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tq + cb * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(prow + cb * 32 + j) = make_float4(
-                __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        }
-      } else {
+      {
 #pragma unroll 1
         for (int ci = 0; ci < kChunks; ++ci) {
           const int cb = cgrp * kChunks + ci;
@@ -338,44 +326,59 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
 
   if (gridDim.z > 1) {
     // Split contraction: the S CTAs of the cluster (one per slice of the
-    // contraction, cluster rank = blockIdx.z) each sum a slice of the tile's
-    // rows over all S partial tiles through distributed shared memory, in
-    // rank order 0..S-1 (deterministic), and write the outputs.  A thread
-    // takes four tokens of one W-side row and has the S partial loads in
-    // flight together; consecutive threads take consecutive rows, so the
-    // stores of a token's outputs are contiguous.
+    // contraction, cluster rank = blockIdx.z) reduce the tile together; CTA o
+    // owns rows [o R, o R + R) of it, R = ceil(128 / S).  Each CTA writes its
+    // accumulator rows straight from tensor memory into the owners' receive
+    // slots (slot = the writer's rank) with remote stores, which pipeline,
+    // and then every owner sums its slots from its own shared memory in rank
+    // order 0..S-1 (deterministic) and writes the outputs.
     __syncwarp();
-    cluster_sync_all();
+    cluster_sync_all();  // every CTA's rings are idle: its dequantiser warps saw accf
     const int S = static_cast<int>(gridDim.z);
-    const int rows_per = (128 + S - 1) / S;
-    const int r0 = z * rows_per, r1 = min(128, r0 + rows_per);
-    const int nrow = r1 - r0;
-    const float* part = reinterpret_cast<const float*>(smem);
+    const int R = (128 + S - 1) / S;
+    const uint32_t slot_bytes = static_cast<uint32_t>(R * P::kPartLd * 4);
+    if (acc_ok) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int erow = q * 32 + lane;
+      const int cgrp = DQW == 4 ? 0 : (warp - 2) / 4;
+      constexpr int kAll = BN / 32;
+      constexpr int kChunks = DQW == 4 ? kAll : (kAll + 1) / 2;
+      const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
+      const int own = erow / R;
+      const uint32_t dst0 = dsmem_addr(smem, static_cast<uint32_t>(own)) + static_cast<uint32_t>(z) * slot_bytes +
+                            static_cast<uint32_t>((erow - own * R) * P::kPartLd * 4);
+#pragma unroll 1
+      for (int ci = 0; ci < kChunks; ++ci) {
+        const int cb = cgrp * kChunks + ci;
+        if (cb >= kAll) break;  // warp-uniform
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tq + cb * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          dsmem_st_f4(dst0 + static_cast<uint32_t>((cb * 32 + j) * 4), __uint_as_float(v[j]),
+                      __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // every slot is written
+    const int r0 = z * R, nrow = min(128, r0 + R) - r0;
+    const float* slots = reinterpret_cast<const float*>(smem);
     const int64_t ld = a.ld_out;
     constexpr int kC4 = BN / 4;
     for (int e = threadIdx.x; e < nrow * kC4; e += blockDim.x) {
-      const int row = r0 + e % nrow, c4 = (e / nrow) * 4;
-      const uint32_t off = static_cast<uint32_t>((row * P::kPartLd + c4) * 4);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k0 = 0; k0 < 8; k0 += 4) {  // four loads in flight, added in rank order
-        float4 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (k0 + k < S) v[k] = dsmem_ld_f4(dsmem_addr(part, static_cast<uint32_t>(k0 + k)) + off);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k0 + k == 0) {
-            acc = v[0];
-          } else if (k0 + k < S) {
-            acc.x = __fadd_rn(acc.x, v[k].x);
-            acc.y = __fadd_rn(acc.y, v[k].y);
-            acc.z = __fadd_rn(acc.z, v[k].z);
-            acc.w = __fadd_rn(acc.w, v[k].w);
-          }
-        }
+      const int row = e % nrow, c4 = (e / nrow) * 4;
+      const float* src = slots + row * P::kPartLd + c4;
+      float4 acc = *reinterpret_cast<const float4*>(src);
+      for (int k = 1; k < S; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(src + k * R * P::kPartLd);
+        acc.x = __fadd_rn(acc.x, v.x);
+        acc.y = __fadd_rn(acc.y, v.y);
+        acc.z = __fadd_rn(acc.z, v.z);
+        acc.w = __fadd_rn(acc.w, v.w);
       }
-      const int orow = row0 + row;
+      const int orow = row0 + r0 + row;
       const float o[4] = {acc.x, acc.y, acc.z, acc.w};
       if (orow < a.rows) {
 #pragma unroll
@@ -388,8 +391,6 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
         }
       }
     }
-    __syncwarp();
-    cluster_sync_all();  // peers may still be reading this CTA's partial tile
   }
 
   tc_fence_before();

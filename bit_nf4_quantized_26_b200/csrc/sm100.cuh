@@ -297,6 +297,12 @@ __device__ __forceinline__ float dsmem_ld_f32(uint32_t cluster_addr) {
   return v;
 }
 
+__device__ __forceinline__ void dsmem_st_f4(uint32_t cluster_addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t cluster_addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
