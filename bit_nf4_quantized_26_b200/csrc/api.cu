@@ -372,6 +372,30 @@ void split_plan(int64_t tiles, int64_t stages, int64_t min_per, int64_t cta_budg
   splits = static_cast<int>(cdiv(stages, p));
 }
 
+// Slices of the contraction for the mid-size kernels (M <= 256, 128 W-side
+// rows x bn tokens per tile, kst 64-deep stages).  The weight streams through
+// once; splitting the contraction (a cluster, reduced in distributed shared
+// memory) fills the SMs, but every slice adds a reduction and its cluster
+// must be placed whole: s minimises waves(s) x (stages per slice + 3 s), with
+// 2 CTAs per SM for tiles of up to 128 tokens (s <= 4) and 1 for 256
+// (s <= 2), at least 8 stages per slice.  This model picked the measured best
+// (or within a few percent of it) for 64-256 tokens on 22016x8192,
+// 8192x22016, 4096x4096 and 11008x4096 weights.
+void mid_splits(int64_t tiles, int64_t kst, int bn, int& splits, int& per) {
+  const int64_t slots = (bn <= 128 ? 2 : 1) * kSms;
+  const int64_t smax = std::min<int64_t>(bn <= 128 ? 4 : 2, std::max<int64_t>(1, kst / 8));
+  int64_t best_s = 1, best_cost = -1;
+  for (int64_t sl = 1; sl <= smax; ++sl) {
+    const int64_t cost = cdiv(tiles * sl, slots) * (cdiv(kst, sl) + (sl > 1 ? 3 * sl : 0));
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_s = sl;
+    }
+  }
+  per = static_cast<int>(cdiv(kst, best_s));
+  splits = static_cast<int>(cdiv(kst, per));
+}
+
 struct FwdPlan {
   int s_down, per_down;
   int bn, s_fwd, per_fwd;
@@ -423,15 +447,7 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   p.bn = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
   const int64_t tiles = cdiv(N, 128) * cdiv(M, p.bn);
   if (M <= 256) {
-    // The weight streams through once: spread it over several waves of CTAs
-    // (balanced SMs), at most 8 slices of the contraction (a cluster, reduced
-    // in distributed shared memory) of at least 8 stages each.
-    int64_t s = cdiv(4 * kSms, tiles);
-    s = std::min<int64_t>(s, kMaxCluster);
-    s = std::min<int64_t>(s, std::max<int64_t>(1, kst / 8));
-    s = std::max<int64_t>(s, 1);
-    p.per_fwd = static_cast<int>(cdiv(kst, s));
-    p.s_fwd = static_cast<int>(cdiv(kst, p.per_fwd));
+    mid_splits(tiles, kst, p.bn, p.s_fwd, p.per_fwd);
   } else {
     p.s_fwd = 1;
     p.per_fwd = static_cast<int>(kst);
@@ -445,7 +461,7 @@ FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
 }
 
 struct BwdPlan {
-  int s_du, per_du, s_db, per_db, s_da, per_da, bn;
+  int s_du, per_du, s_db, per_db, s_da, per_da, bn, s_dx, per_dx;
   size_t off_sucat, off_ducat, total;
 };
 
@@ -463,6 +479,10 @@ BwdPlan plan_bwd(int64_t M, int64_t N, int64_t K, int32_t r, int G, int64_t n_ma
   split_plan(cdiv(N, 128), cdiv(M, 64), 4, kSms / 2, p.s_db, p.per_db);
   split_plan(cdiv(K, 128) * G, cdiv(M, 64), 4, kSms / 2, p.s_da, p.per_da);
   p.bn = M > 128 ? 256 : 128;
+  // the mid-size dX GEMM (M <= 256): contraction over the N outputs
+  p.s_dx = 1;
+  p.per_dx = static_cast<int>(n_max / 64);
+  if (M <= kWideM) mid_splits(cdiv(K, 128) * cdiv(M, p.bn), N / 64, p.bn, p.s_dx, p.per_dx);
   size_t off = 0;
   p.off_sucat = off;
   off += align256(static_cast<size_t>(M) * 2 * G * r * 2);
@@ -952,12 +972,12 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     fa.k_in = Ki;
     fa.r = gemm_r;
     fa.kt_total = static_cast<int>(N / 64);
-    fa.kt_per_split = static_cast<int>(N / 64);
+    fa.kt_per_split = p.per_dx;
     fa.status = d_status;
     fa.tab = tables();
     fa.groups = 1;
     ProfScope ps(kKFusedDX, cs);
-    if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, cs))) return st;
+    if (qlora_status st = from_cuda(launch_fused_dx(p.bn, mdy, mc, mdu, mal, fa, p.s_dx, cs))) return st;
   }
   if (drop) {  // dX = dX_main + keep * c * (dU A), on the caller's stream after the GEMM
     ProfScope ps(kKDropoutDx, cs);

@@ -798,11 +798,11 @@ cudaError_t launch_fused_fwd(int bn, const CUtensorMap& tm_x, const CUtensorMap&
 }
 
 cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap& tm_codes,
-                            const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a,
+                            const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a, int splits,
                             cudaStream_t stream) {
   switch (bn) {
-    case 128: return launch_fused_dqw<128, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
-    case 256: return launch_fused_dqw<256, true>(tm_dy, tm_codes, tm_duc, tm_al, a, 1, stream);
+    case 128: return launch_fused_dqw<128, true>(tm_dy, tm_codes, tm_duc, tm_al, a, splits, stream);
+    case 256: return launch_fused_dqw<256, true>(tm_dy, tm_codes, tm_duc, tm_al, a, splits, stream);
     default: return cudaErrorInvalidValue;
   }
 }

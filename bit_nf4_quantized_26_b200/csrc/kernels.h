@@ -163,7 +163,7 @@ cudaError_t launch_fused_fwd(int bn, const CUtensorMap& tm_x, const CUtensorMap&
 //   tm_dy: dY [M,N] box {64, BN} SW128; tm_codes: codes [N, K/2] box {64, 64};
 //   tm_duc: dUcat [M, 2r] box {64, BN} SW128; tm_al: A [r, K] box {64, 64} SW128.
 cudaError_t launch_fused_dx(int bn, const CUtensorMap& tm_dy, const CUtensorMap& tm_codes,
-                            const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a,
+                            const CUtensorMap& tm_duc, const CUtensorMap& tm_al, const FusedArgs& a, int splits,
                             cudaStream_t stream);
 
 // Large-M forward / dX: 128 W-side rows x 512 tokens per CTA, 32-deep stages.
