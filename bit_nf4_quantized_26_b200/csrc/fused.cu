@@ -247,6 +247,12 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       int64_t bdummy;
       const bool valid = block_of(t, bdummy);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
+      // With two groups and an odd ring the slot's previous stage t - kStages
+      // belongs to the other group, and this group may get here before that
+      // stage's copy has landed; a parity wait on full[s] would then see the
+      // older phase as this one.  Waiting first for the MMA of stage
+      // t - kStages (which the refill needs anyway) rules that out.
+      if (kStep == 2 && (P::kStages & 1) && u > 0 && !mbar_wait_all(&empty[s], (u - 1) & 1, wc)) break;
       if (!mbar_wait_all(&full[s], u & 1, wc)) break;
       uint8_t* st = smem + s * P::kStage;
       const uint8_t* src;

@@ -37,6 +37,9 @@ struct PlanPair {
   static constexpr uint32_t kSmem = 1024 + kBarOff + 512;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kSmem <= 232448u, "too much shared memory");
+  // two dequantiser groups take alternate stages: with an even ring a slot's
+  // previous stage is the same group's, so the parity waits cannot alias
+  static_assert(kStages % 2 == 0, "two alternating dequantiser groups need an even ring");
 };
 
 }  // namespace

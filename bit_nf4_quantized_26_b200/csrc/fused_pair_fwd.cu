@@ -47,9 +47,10 @@ struct PlanPairT {
   static constexpr uint32_t kExtBufs = 4;        // one per adapter stage: r / 16 <= 4
   static constexpr int kASlots = ASLOTS;
   static constexpr uint32_t kACol = 2 * kN;      // first tensor-memory column of the A ring
-  // As many stages as shared memory holds beside the adapter buffers: the
-  // ring's depth in time is what hides the copies' latency.
-  static constexpr uint32_t kStages = (232448u - 1024u - 512u - kExtBufs * kExt) / kStage;
+  // As many stages as shared memory holds beside the adapter buffers (the
+  // ring's depth in time is what hides the copies' latency), rounded down to
+  // an even count for the two alternating dequantiser groups.
+  static constexpr uint32_t kStages = ((232448u - 1024u - 512u - kExtBufs * kExt) / kStage) & ~1u;
   static constexpr uint32_t kExtOff = kStages * kStage;
   static constexpr uint32_t kBarOff = kExtOff + kExtBufs * kExt;
   static constexpr uint32_t kSmem = 1024 + kBarOff + 512;
@@ -57,6 +58,9 @@ struct PlanPairT {
   static_assert(kBq % 512 == 0, "64-byte swizzle atoms");
   static_assert(kACol + 16 * kASlots <= 512, "tensor memory");
   static_assert(kStages >= 8 && kStages <= 16, "ring depth");
+  // two dequantiser groups take alternate stages: with an even ring a slot's
+  // previous stage is the same group's, so the parity waits cannot alias
+  static_assert(kStages % 2 == 0, "two alternating dequantiser groups need an even ring");
   static_assert(kSmem <= 232448u, "too much shared memory");
 };
 
