@@ -418,6 +418,20 @@ def qlora_selftest_timeout(status, limit_ns, stream=None):
     _check(_lib.qlora_selftest_timeout(_ptr(status), int(limit_ns), _stream(stream)), "qlora_selftest_timeout")
 
 
+# ------------------------------------------------------ few-token kernel choice
+
+_lib.qlora_set_few_token_threshold.argtypes = [_I64]
+_lib.qlora_set_few_token_threshold.restype = _I64
+EXPORTED = EXPORTED + ("qlora_set_few_token_threshold",)
+DEFAULT_FEW_TOKEN_THRESHOLD = 1 << 26
+
+
+def qlora_set_few_token_threshold(min_weight_elems):
+    """Weights of at least this many elements run the few-token kernel for
+    M <= 16 tokens (0: always, a huge value: never); returns the previous value."""
+    return int(_lib.qlora_set_few_token_threshold(int(min_weight_elems)))
+
+
 # ------------------------------------------------------ grouped projections
 # (include/qlora_nf4.h: linears sharing one input, stacked along the outputs)
 

@@ -1,6 +1,7 @@
 // api.cu — the C ABI declared in include/qlora_nf4.h: argument checks,
 // workspace planning, TMA descriptor creation and kernel launches.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -412,7 +413,7 @@ FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   FwdPlan p{};
   p.low = true;
   split_plan(G, K / 64, 4, 2 * kSms, p.s_down, p.per_down);
-  p.low_mpad = M <= 8 ? 8 : (M <= 16 ? 16 : 32);
+  p.low_mpad = M <= 8 ? 8 : 16;
   p.low_tiles = static_cast<int>(cdiv(N, kLowmRows));
   p.low_kc = static_cast<int>(cdiv(K / 64, 4));
   const int64_t units = static_cast<int64_t>(p.low_tiles) * p.low_kc;
@@ -431,8 +432,19 @@ FwdPlan plan_fwd_low(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
   return p;
 }
 
+// Few tokens run the register-path kernel only on a large weight: it streams
+// the weight at a higher rate there (22016x8192 at 1 token: 68.6 us against
+// 83.0 for the mid-size kernel), while on smaller weights its fixed costs
+// dominate and the mid-size kernel is faster (4096x4096: 25.6 against 20.5
+// us).  The threshold is a process-wide setting (qlora_set_few_token_threshold).
+std::atomic<int64_t> g_few_token_min_elems{int64_t(1) << 26};
+
+bool few_token_path(int64_t M, int64_t N, int64_t K) {
+  return M <= kLowmMaxM && N * K >= g_few_token_min_elems.load(std::memory_order_relaxed);
+}
+
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
-  if (M <= kLowmMaxM) return plan_fwd_low(M, N, K, r, G);
+  if (few_token_path(M, N, K)) return plan_fwd_low(M, N, K, r, G);
   FwdPlan p{};
   const int64_t kst = K / 64;
   split_plan(cdiv(M, 128) * G, kst, 4, 2 * kSms, p.s_down, p.per_down);
@@ -580,6 +592,10 @@ int32_t qlora_profile_collect(int32_t* kernel_ids, float* ms, int32_t capacity) 
 
 const char* qlora_kernel_name(int32_t id) {
   return (id >= 0 && id < kKCount) ? kKernelNames[id] : "unknown";
+}
+
+int64_t qlora_set_few_token_threshold(int64_t min_weight_elems) {
+  return g_few_token_min_elems.exchange(min_weight_elems < 0 ? 0 : min_weight_elems);
 }
 
 const char* qlora_strerror(qlora_status s) {

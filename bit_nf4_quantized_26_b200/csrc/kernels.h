@@ -202,7 +202,7 @@ cudaError_t launch_skinny(int mode, const CUtensorMap& tmA, const CUtensorMap& t
 // s U B^T (U from the rank-r kernel launched just before).  See lowm.cu.
 constexpr int kLowmThreads = 256;
 constexpr int kLowmRows = 128;
-constexpr int kLowmMaxM = 32;
+constexpr int kLowmMaxM = 16;  // token rows the few-token kernel takes (8 or 16 per MMA column block)
 
 struct LowmArgs {
   const uint8_t* codes;  // [N, K/2]

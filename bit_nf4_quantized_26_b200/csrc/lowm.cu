@@ -1,10 +1,10 @@
-// lowm.cu — QLoRA linear forward for a few tokens (M <= 32):
+// lowm.cu — QLoRA linear forward for a few tokens (M <= 16) on a large weight:
 //   Y = X W'^T + s (X A^T) B^T,  W' = NF4-dequantised frozen weight
 // ("QLoRA" encyclopedia entry, tonho.wtf, section "como funciona": the
 // frozen weight is stored in NF4 and turned back into BFloat16 only where it
 // is used; the adapters stay 16-bit).
 //
-// At M <= 32 the product does at most 64 flops per byte of NF4 codes, so the
+// At M <= 16 the product does at most 64 flops per byte of NF4 codes, so the
 // weight stream and the nibble-to-bf16 lookups bound it, not the tensor
 // pipe.  This kernel therefore keeps the dequantised weight in registers:
 // every lane turns its own codes into bf16 pairs with byte-permute lookups
@@ -25,7 +25,7 @@
 //
 // Lane 0 of warp 0 streams each unit's codes (one 128 x 128-byte TMA box) and
 // its X slice (four 64-feature boxes; rows past M and features past K arrive
-// as zeros) into a shared-memory ring (four stages, three for 32 tokens), two
+// as zeros) into a shared-memory ring of four stages, two
 // units ahead of the unit being computed.  No warp is set aside for the
 // copies, so every warp has the full register budget.
 //
@@ -50,7 +50,7 @@ template <int NT>
 struct LowmPlan {
   static constexpr uint32_t kXBox = 8 * NT * 128;  // {64 features, 8 NT tokens} bf16
   static constexpr uint32_t kStage = kLowmCodes + 4 * kXBox;
-  static constexpr int kStages = NT <= 2 ? 4 : 3;  // two CTAs per SM either way
+  static constexpr int kStages = 4;  // two CTAs per SM
   static constexpr uint32_t kBarOff = kStages * kStage;
   static constexpr uint32_t kSmem = kBarOff + 2 * kStages * 8 + 16 + 1024;
   static_assert(kStages > kLowmAhead, "ring must hold the units in flight plus the one computed");
@@ -416,7 +416,6 @@ cudaError_t launch_lowm_fwd(const CUtensorMap& tm_codes, const CUtensorMap& tm_x
   switch (a.mpad) {
     case 8: return launch_lowm_impl<1>(tm_codes, tm_x, a, stream);
     case 16: return launch_lowm_impl<2>(tm_codes, tm_x, a, stream);
-    case 32: return launch_lowm_impl<4>(tm_codes, tm_x, a, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -352,6 +352,22 @@ QLORA_API const char* qlora_kernel_name(int32_t kernel_id);
  */
 QLORA_API qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_ns, void* stream);
 
+/*
+ * qlora_set_few_token_threshold — which forward kernel runs for few tokens
+ * (a performance setting; results are the same within the GEMM tolerances,
+ * and the dequantised weight is bit-exact either way).  A forward (or a
+ * group's) with M <= 16 token rows and a weight of at least
+ * `min_weight_elems` elements (N x K, stacked outputs for a group) runs the
+ * register-path few-token kernel; anything else with M <= 256 runs the
+ * mid-size tensor-core kernel.  Default 2^26 elements, the measured
+ * crossover on B200 (the few-token kernel streams large weights faster; on
+ * smaller ones its fixed costs dominate).  0 selects the few-token kernel
+ * for every M <= 16; INT64_MAX never.  Negative values count as 0.
+ * Process-wide and thread-safe; it changes the workspace sizes of later
+ * queries, so set it before querying.  Returns the previous value.
+ */
+QLORA_API int64_t qlora_set_few_token_threshold(int64_t min_weight_elems);
+
 /* Static, NUL-terminated description of a status code. */
 QLORA_API const char* qlora_strerror(qlora_status status);
 

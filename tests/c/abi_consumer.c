@@ -36,6 +36,11 @@ int main(void) {
 
   /* Status strings. */
   CHECK(strcmp(qlora_strerror(QLORA_OK), "ok") == 0);
+  {
+    const int64_t prev = qlora_set_few_token_threshold(0);
+    CHECK(prev == ((int64_t)1 << 26));
+    CHECK(qlora_set_few_token_threshold(prev) == 0);
+  }
   for (int s = 0; s <= QLORA_ERR_INTERNAL; ++s) CHECK(qlora_strerror((qlora_status)s) != NULL);
 
   /* Argument checks that return before any device work. */

@@ -27,3 +27,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture
+def few_token_kernel():
+    """Run every forward with M <= 16 tokens on the few-token kernel, whatever
+    the weight's size (the library's default sends small weights to the
+    mid-size kernel); restores the previous setting afterwards."""
+    import bit_nf4_quantized_26_b200 as lib
+    prev = lib.qlora_set_few_token_threshold(0)
+    yield
+    lib.qlora_set_few_token_threshold(prev)

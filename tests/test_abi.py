@@ -27,7 +27,7 @@ def declared_functions():
 
 def test_header_declarations_are_exported():
     names = declared_functions()
-    assert len(names) == 27
+    assert len(names) == 28
     lib = q.raw()
     for n in names:
         assert hasattr(lib, n), n
@@ -238,3 +238,20 @@ def test_selftest_timeout_argument_checks():
     assert f(P(256), 10, None) == SHAPE
     assert f(P(256), 3_000_000_000, None) == SHAPE
     assert f(P(260), 5_000_000, None) == ALIGN
+
+
+def test_few_token_threshold_setting():
+    """The setter returns the previous value (default 2^26 elements) and
+    changes the forward's plan: M <= 16 on a small weight uses the few-token
+    kernel's partial buffers only when forced (host-only workspace queries)."""
+    prev = q.qlora_set_few_token_threshold(0)
+    assert prev == q.DEFAULT_FEW_TOKEN_THRESHOLD
+    try:
+        forced = q.qlora_fwd_workspace_size(8, 512, 512, 16)
+        assert q.qlora_set_few_token_threshold(1 << 62) == 0
+        mid = q.qlora_fwd_workspace_size(8, 512, 512, 16)
+        assert forced != mid
+        assert q.qlora_set_few_token_threshold(-5) == 1 << 62
+        assert q.qlora_set_few_token_threshold(prev) == 0  # negative counts as 0
+    finally:
+        q.qlora_set_few_token_threshold(prev)

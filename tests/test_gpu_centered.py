@@ -90,7 +90,7 @@ def _sub(lib, W, n):
 
 
 @pytest.mark.parametrize("M", [8, 32, 64, 200, 1024])
-def test_centred_forward_dequant_is_exact(centred, M):
+def test_centred_forward_dequant_is_exact(centred, M, few_token_kernel):
     """Y = one-hot X W'^T with B = 0 equals W'[:, cols]^T: few tokens, 64- and
     256-token tiles, and above 256 tokens both the single-CTA kernel (1920
     rows) and the CTA pairs (the first 1792 rows)."""
@@ -139,7 +139,7 @@ def test_centred_pair_dx_dequant_is_exact():
 
 
 @pytest.mark.parametrize("M", [16, 128, 700])
-def test_centred_linear_matches_oracle(M):
+def test_centred_linear_matches_oracle(M, few_token_kernel):
     """Forward and backward on a mean-centred weight against the fp64 oracle
     on the oracle's centred dequantised weight."""
     lib = _lib()

@@ -25,9 +25,9 @@ position within an NF4 block and within a kernel's contraction chunk), where
 the test also checks that all 16 codes occur.
 
 Paths, by the library's dispatch rules:
-  forward  M <= 32: few-token kernel (8, 16, 32 token rows);
-           33..256: tcgen05 kernel with 64 (eight dequantiser warps, half a
-           block per thread), 128 and 256 token columns and a split
+  forward  M <= 16 on a weight of at least 2^26 elements (this one): the
+           few-token kernel (8, 16 token rows); other M <= 256: tcgen05
+           kernel with 32, 64, 128 and 256 token columns and a split
            contraction;  > 256: CTA-pair kernel (W rows % 256 == 0) or the
            single-CTA 512-token kernel (other W row counts);
   dX       M <= 256: tcgen05 kernel, 128 / 256 token columns, MN-major tiles;

@@ -37,7 +37,7 @@ SHAPES = [(16, 320, 512, 16),     # few tokens (register path)
 
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("p", [0.05, 0.5])
-def test_dropout_forward_backward_match_oracle(shape, p):
+def test_dropout_forward_backward_match_oracle(shape, p, few_token_kernel):
     M, N, K, r = shape
     d, g, W, wd = _case(M, N, K, r)
     s, seed = 0.25, 1234567 + (1 << 33)
@@ -72,7 +72,7 @@ def test_dropout_adapter_term_of_dx_matches_oracle_in_fp32():
     assert ol.rel_frobenius(term, term_ref) <= 1e-3
 
 
-def test_dropout_p_zero_forward_equals_plain_forward():
+def test_dropout_p_zero_forward_equals_plain_forward(few_token_kernel):
     M, N, K, r = 600, 512, 768, 64
     d, g, W, wd = _case(M, N, K, r, seed=5)
     Y, U, Xd = q.qlora_linear_fwd_dropout(g["X"], W, g["A"], g["B"], 0.5, 0.0, 1)

@@ -15,7 +15,7 @@ def _bits(t):
 
 
 @pytest.mark.parametrize("M,N,K,r", [(64, 512, 512, 16), (12, 1024, 2048, 64), (700, 512, 1024, 32)])
-def test_graph_replay_matches_eager(M, N, K, r):
+def test_graph_replay_matches_eager(M, N, K, r, few_token_kernel):
     import bit_nf4_quantized_26_b200 as lib
     dev = torch.device("cuda")
     g = {k: v.to(dev) for k, v in synth.linear_inputs(synth.Linear("g", N, K), M, r, 3).items()}

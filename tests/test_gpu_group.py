@@ -65,7 +65,7 @@ def _run(d, members, s, dtype):
     (700, (512, 256, 256), 768, 64),    # CTA pairs (boundaries on 256 rows)
     (600, (384, 128), 512, 48),         # single-CTA 512-token kernel (boundary on 384)
 ])
-def test_group_matches_oracle(M, members, K, r):
+def test_group_matches_oracle(M, members, K, r, few_token_kernel):
     s = 16.0 / r
     d = _inputs(M, members, K, r, seed=M + K)
     for dtype, tol in ((1, TOL_F32), (0, TOL_BF16)):

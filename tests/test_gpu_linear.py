@@ -92,16 +92,24 @@ def test_ragged_shapes(M, N, K, r):
     (11, 1024, 16384, 48), (16, 4096, 4096, 32), (17, 320, 832, 48), (24, 1088, 2112, 64),
     (32, 960, 4160, 16), (29, 2048, 8192, 32),
 ])
-def test_few_tokens(M, N, K, r):
-    """M <= 32 forward path: row tiles with a half-empty last tile (N % 128 =
-    64), K chunks with 1..3 of their 4 blocks present, 1..19 units per CTA,
-    ranges that start and end inside a tile, r = 16..64 rows of A, 1, 2 and 4
-    token tiles of 8."""
+def test_few_tokens(M, N, K, r, few_token_kernel):
+    """M <= 16: the few-token kernel, forced whatever the weight's size: row
+    tiles with a half-empty last tile (N % 128 = 64), K chunks with 1..3 of
+    their 4 blocks present, 1..19 units per CTA, ranges that start and end
+    inside a tile, r = 16..64, 1 and 2 token tiles of 8.  M = 17..32: the
+    mid-size kernel with 32-token tiles."""
     _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=1)
     _check_full(M, N, K, r, 16.0 / r, 3 * M + N + K, out_dtype=0)
 
 
-def test_few_tokens_forward_is_deterministic():
+@pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 16), (12, 1088, 2112, 32), (16, 4096, 4096, 32), (9, 4096, 11008, 64)])
+def test_few_tokens_default_dispatch(M, N, K, r):
+    """With the library's default threshold a weight below 2^26 elements runs
+    few tokens on the mid-size kernel: the same tolerances."""
+    _check_full(M, N, K, r, 16.0 / r, 5 * M + N + K, out_dtype=1)
+
+
+def test_few_tokens_forward_is_deterministic(few_token_kernel):
     lib = _lib()
     d = {k: v.cuda() for k, v in _inputs(13, 2048, 8192, 64, 12).items()}
     W = lib.quantize_weight(d["W"])
@@ -110,6 +118,34 @@ def test_few_tokens_forward_is_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(u1.view(torch.int32), u2.view(torch.int32))
+
+
+@pytest.mark.parametrize("M,N,K,r", [(9, 4096, 11008, 64), (100, 4096, 11008, 64), (48, 2048, 8192, 32)])
+def test_mid_size_repeatable_under_churn(M, N, K, r):
+    """Mid-size GEMMs with split contractions and two dequantiser groups over
+    a three-stage ring: every repetition, with other work between them to
+    shift the copies' timing, gives the same bits (a stage dequantised from a
+    stale ring slot shows as a tile that differs), and the first matches the
+    oracle."""
+    lib = _lib()
+    d = {k: v.cuda() for k, v in _inputs(M, N, K, r, 7 * M + r).items()}
+    W = lib.quantize_weight(d["W"])
+    churn = torch.empty(64 << 20, dtype=torch.float32, device="cuda")  # 256 MB: more than L2
+    y0, u0 = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.5)
+    g0 = lib.qlora_linear_bwd(d["dY"], d["X"], u0, W, d["A"], d["B"], 0.5)
+    for i in range(12):
+        churn.add_(1.0)
+        y, u = lib.qlora_linear_fwd(d["X"], W, d["A"], d["B"], 0.5)
+        g = lib.qlora_linear_bwd(d["dY"], d["X"], u, W, d["A"], d["B"], 0.5)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), y0.view(torch.int16)), f"Y differs at repetition {i}"
+        assert torch.equal(g[0].view(torch.int16), g0[0].view(torch.int16)), f"dX differs at repetition {i}"
+    got = {"Y": y0.float().cpu().numpy(), "dX": g0[0].float().cpu().numpy()}
+    Wd = oracle_dequant_full(bits(d["W"]))
+    _, Y = ol.linear_fwd(bits(d["X"]), Wd, bits(d["A"]), bits(d["B"]), 0.5)
+    assert rel(got["Y"], Y) <= TOL_BF16
+    dX = ol.linear_bwd(bits(d["dY"]), bits(d["X"]), Wd, bits(d["A"]), bits(d["B"]), 0.5)[0]
+    assert rel(got["dX"], dX) <= TOL_BF16
 
 
 def test_lora_path_alone_w_zero():

@@ -43,7 +43,7 @@ def _noalloc_raw(lib, X, W, A, B, s, Y, U, status):
                                               float(s), _p(Y), 0, _p(U), _p(status), stream)
 
 
-def test_noalloc_forward_matches_workspace_forward_and_oracle():
+def test_noalloc_forward_matches_workspace_forward_and_oracle(few_token_kernel):
     lib = _lib()
     # few-token kernel (split partials in the scratch), 64-token tiles with a
     # split contraction, and the CTA-pair kernel; one call after another
