@@ -344,6 +344,19 @@ class LayerStep:
             u["opt"].close()
 
 
+def with_clocks(dev, fn):
+    """Run fn() with the SM clock sampled beside it: (*result, clocks) for a
+    tuple result, else (result, clocks)."""
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.2)
+    try:
+        res = fn()
+    finally:
+        clocks = sampler.stop()
+    return (*res, clocks) if isinstance(res, tuple) else (res, clocks)
+
+
 def time_steps(torch, step, stream, steps, flush, dist=None):
     """Per-step device times (ms) of `steps` steps, one event pair each, L2
     flushed (512 MB memset) before every step outside its events."""
@@ -753,10 +766,27 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     M = args.tokens
-    layer = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=not args.no_group)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     dd = dist if world > 1 else None
+    peaks = load_peaks()
+
+    # The standalone NF4 streams first: quantisation runs when a model is
+    # loaded, not in the power-capped wake of a training step, and both
+    # kernels are issue- or bandwidth-bound, so they follow the SM clock
+    # (sampled beside them).
+    nf4_extras = {}
+    if rank == 0 and not args.no_sweep:
+        quant_gbs, dequant_gbs, nf4_clocks = with_clocks(
+            dev, lambda: nf4_stream_timing(lib, synth, torch, dev, flush))
+        nf4_extras["nf4_quantize_gbs"] = quant_gbs
+        nf4_extras["nf4_dequantize_gbs"] = dequant_gbs
+        nf4_extras["nf4_hbm_frac"] = {"quantize": quant_gbs / peaks["hbm_gbs"],
+                                      "dequantize": dequant_gbs / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
+                                      "peak_source": peaks["source"], "clocks": nf4_clocks,
+                                      "when": "before the layer-step phases"}
+
+    layer = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=not args.no_group)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -788,7 +818,6 @@ def run_ours(args, rank, world):
     assert int(layer.status[0].item()) == 0, f"device status {int(layer.status[0].item())}"
 
     kern = kernel_table(records, args.steps)
-    peaks = load_peaks()
     tc = {n: k for n, k in kern.items() if n in ("fused_fwd", "fused_dx")}
     roofline = None
     if tc:
@@ -870,19 +899,19 @@ def run_ours(args, rank, world):
         again.close()
         del flat, again
     if rank == 0 and not args.no_sweep:
-        quant_gbs, dequant_gbs = nf4_stream_timing(lib, synth, torch, dev, flush)
-        extras["nf4_quantize_gbs"] = quant_gbs
-        extras["nf4_dequantize_gbs"] = dequant_gbs
-        extras["nf4_hbm_frac"] = {"quantize": quant_gbs / peaks["hbm_gbs"], "dequantize": dequant_gbs / peaks["hbm_gbs"],
-                                  "peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]}
-        extras["c2_step"] = c2_step_timing(lib, synth, torch, dev, flush)
-        extras["adamw8"] = adamw8_timing(lib, synth, torch, dev, flush, peaks)
-        extras["lora_dropout"] = dropout_timing(lib, synth, torch, dev, flush)
-        extras["c5_forward"] = c5_forward_sweep(lib, synth, torch, dev, flush, peaks)
-        extras["c5_quantize_sweep"] = c5_quantize_sweep(lib, synth, torch, dev)
+        extras.update(nf4_extras)
+        # Each secondary measurement carries the SM clock it ran at.
+        for key, fn in (("c2_step", lambda: c2_step_timing(lib, synth, torch, dev, flush)),
+                        ("adamw8", lambda: adamw8_timing(lib, synth, torch, dev, flush, peaks)),
+                        ("lora_dropout", lambda: dropout_timing(lib, synth, torch, dev, flush)),
+                        ("c5_forward", lambda: c5_forward_sweep(lib, synth, torch, dev, flush, peaks)),
+                        ("c5_quantize_sweep", lambda: c5_quantize_sweep(lib, synth, torch, dev)),
+                        ("c1_graph", lambda: c1_graph_timing(lib, synth, torch, dev)),
+                        ("centered_dq", lambda: centered_cost(lib, synth, torch, dev, flush))):
+            res, clk = with_clocks(dev, fn)
+            res["clocks"] = clk
+            extras[key] = res
         extras["c5_quantize_sweep"]["hbm_frac"] = extras["c5_quantize_sweep"]["quantize_gbs"] / peaks["hbm_gbs"]
-        extras["c1_graph"] = c1_graph_timing(lib, synth, torch, dev)
-        extras["centered_dq"] = centered_cost(lib, synth, torch, dev, flush)
 
     value = world * fl / (ms * 1e-3) / 1e12
     cpu = None
