@@ -7,12 +7,13 @@
 //   dX:       dX^T tile [128 k x BN m] = W'[n, k]^T . dY[m, n]^T   (+ A^T . dU^T)
 //
 // The W side is the MMA's M = 128 dimension, tokens are its N = BN dimension,
-// so one dequantised element feeds BN tokens.  Warp roles (192 threads):
+// so one dequantised element feeds BN tokens.  Warp roles (64 + 32 DQW threads):
 //   warp 0      TMA producer (token tile + packed codes; LoRA operands)
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
-//   warps 2..5  dequantisers: one thread per 64-element NF4 block per stage,
-//               16 lookups of bf16 pairs written straight into the 128-byte
-//               swizzled operand layout; afterwards the epilogue (TMEM -> global)
+//   warp 1      TMEM owner and tcgen05.mma issuer (warp-uniform loop, elected lane)
+//   warps 2..   dequantisers, DQW / 4 groups of four taking stages in turn: one
+//               thread per 64-element NF4 block per stage, 16 lookups of bf16
+//               pairs written straight into the 128-byte swizzled operand
+//               layout; afterwards the epilogue (TMEM -> global)
 // The LoRA up-projection is appended to the contraction as extra K steps over
 // the interleaved hi/lo bf16 split of the fp32 down-projection, accumulated in
 // the same TMEM accumulator (no second pass over Y).  No TMA multicast.
@@ -110,10 +111,24 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     // Grouped forward: this tile's member reads its own columns of the hi/lo copy of s*U.
     const int uc0 = DX ? 0 : group_member(a.grp_end, a.groups, row0) * 2 * a.r;
     if (lane == 0) {
+      // The codes are the part of a stage that streams from DRAM (each is
+      // read by one CTA).  With one CTA per SM they are pulled into L2 ahead
+      // (stages kStages .. kPfAhead - 1 now, stage t + kPfAhead with stage
+      // t): 4-7% at 200-256 tokens.  With two CTAs per SM it measured
+      // neutral to 2% slower, and is off.
+      constexpr int kPfAhead = P::kCtasPerSm == 1 ? static_cast<int>(P::kStages) + 4 : 0;
+      auto prefetch_codes = [&](int t) {
+        if (kPfAhead == 0 || t >= nmain) return;
+        const int kt = kt0 + t;
+        if (!DX) tma_prefetch_l2_2d(&tm_codes, kt * 32, row0);
+        else tma_prefetch_l2_2d(&tm_codes, row0 / 2, kt * 64);
+      };
+      for (int t = P::kStages; t < kPfAhead; ++t) prefetch_codes(t);
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const uint32_t s = t % P::kStages, u = t / P::kStages;
         if (t >= static_cast<int>(P::kStages) && !mbar_wait(&empty[s], (u - 1) & 1, wc)) break;
+        prefetch_codes(t + kPfAhead);
         uint8_t* st = smem + s * P::kStage;
         if (t < nmain) {
           const int kt = kt0 + t;
@@ -247,12 +262,13 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       int64_t bdummy;
       const bool valid = block_of(t, bdummy);
       const uint32_t s = t % P::kStages, u = t / P::kStages;
-      // With two groups and an odd ring the slot's previous stage t - kStages
-      // belongs to the other group, and this group may get here before that
-      // stage's copy has landed; a parity wait on full[s] would then see the
-      // older phase as this one.  Waiting first for the MMA of stage
-      // t - kStages (which the refill needs anyway) rules that out.
-      if (kStep == 2 && (P::kStages & 1) && u > 0 && !mbar_wait_all(&empty[s], (u - 1) & 1, wc)) break;
+      // When the ring is not a multiple of the group count the slot's
+      // previous stage t - kStages belongs to another group, and this group
+      // may get here before that stage's copy has landed; a parity wait on
+      // full[s] would then see the older phase as this one.  Waiting first
+      // for the MMA of stage t - kStages (which the refill needs anyway)
+      // rules that out.
+      if (P::kStages % kStep != 0 && u > 0 && !mbar_wait_all(&empty[s], (u - 1) & 1, wc)) break;
       if (!mbar_wait_all(&full[s], u & 1, wc)) break;
       uint8_t* st = smem + s * P::kStage;
       const uint8_t* src;
@@ -284,16 +300,16 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
     grid_dependents_launch();
 
     // ------------------------------------------------------------ epilogue
-    // Warp w reads TMEM lane quadrant w % 4; with 8 dequant warps the two
-    // warps of a quadrant split the BN accumulator columns in halves.
+    // Warp w reads TMEM lane quadrant w % 4; the groups' warps of a quadrant
+    // split the BN accumulator columns between them.
     acc_ok = mbar_wait_warp(accf, 0, wc);
     if (acc_ok && gridDim.z == 1) {
       tc_fence_after();
       const int q = warp & 3;
       const int erow = q * 32 + lane;
-      const int cgrp = DQW == 4 ? 0 : (warp - 2) / 4;
-      constexpr int kAll = BN / 32;                                  // 32-column chunks
-      constexpr int kChunks = DQW == 4 ? kAll : (kAll + 1) / 2;      // per column group
+      const int cgrp = (warp - 2) / 4;
+      constexpr int kAll = BN / 32;                              // 32-column chunks
+      constexpr int kChunks = (kAll + DQW / 4 - 1) / (DQW / 4);  // per column group
       const int orow = row0 + erow;
       const bool rok = orow < a.rows;
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
@@ -347,9 +363,9 @@ __global__ void __launch_bounds__(64 + 32 * DQW, FusedPlan<BN>::kCtasPerSm)
       tc_fence_after();
       const int q = warp & 3;
       const int erow = q * 32 + lane;
-      const int cgrp = DQW == 4 ? 0 : (warp - 2) / 4;
+      const int cgrp = (warp - 2) / 4;
       constexpr int kAll = BN / 32;
-      constexpr int kChunks = DQW == 4 ? kAll : (kAll + 1) / 2;
+      constexpr int kChunks = (kAll + DQW / 4 - 1) / (DQW / 4);
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
       const int own = erow / R;
       const uint32_t dst0 = dsmem_addr(smem, static_cast<uint32_t>(own)) + static_cast<uint32_t>(z) * slot_bytes +
@@ -773,8 +789,9 @@ static cudaError_t launch_fused_impl(const CUtensorMap& m0, const CUtensorMap& m
 // stages) measured 3-6% faster than four at 64 to 256 tokens on 22016 x 8192
 // and 8192 x 22016 weights (200 tokens: 196 against 208 us); each stage's
 // dequantisation is a chain of dependent byte permutes, and two groups give
-// each SM sub-partition two of them to interleave.  QLORA_DEQUANT_WARPS=4
-// selects four.
+// each SM sub-partition two of them to interleave (three groups of four, with
+// one CTA per SM, measured within 2% of two).  QLORA_DEQUANT_WARPS=4 selects
+// four.
 static int dequant_warps(int bn) {
   static int forced = [] {
     const char* e = getenv("QLORA_DEQUANT_WARPS");
