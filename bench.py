@@ -911,8 +911,10 @@ def run_ours(args, rank, world):
     if rank == 0 and not args.no_sweep and grouped:
         # Grouped against per-linear calls, timed in alternation (rounds of a
         # few steps each) so that both see the same clocks and power state.
-        flat = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=False)
-        again = LayerStep(lib, synth, torch, dev, M, rank, world, grouped=True)
+        # Rank 0 alone runs this: its layers are single-GPU ones (world 1, no
+        # gradient all-reduce that the other ranks would never join).
+        flat = LayerStep(lib, synth, torch, dev, M, rank, 1, grouped=False)
+        again = LayerStep(lib, synth, torch, dev, M, rank, 1, grouped=True)
         for _ in range(3):
             flat.step()
             again.step()
