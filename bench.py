@@ -434,16 +434,16 @@ def c2_step_timing(lib, synth, torch, dev, flush, reps=20):
             "ms": ms, "tflops": flops_fwd_bwd(M, N, K, r) / (ms * 1e-3) / 1e12}
 
 
-def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
+def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=7):
     """Forward of the 65B-shaped 8192<->22016 linears over M in {1,16,128,2048,16384}.
 
     Per case: algorithmic bytes 0.5159 N K + 2 M K + 2 M N + 2 r (K + N) and
-    FLOPs 2 M N K + 2 M K r + 2 M N r, over the mean device time of the
-    forward call (L2 flushed before each run).  kernels_ms: per-kernel event
-    times averaged over `reps` further calls with every kernel bracketed by
-    events (the brackets serialise the kernels, which otherwise overlap
-    through programmatic dependent launch); ms_bracketed is the outer time of
-    those same calls.
+    FLOPs 2 M N K + 2 M K r + 2 M N r, over the median device time of the
+    forward call (L2 flushed before each call).  Plain calls alternate with
+    calls that bracket every kernel with events (the brackets serialise the
+    kernels, which otherwise overlap through programmatic dependent launch),
+    so both see the same clocks: kernels_ms is the per-kernel median over the
+    bracketed calls and ms_bracketed their median outer time.
     """
     out = {}
     r, s = 64, 0.25
@@ -463,23 +463,39 @@ def c5_forward_sweep(lib, synth, torch, dev, flush, peaks, reps=5):
             def call():
                 lib.qlora_linear_fwd(X, W, A, B, s, Y=Y, U=U, ws=ws)
 
+            def timed():
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                call()
+                e1.record()
+                e1.synchronize()
+                return e0.elapsed_time(e1)
+
             for _ in range(3):
                 call()
-            ts = time_steps(torch, call, torch.cuda.current_stream(), reps, flush)
-            ms = float(np.mean(ts))
-            lib.profile_enable(True)
-            tb = time_steps(torch, call, torch.cuda.current_stream(), reps, flush)
-            lib.profile_enable(False)
-            kern = {}
-            for name, kms in lib.profile_collect():
-                kern[name] = kern.get(name, 0.0) + kms / reps
+            torch.cuda.synchronize()
+            lib.profile_collect()
+            ts, tb, per = [], [], {}
+            for _ in range(reps):
+                ts.append(timed())
+                lib.profile_enable(True)
+                tb.append(timed())
+                lib.profile_enable(False)
+                this = {}
+                for name, kms in lib.profile_collect():
+                    this[name] = this.get(name, 0.0) + kms
+                for name, kms in this.items():
+                    per.setdefault(name, []).append(kms)
+            ms = float(statistics.median(ts))
+            kern = {k: float(statistics.median(v)) for k, v in per.items()}
             byts = 0.51587 * N * K + 2 * M * K + 2 * M * N + 2 * r * (K + N)
             fl = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
             out[f"{lin.name}_{N}x{K}_M{M}"] = {
                 "ms": round(ms, 5), "tflops": round(fl / ms / 1e9, 2), "gbs": round(byts / ms / 1e6, 1),
                 "hbm_frac": round(byts / ms / 1e6 / peaks["hbm_gbs"], 4),
                 "tensor_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4),
-                "ms_bracketed": round(float(np.mean(tb)), 5),
+                "ms_bracketed": round(float(statistics.median(tb)), 5),
                 "kernels_ms": {k: round(v, 5) for k, v in kern.items()}}
             del X, Y, U, ws
         del W, A, B
