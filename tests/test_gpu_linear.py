@@ -80,6 +80,11 @@ def test_c1_full_f32_outputs():
     (300, 192, 320, 64), (128, 64, 64, 16), (257, 384, 576, 64), (33, 64, 1024, 32),
     (700, 320, 448, 48), (1000, 192, 576, 16), (513, 128, 128, 64), (2000, 384, 192, 32),
     (700, 256, 512, 48), (1300, 512, 256, 16), (600, 768, 1024, 64),
+    # extremes of the shape rules: K = 64 (one block per row: two 32-deep
+    # stages in the CTA pair, one 64-deep stage in the mid-size kernel),
+    # N = 64 (a single half-filled W tile), an odd large M
+    (1024, 256, 64, 16), (257, 256, 64, 64), (100, 512, 64, 32), (300, 64, 4096, 64),
+    (4097, 128, 128, 16),
 ])
 def test_ragged_shapes(M, N, K, r):
     _check_full(M, N, K, r, 16.0 / r, M + N + K, out_dtype=1)
