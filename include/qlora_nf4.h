@@ -364,7 +364,9 @@ QLORA_API qlora_status qlora_selftest_timeout(int32_t* d_status, int64_t limit_n
  * smaller ones its fixed costs dominate).  0 selects the few-token kernel
  * for every M <= 16; INT64_MAX never.  Negative values count as 0.
  * Process-wide and thread-safe; it changes the workspace sizes of later
- * queries, so set it before querying.  Returns the previous value.
+ * queries, so set it before querying (a call given a workspace smaller than
+ * the current setting needs returns QLORA_ERR_WORKSPACE before anything is
+ * enqueued).  Returns the previous value.
  */
 QLORA_API int64_t qlora_set_few_token_threshold(int64_t min_weight_elems);
 
