@@ -204,12 +204,15 @@ qlora_status check_device() {
   return arch_ok[dev] == 1 ? QLORA_OK : QLORA_ERR_ARCH;
 }
 
+constexpr int32_t kChunkRank = 64;  // largest rank the rank-r kernels take in one CTA
+constexpr int32_t kMaxRank = 256;
+
 qlora_status check_linear_shape(int64_t M, const nf4_weight& W, int32_t r) {
   const int64_t N = W.n_out, K = W.k_in;
   if (M < 0 || M >= (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
   if (N < 64 || K < 64 || N % 64 != 0 || K % 64 != 0) return QLORA_ERR_SHAPE;
   if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N * K >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
-  if (r < 16 || r > 64 || r % 16 != 0) return QLORA_ERR_SHAPE;
+  if (r < 16 || r % 16 != 0 || r > kMaxRank || (r > kChunkRank && r % kChunkRank != 0)) return QLORA_ERR_SHAPE;
   return QLORA_OK;
 }
 
@@ -444,7 +447,7 @@ bool few_token_path(int64_t M, int64_t N, int64_t K) {
 }
 
 FwdPlan plan_fwd(int64_t M, int64_t N, int64_t K, int32_t r, int G) {
-  if (few_token_path(M, N, K)) return plan_fwd_low(M, N, K, r, G);
+  if (r <= kChunkRank && few_token_path(M, N, K)) return plan_fwd_low(M, N, K, r, G);
   FwdPlan p{};
   const int64_t kst = K / 64;
   split_plan(cdiv(M, 128) * G, kst, 4, 2 * kSms, p.s_down, p.per_down);
@@ -519,6 +522,11 @@ Group single_group(int64_t N) {
   g.n_max = N;
   return g;
 }
+
+// A single linear of rank r > 64 runs its rank-r products as r / 64 chunks
+// of rank 64 (the layout of a group's members: U [M, r], the hi/lo of s U
+// [M, 2 r], dA [r, K]); the GEMMs take the whole rank in their adapter stages.
+bool rank_chunks(const Group& g, int32_t r) { return g.G == 1 && r > kChunkRank; }
 
 // Members 1..4, each a multiple of 128 rows (tiles never straddle members),
 // summing to the stacked weight's rows.
@@ -749,11 +757,15 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   // bf16 hi/lo of s*U; the G CTAs of a token tile read the same X rows.
   CUtensorMap mx_down, ma_down;
   if (!map_bf16(&mx_down, Xa, M, K, 64, 128) || !map_bf16(&ma_down, A, ra, K, 64, 64)) return QLORA_ERR_CUDA;
+  // A rank above 64 runs as r / 64 chunks of rank 64: the G CTAs of a token
+  // tile are then the chunks instead of the members.
+  const bool chunks = rank_chunks(grp, r);
+  const int Gd = chunks ? r / kChunkRank : G;
   SkinnyArgs sa{};
   sa.M = static_cast<int>(M);
   sa.N = static_cast<int>(N);
   sa.K = static_cast<int>(K);
-  sa.r = r;
+  sa.r = chunks ? kChunkRank : r;
   sa.stages_total = static_cast<int>(K / 64);
   sa.stages_per_split = p.per_down;
   sa.s = s;
@@ -761,6 +773,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   sa.out_cat = ucat;
   sa.status = d_status;
   fill_group(grp, &sa);
+  sa.groups = Gd;
   uint32_t* tile_count = reinterpret_cast<uint32_t*>(wsb + p.off_cnt);
   if (p.low) {  // the few-token kernel's tile counters start at zero
     sa.zero = tile_count;
@@ -769,7 +782,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   {
     ProfScope ps(kKDown, cs);
     if (qlora_status st = from_cuda(launch_skinny(kSkDown, mx_down, ma_down, sa,
-                                                  static_cast<int>(cdiv(M, 128)) * G, p.s_down, cs)))
+                                                  static_cast<int>(cdiv(M, 128)) * Gd, p.s_down, cs)))
       return st;
   }
 
@@ -810,7 +823,7 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   // Y = X W'^T + (sU) B^T, W' dequantised inside the GEMM.
   if (M > kWideM) {
     const bool pair = use_pair(N) && group_pairs(grp);
-    const bool tmem_a = pair && use_tmem_a();
+    const bool tmem_a = pair && use_tmem_a() && r <= kChunkRank;  // its adapter buffers hold r <= 64
     const uint32_t tok_box = tmem_a ? static_cast<uint32_t>(pair_fwd_tokens(tmem_a_slots()) / 4) : (pair ? 128 : 256);
     CUtensorMap wx, wc, wu, wb;
     if (!map_bf16(&wx, X, M, K, 32, tok_box, 64) || !map_u8(&wc, W.codes, N, K / 2, 16, 128) ||
@@ -881,6 +894,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
                                     void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
                                     int32_t* d_status, void* stream, const DropoutArgs* drop) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (drop && r > kChunkRank) return QLORA_ERR_SHAPE;  // the dropout dX pass holds r <= 64
   if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
   if (!dY || !X || !U || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
@@ -906,13 +920,19 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   const int gemm_r = drop ? 0 : ra;                               // adapter stages in the GEMM (all members)
   const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
 
+  // A rank above 64: r / 64 chunks of rank 64 (DU and DA: G CTAs per tile;
+  // DB: G CTAs per row tile, each writing its columns of dB).
+  const bool chunks = rank_chunks(grp, r);
+  const int Gs = chunks ? r / kChunkRank : G;
   SkinnyArgs sa{};
   sa.M = Mi;
   sa.N = Ni;
   sa.K = Ki;
-  sa.r = r;
+  sa.r = chunks ? kChunkRank : r;
   sa.status = d_status;
   fill_group(grp, &sa);
+  sa.groups = Gs;
+  sa.chunks = chunks ? 1 : 0;
 
   // dU = s dY B per member (contraction over the member's outputs, split over
   // a cluster) -> bf16 hi/lo, and the bf16 hi/lo of s*U for dB from the saved U.
@@ -928,7 +948,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   {
     ProfScope ps(kKDU, cs);
     if (qlora_status st =
-            from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)) * G, p.s_du, cs)))
+            from_cuda(launch_skinny(kSkDU, mdy128, mbl, sa, static_cast<int>(cdiv(M, 128)) * Gs, p.s_du, cs)))
       return st;
   }
 
@@ -1015,7 +1035,8 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   {
     ProfScope ps(kKDB, side);
     if (qlora_status st =
-            from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)), p.s_db, side)))
+            from_cuda(launch_skinny(kSkDB, mdy64, msu, sa, static_cast<int>(cdiv(N, 128)) * (chunks ? Gs : 1), p.s_db,
+                                    side)))
       return st;
   }
 
@@ -1031,7 +1052,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
     da.out_cat = nullptr;
     ProfScope ps(kKDA, side);
     if (qlora_status st = from_cuda(
-            launch_skinny(kSkDA, mduc, mx, da, static_cast<int>(cdiv(K, 128)) * G, p.s_da, side)))
+            launch_skinny(kSkDA, mduc, mx, da, static_cast<int>(cdiv(K, 128)) * Gs, p.s_da, side)))
       return st;
   }
 
@@ -1061,6 +1082,7 @@ qlora_status qlora_group_fwd(const uint16_t* X, int64_t M, nf4_weight W, int32_t
                              const uint16_t* A, const uint16_t* B, int32_t r, float s, void* Y, int32_t y_dtype,
                              float* U_out, void* ws, size_t ws_bytes, int32_t* d_status, void* stream) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (members > 1 && r > kChunkRank) return QLORA_ERR_SHAPE;  // members' ranks are at most 64
   Group grp;
   if (qlora_status st = make_group(members, n_member, W.n_out, &grp)) return st;
   return linear_fwd_impl(X, X, M, W, grp, A, B, r, s, Y, y_dtype, U_out, ws, ws_bytes, d_status, stream);
@@ -1071,6 +1093,7 @@ qlora_status qlora_group_bwd(const uint16_t* dY, const uint16_t* X, const float*
                              int32_t r, float s, void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws,
                              size_t ws_bytes, int32_t* d_status, void* stream) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (members > 1 && r > kChunkRank) return QLORA_ERR_SHAPE;  // members' ranks are at most 64
   Group grp;
   if (qlora_status st = make_group(members, n_member, W.n_out, &grp)) return st;
   return linear_bwd_impl(dY, X, U, M, W, grp, A, B, r, s, dX, dx_dtype, dA, dB, ws, ws_bytes, d_status, stream,
@@ -1112,6 +1135,7 @@ qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W
   DropoutArgs d{};
   if (!dropout_args(p, seed, &d)) return QLORA_ERR_SHAPE;
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
+  if (r > kChunkRank) return QLORA_ERR_SHAPE;  // the dropout dX pass holds r <= 64
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
   if (!X || !X_drop || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   // 128 rows are the hi/lo columns of dU and its tiles walk K in 128s.  The
   // member g: DOWN, DU and DA have G CTAs per tile; DB's rows lie in one member.
   const int G = a.groups;
-  const bool per_tile = MODE != kSkDB;
+  const bool per_tile = MODE != kSkDB || a.chunks;
   const int tile = per_tile ? static_cast<int>(blockIdx.x) / G : static_cast<int>(blockIdx.x);
   const int row0 = tile * 128;
   int g = per_tile ? static_cast<int>(blockIdx.x) % G : 0;
@@ -81,10 +81,10 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     for (int i = 1; i < G; ++i) g += row0 >= a.grp_n[i] ? 1 : 0;
   const int ra = G * a.r;                // U row stride
   const int ucol = g * 2 * a.r;          // this member's first hi/lo column
-  const int nbase = a.grp_n[g];          // DU: this member's first output feature
+  const int nbase = a.chunks ? 0 : a.grp_n[g];  // DU: this member's first output feature
   const int z = blockIdx.y;
   const int st0 = z * a.stages_per_split;
-  const int st_all = MODE == kSkDU ? (a.grp_n[g + 1] - nbase) / 64 : a.stages_total;
+  const int st_all = MODE == kSkDU && !a.chunks ? (a.grp_n[g + 1] - nbase) / 64 : a.stages_total;
   const int T = min(st_all, st0 + a.stages_per_split) - st0;  // <= 0: no MMA, the partial is zero
   const int nc = (2 * a.r > 64) ? 128 : 64;  // DB: width of the sU operand
 
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         } else if (MODE == kSkDU) {
           mbar_arrive_expect_tx(&full[s], 16384 + 8192);
           tma_load_2d(sa, &tmA, &full[s], nbase + kt * 64, row0);  // this member's columns of dY
-          tma_load_2d(sb, &tmB, &full[s], 0, nbase + kt * 64);     // and rows of B
+          tma_load_2d(sb, &tmB, &full[s], a.chunks ? g * a.r : 0, nbase + kt * 64);  // and rows of B
         } else if (MODE == kSkDB) {
           const bool a2 = row0 + 64 < a.N;
           mbar_arrive_expect_tx(&full[s], 8192u * ((a2 ? 2 : 1) + nc / 64));
@@ -291,7 +291,10 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         }
       } else if (MODE == kSkDB) {
         const int n = row0 + row;
-        if (n < a.N) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(n) * a.r + col) = acc;
+        if (n < a.N) {
+          float* o = a.chunks ? a.out_f32 + static_cast<int64_t>(n) * ra + g * a.r : a.out_f32 + static_cast<int64_t>(n) * a.r;
+          *reinterpret_cast<float4*>(o + col) = acc;
+        }
       } else {
         const int k = row0 + col;
         if (k < a.K) *reinterpret_cast<float4*>(a.out_f32 + static_cast<int64_t>(g * a.r + row) * a.K + k) = acc;

@@ -86,7 +86,12 @@ def test_fwd_argument_errors():
     assert _fwd(U=None) == NULL
     assert _fwd(W=_w(k=4096 + 32)) == SHAPE          # K % 64 != 0
     assert _fwd(W=_w(n=4096 + 16)) == SHAPE          # N % 64 != 0
-    assert _fwd(r=8) == SHAPE and _fwd(r=24) == SHAPE and _fwd(r=128) == SHAPE
+    assert _fwd(r=8) == SHAPE and _fwd(r=24) == SHAPE and _fwd(r=320) == SHAPE
+    # above 64 the rank must be a multiple of 64 (chunks of 64)
+    assert _fwd(r=80) == SHAPE and _fwd(r=144) == SHAPE and _fwd(r=272) == SHAPE
+    for r in (128, 192, 256):
+        assert _fwd(M=0, r=r, X=None, Y=None, U=None, ws=None) == OK   # accepted: no-op
+        assert _bwd(M=0, r=r, dY=None) == OK
     assert _fwd(M=-1) == SHAPE
     assert _fwd(X=FAKE + 8) == ALIGN
     assert _fwd(W=_w(c8=FAKE + 4)) == ALIGN
@@ -138,6 +143,13 @@ def test_group_argument_errors():
     assert fwd(3, members(4096, 4096, 4096), M=0) == OK
     assert b(FAKE, FAKE, FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 8, 0.25, FAKE, 0, FAKE, FAKE,
              FAKE, 1 << 40, None, None) == SHAPE                # r = 8
+    # members of a real group take r <= 64; one member is a single linear
+    assert b(FAKE, FAKE, FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 128, 0.25, FAKE, 0, FAKE, FAKE,
+             FAKE, 1 << 40, None, None) == SHAPE
+    assert f(FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 128, 0.25, FAKE, 0, FAKE, FAKE, 1 << 40,
+             None, None) == SHAPE
+    assert f(FAKE, 0, _w(n=8192), 1, members(8192), FAKE, FAKE, 128, 0.25, FAKE, 0, FAKE, FAKE, 1 << 40,
+             None, None) == OK
     assert b(FAKE, FAKE, FAKE, 64, _w(n=8192), 2, members(4096, 4096), FAKE, FAKE, 64, 0.25, FAKE, 0, FAKE, FAKE,
              FAKE, 16, None, None) == WS
     assert q.qlora_group_fwd_workspace_size(4096, 12288, 4096, 1, 64) == q.qlora_fwd_workspace_size(4096, 12288,
@@ -227,6 +239,11 @@ def test_dropout_rejects_bad_probability_before_touching_a_device():
              1 << 20, None, None) == SHAPE
     assert f(P(256), 64, w, P(256), P(256), 16, 1.0, 0.1, 7, None, P(256), 0, P(256), P(256), 1 << 20,
              None, None) == NULL
+    # LoRA dropout takes r <= 64 (its dX pass holds one 64-wide rank block)
+    assert f(P(256), 64, w, P(256), P(256), 128, 1.0, 0.1, 7, P(256), P(256), 0, P(256), P(256), 1 << 20,
+             None, None) == SHAPE
+    assert g(P(256), P(256), P(256), 64, w, P(256), P(256), 128, 1.0, 0.1, 7, P(256), 0, P(256), P(256), P(256),
+             1 << 20, None, None) == SHAPE
     assert q.qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) == \
         q.qlora_bwd_workspace_size(4096, 4096, 4096, 64) + 4096 * 4096 * 4
 

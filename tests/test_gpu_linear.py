@@ -92,6 +92,21 @@ def test_ragged_shapes(M, N, K, r):
 
 
 @pytest.mark.parametrize("M,N,K,r", [
+    (100, 512, 384, 128),     # mid-size forward and dX
+    (12, 4096, 16384, 128),   # few tokens on a 2^26 weight: the mid-size kernel (the few-token one takes r <= 64)
+    (700, 512, 768, 256),     # CTA-pair forward and dX (W rows and K multiples of 256)
+    (600, 320, 448, 192),     # the 512-token single-CTA kernels both ways
+    (257, 256, 64, 256),      # K = 64 with the widest rank
+])
+def test_ranks_above_64(M, N, K, r):
+    """Ranks 128..256 run U, dU, dB and dA as chunks of 64 (the layout of a
+    group's members) and the whole rank in the GEMMs' adapter stages: the
+    same tolerances against the oracle, fp32 and bf16 outputs."""
+    _check_full(M, N, K, r, 16.0 / r, 11 * M + N + K + r, out_dtype=1)
+    _check_full(M, N, K, r, 16.0 / r, 11 * M + N + K + r, out_dtype=0)
+
+
+@pytest.mark.parametrize("M,N,K,r", [
     (1, 64, 64, 16), (3, 320, 832, 48), (8, 448, 1344, 64), (9, 128, 64, 16),
     (12, 1088, 2112, 32), (16, 960, 4160, 64), (5, 4096, 256, 16), (7, 2048, 8192, 64),
     (11, 1024, 16384, 48), (16, 4096, 4096, 32), (17, 320, 832, 48), (24, 1088, 2112, 64),
