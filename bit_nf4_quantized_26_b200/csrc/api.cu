@@ -212,7 +212,7 @@ qlora_status check_linear_shape(int64_t M, const nf4_weight& W, int32_t r) {
   if (M < 0 || M >= (int64_t(1) << 31)) return QLORA_ERR_SHAPE;
   if (N < 64 || K < 64 || N % 64 != 0 || K % 64 != 0) return QLORA_ERR_SHAPE;
   if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N * K >= (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
-  if (r < 16 || r % 16 != 0 || r > kMaxRank || (r > kChunkRank && r % kChunkRank != 0)) return QLORA_ERR_SHAPE;
+  if (r < 16 || r % 16 != 0 || r > kMaxRank) return QLORA_ERR_SHAPE;
   return QLORA_OK;
 }
 
@@ -523,9 +523,10 @@ Group single_group(int64_t N) {
   return g;
 }
 
-// A single linear of rank r > 64 runs its rank-r products as r / 64 chunks
-// of rank 64 (the layout of a group's members: U [M, r], the hi/lo of s U
-// [M, 2 r], dA [r, K]); the GEMMs take the whole rank in their adapter stages.
+// A single linear of rank r > 64 runs its rank-r products as ceil(r / 64)
+// chunks of rank 64 (the last one r - 64 (chunks - 1) wide), laid out as a
+// group's members: U [M, r], the hi/lo of s U [M, 2 r], dA [r, K].  The GEMMs
+// take the whole rank in their adapter stages.
 bool rank_chunks(const Group& g, int32_t r) { return g.G == 1 && r > kChunkRank; }
 
 // Members 1..4, each a multiple of 128 rows (tiles never straddle members),
@@ -757,10 +758,10 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   // bf16 hi/lo of s*U; the G CTAs of a token tile read the same X rows.
   CUtensorMap mx_down, ma_down;
   if (!map_bf16(&mx_down, Xa, M, K, 64, 128) || !map_bf16(&ma_down, A, ra, K, 64, 64)) return QLORA_ERR_CUDA;
-  // A rank above 64 runs as r / 64 chunks of rank 64: the G CTAs of a token
-  // tile are then the chunks instead of the members.
+  // A rank above 64 runs as ceil(r / 64) chunks of rank 64: the G CTAs of a
+  // token tile are then the chunks instead of the members.
   const bool chunks = rank_chunks(grp, r);
-  const int Gd = chunks ? r / kChunkRank : G;
+  const int Gd = chunks ? (r + kChunkRank - 1) / kChunkRank : G;
   SkinnyArgs sa{};
   sa.M = static_cast<int>(M);
   sa.N = static_cast<int>(N);
@@ -774,6 +775,8 @@ static qlora_status linear_fwd_impl(const uint16_t* X, const uint16_t* Xa, int64
   sa.status = d_status;
   fill_group(grp, &sa);
   sa.groups = Gd;
+  sa.chunks = chunks ? 1 : 0;
+  sa.r_total = r;
   uint32_t* tile_count = reinterpret_cast<uint32_t*>(wsb + p.off_cnt);
   if (p.low) {  // the few-token kernel's tile counters start at zero
     sa.zero = tile_count;
@@ -920,10 +923,10 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   const int gemm_r = drop ? 0 : ra;                               // adapter stages in the GEMM (all members)
   const int Mi = static_cast<int>(M), Ni = static_cast<int>(N), Ki = static_cast<int>(K);
 
-  // A rank above 64: r / 64 chunks of rank 64 (DU and DA: G CTAs per tile;
-  // DB: G CTAs per row tile, each writing its columns of dB).
+  // A rank above 64: ceil(r / 64) chunks of rank 64 (DU and DA: G CTAs per
+  // tile; DB: G CTAs per row tile, each writing its columns of dB).
   const bool chunks = rank_chunks(grp, r);
-  const int Gs = chunks ? r / kChunkRank : G;
+  const int Gs = chunks ? (r + kChunkRank - 1) / kChunkRank : G;
   SkinnyArgs sa{};
   sa.M = Mi;
   sa.N = Ni;
@@ -933,6 +936,7 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
   fill_group(grp, &sa);
   sa.groups = Gs;
   sa.chunks = chunks ? 1 : 0;
+  sa.r_total = r;
 
   // dU = s dY B per member (contraction over the member's outputs, split over
   // a cluster) -> bf16 hi/lo, and the bf16 hi/lo of s*U for dB from the saved U.

@@ -104,10 +104,12 @@ struct SkinnyArgs {
   int grp_n[5];         // member offsets along N (grp_n[0] = 0, grp_n[G] = N)
   uint32_t* zero;       // DOWN: words cleared by the first CTA (the few-token forward's tile counters)
   int zero_count;
-  // 1: the "members" are rank chunks of one linear of rank G r (r = 64 each):
-  // DU reads all N outputs of dY and columns g r .. g r + r - 1 of B [N, G r];
-  // DB runs G CTAs per row tile and writes columns g r .. of dB [N, G r].
+  // 1: the "members" are rank chunks of one linear of rank r_total: chunk g
+  // holds ranks g r .. g r + rw - 1, rw = min(r, r_total - g r) (r = 64);
+  // DU reads all N outputs of dY and those columns of B [N, r_total]; DB runs
+  // G CTAs per row tile and writes those columns of dB [N, r_total].
   int chunks;
+  int r_total;
 };
 
 // One CTA waits on an mbarrier nothing completes, with a `limit_ns` bound,

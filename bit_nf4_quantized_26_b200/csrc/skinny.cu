@@ -79,14 +79,15 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   int g = per_tile ? static_cast<int>(blockIdx.x) % G : 0;
   if (!per_tile)
     for (int i = 1; i < G; ++i) g += row0 >= a.grp_n[i] ? 1 : 0;
-  const int ra = G * a.r;                // U row stride
-  const int ucol = g * 2 * a.r;          // this member's first hi/lo column
+  const int ra = a.chunks ? a.r_total : G * a.r;  // U row stride
+  const int ucol = g * 2 * a.r;                   // this member's first hi/lo column
+  const int rw = a.chunks ? min(a.r, a.r_total - g * a.r) : a.r;  // this member's rank
   const int nbase = a.chunks ? 0 : a.grp_n[g];  // DU: this member's first output feature
   const int z = blockIdx.y;
   const int st0 = z * a.stages_per_split;
   const int st_all = MODE == kSkDU && !a.chunks ? (a.grp_n[g + 1] - nbase) / 64 : a.stages_total;
   const int T = min(st_all, st0 + a.stages_per_split) - st0;  // <= 0: no MMA, the partial is zero
-  const int nc = (2 * a.r > 64) ? 128 : 64;  // DB: width of the sU operand
+  const int nc = (2 * rw > 64) ? 128 : 64;  // DB: width of the sU operand
 
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < P::kStages; ++s) {
@@ -186,14 +187,14 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
       const uint32_t tq = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
       if (MODE == kSkDown || MODE == kSkDU) {
         // rows = tokens, columns j < r
-        for (int cb = 0; cb < (a.r + 31) / 32; ++cb) {
+        for (int cb = 0; cb < (rw + 31) / 32; ++cb) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
           tmem_ld_wait();
           if (T <= 0)
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           float* dst = part + rl * P::kLdRows + cb * 32;
-          const int nv = min(32, a.r - cb * 32);
+          const int nv = min(32, rw - cb * 32);
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             if (j < nv)
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         }
       } else if (MODE == kSkDB) {
         // rows = output features, columns = hi/lo pairs of j -> combined
-        for (int jb = 0; jb < a.r / 16; ++jb) {
+        for (int jb = 0; jb < rw / 16; ++jb) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + jb * 32, v);
           tmem_ld_wait();
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
         }
       } else {  // DA: TMEM rows c = 32q + lane; hi row (lane < 16) plus lo row (lane + 16)
         const int j = 16 * q + lane;
-        const bool jok = lane < 16 && j < a.r;
+        const bool jok = lane < 16 && j < rw;
         for (int cb = 0; cb < 4; ++cb) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tq + cb * 32, v);
@@ -253,8 +254,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
     const uint32_t self = cluster_ctarank();
     auto holder = [&](uint32_t z) { return S == 1 ? self : z; };
     const bool by_rows = (MODE != kSkDA);
-    const int R = by_rows ? 128 : a.r;                 // rows of the partial tile
-    const int C = by_rows ? a.r : 128;                 // columns
+    const int R = by_rows ? 128 : rw;                  // rows of the partial tile
+    const int C = by_rows ? rw : 128;                  // columns
     const int ld = by_rows ? P::kLdRows : P::kLdCols;  // floats per smem row
     const int rows_per = (R + static_cast<int>(S) - 1) / static_cast<int>(S);
     const int r0 = static_cast<int>(rank) * rows_per;

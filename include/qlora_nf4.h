@@ -175,10 +175,9 @@ QLORA_API qlora_status nf4_dequantize_centered(const uint8_t* codes, const uint8
  *  ws     device workspace of at least qlora_fwd_workspace_size(M, N, K, r) bytes
  *
  * Constraints: M >= 0 (0 = no-op), K % 64 == 0, N % 64 == 0, K >= 64,
- * N >= 64, M < 2^31, N*K < 2^40; r in {16, 32, 48, 64, 128, 192, 256}
- * (r % 16 == 0 up to 64, above that a multiple of 64: ranks above 64 run
- * their rank-r products as chunks of 64).  The grouped calls with more than
- * one member and the LoRA dropout calls take r <= 64.
+ * N >= 64, M < 2^31, N*K < 2^40, r % 16 == 0 and 16 <= r <= 256 (ranks
+ * above 64 run their rank-r products as chunks of 64).  The grouped calls
+ * with more than one member and the LoRA dropout calls take r <= 64.
  * Accuracy: fp32 accumulation over exact bf16 inputs; relative Frobenius
  * error of Y within 2e-3 of the fp64 product on the same dequantised weights.
  */

@@ -86,10 +86,8 @@ def test_fwd_argument_errors():
     assert _fwd(U=None) == NULL
     assert _fwd(W=_w(k=4096 + 32)) == SHAPE          # K % 64 != 0
     assert _fwd(W=_w(n=4096 + 16)) == SHAPE          # N % 64 != 0
-    assert _fwd(r=8) == SHAPE and _fwd(r=24) == SHAPE and _fwd(r=320) == SHAPE
-    # above 64 the rank must be a multiple of 64 (chunks of 64)
-    assert _fwd(r=80) == SHAPE and _fwd(r=144) == SHAPE and _fwd(r=272) == SHAPE
-    for r in (128, 192, 256):
+    assert _fwd(r=8) == SHAPE and _fwd(r=24) == SHAPE and _fwd(r=320) == SHAPE and _fwd(r=272) == SHAPE
+    for r in (80, 128, 144, 192, 240, 256):
         assert _fwd(M=0, r=r, X=None, Y=None, U=None, ws=None) == OK   # accepted: no-op
         assert _bwd(M=0, r=r, dY=None) == OK
     assert _fwd(M=-1) == SHAPE

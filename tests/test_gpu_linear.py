@@ -97,11 +97,15 @@ def test_ragged_shapes(M, N, K, r):
     (700, 512, 768, 256),     # CTA-pair forward and dX (W rows and K multiples of 256)
     (600, 320, 448, 192),     # the 512-token single-CTA kernels both ways
     (257, 256, 64, 256),      # K = 64 with the widest rank
+    (80, 384, 320, 80),       # a last chunk of 16 (mid-size kernels)
+    (900, 768, 512, 160),     # a last chunk of 32 (CTA pair both ways)
+    (520, 448, 704, 240),     # a last chunk of 48 (the 512-token single-CTA kernels)
 ])
 def test_ranks_above_64(M, N, K, r):
-    """Ranks 128..256 run U, dU, dB and dA as chunks of 64 (the layout of a
-    group's members) and the whole rank in the GEMMs' adapter stages: the
-    same tolerances against the oracle, fp32 and bf16 outputs."""
+    """Ranks above 64 run U, dU, dB and dA as chunks of 64 (the layout of a
+    group's members; the last chunk r - 64 (chunks - 1) wide) and the whole
+    rank in the GEMMs' adapter stages: the same tolerances against the
+    oracle, fp32 and bf16 outputs."""
     _check_full(M, N, K, r, 16.0 / r, 11 * M + N + K + r, out_dtype=1)
     _check_full(M, N, K, r, 16.0 / r, 11 * M + N + K + r, out_dtype=0)
 
