@@ -16,7 +16,9 @@
 // result is deterministic and needs no partial buffers in global memory and
 // no extra launch.  The fp32 operands (sU, dU) enter the tensor core as a
 // bf16 hi/lo pair in the interleaved "hi/lo per 16" column layout: column c
-// holds part (c/16)%2 (0 = hi, 1 = lo) of j = 16*(c/32) + c%16.
+// holds part (c/16)%2 (0 = hi, 1 = lo) of j = 16*(c/32) + c%16.  A single
+// linear of rank above 64 runs as rank chunks of 64 in the members' place
+// (SkinnyArgs::chunks), the same layout.
 #include "kernels.h"
 
 namespace qnf4 {
@@ -71,7 +73,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Tile origin: DOWN/DU rows are tokens, DB rows are output features, DA's
   // 128 rows are the hi/lo columns of dU and its tiles walk K in 128s.  The
-  // member g: DOWN, DU and DA have G CTAs per tile; DB's rows lie in one member.
+  // member g: DOWN, DU and DA have G CTAs per tile; DB's rows lie in one member
+  // (rank chunks of one linear: DB too has G CTAs per row tile).
   const int G = a.groups;
   const bool per_tile = MODE != kSkDB || a.chunks;
   const int tile = per_tile ? static_cast<int>(blockIdx.x) / G : static_cast<int>(blockIdx.x);
@@ -293,7 +296,8 @@ __global__ void __launch_bounds__(192, SkPlan<MODE>::kCtasPerSm)
       } else if (MODE == kSkDB) {
         const int n = row0 + row;
         if (n < a.N) {
-          float* o = a.chunks ? a.out_f32 + static_cast<int64_t>(n) * ra + g * a.r : a.out_f32 + static_cast<int64_t>(n) * a.r;
+          float* o = a.chunks ? a.out_f32 + static_cast<int64_t>(n) * ra + g * a.r
+                              : a.out_f32 + static_cast<int64_t>(n) * a.r;
           *reinterpret_cast<float4*>(o + col) = acc;
         }
       } else {
