@@ -897,7 +897,6 @@ static qlora_status linear_bwd_impl(const uint16_t* dY, const uint16_t* X, const
                                     void* dX, int32_t dx_dtype, float* dA, float* dB, void* ws, size_t ws_bytes,
                                     int32_t* d_status, void* stream, const DropoutArgs* drop) {
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
-  if (drop && r > kChunkRank) return QLORA_ERR_SHAPE;  // the dropout dX pass holds r <= 64
   if (dx_dtype != QLORA_DTYPE_BF16 && dx_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
   if (!dY || !X || !U || !A || !B || !dX || !dA || !dB) return QLORA_ERR_NULL;
@@ -1139,7 +1138,6 @@ qlora_status qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, nf4_weight W
   DropoutArgs d{};
   if (!dropout_args(p, seed, &d)) return QLORA_ERR_SHAPE;
   if (qlora_status st = check_linear_shape(M, W, r)) return st;
-  if (r > kChunkRank) return QLORA_ERR_SHAPE;  // the dropout dX pass holds r <= 64
   if (y_dtype != QLORA_DTYPE_BF16 && y_dtype != QLORA_DTYPE_F32) return QLORA_ERR_DTYPE;
   if (M == 0) return QLORA_OK;
   if (!X || !X_drop || !A || !B || !Y || !U_out) return QLORA_ERR_NULL;

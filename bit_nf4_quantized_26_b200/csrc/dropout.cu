@@ -63,7 +63,8 @@ __global__ void __launch_bounds__(256) dropout_apply_kernel(const uint16_t* __re
 // (column c holds part (c/16)%2 of j = 16 floor(c/32) + c%16), A bf16 [r, K].
 // A CTA computes a 64 x 64 block of (m, k): dU A on the tensor cores
 // (register-operand m16n8k16 MMAs, fp32 accumulate, the hi and the lo part of
-// dU each once), then per element the mask and the add.  Warp w takes rows
+// dU each once), over the rank in blocks of 64 staged in turn, then per
+// element the mask and the add.  Warp w takes rows
 // 16 (w % 4) .. + 15 and columns 32 (w / 4) .. + 31 of the block.
 constexpr int kDxTile = 64;
 constexpr int kDxLd = 64 + 8;  // bf16 per shared-memory row: 144 bytes, conflict-free fragment loads
@@ -88,40 +89,44 @@ __global__ void __launch_bounds__(256) dropout_dx_kernel(const float* __restrict
   const int m0 = blockIdx.y * kDxTile, k0 = blockIdx.x * kDxTile;
   grid_dependency_wait();
   grid_dependents_launch();
-  for (int e = tid; e < kDxTile * kDxTile; e += 256) {
-    const int mm = e / kDxTile, j = e % kDxTile;
-    uint16_t hi = 0, lo = 0;
-    if (m0 + mm < M && j < r) {
-      const uint16_t* row = ducat + static_cast<int64_t>(m0 + mm) * 2 * r;
-      const int col = 32 * (j >> 4) + (j & 15);
-      hi = row[col];
-      lo = row[col + 16];
-    }
-    uh[mm][j] = hi;
-    ul[mm][j] = lo;
-    const int jj = e / kDxTile, kk = e % kDxTile;
-    at[kk][jj] = jj < r ? A[static_cast<int64_t>(jj) * K + k0 + kk] : uint16_t(0);
-  }
-  __syncthreads();
   const int mr = (warp & 3) * 16, kc = (warp >> 2) * 32;
   float acc[4][4] = {};
-  for (int ks = 0; ks < r; ks += 16) {
-    const int jc = ks + 2 * t;
-    const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc]);
-    const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc]);
-    const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc + 8]);
-    const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc + 8]);
-    const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc]);
-    const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc]);
-    const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc + 8]);
-    const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc + 8]);
+  // The rank in blocks of 64 staged one after the other (one for r <= 64).
+  for (int j0 = 0; j0 < r; j0 += kDxTile) {
+    if (j0 > 0) __syncthreads();  // the previous block's fragments are read
+    for (int e = tid; e < kDxTile * kDxTile; e += 256) {
+      const int mm = e / kDxTile, j = e % kDxTile;
+      uint16_t hi = 0, lo = 0;
+      if (m0 + mm < M && j0 + j < r) {
+        const uint16_t* row = ducat + static_cast<int64_t>(m0 + mm) * 2 * r;
+        const int col = 32 * ((j0 + j) >> 4) + ((j0 + j) & 15);
+        hi = row[col];
+        lo = row[col + 16];
+      }
+      uh[mm][j] = hi;
+      ul[mm][j] = lo;
+      const int jj = e / kDxTile, kk = e % kDxTile;
+      at[kk][jj] = j0 + jj < r ? A[static_cast<int64_t>(j0 + jj) * K + k0 + kk] : uint16_t(0);
+    }
+    __syncthreads();
+    for (int ks = 0; ks < min(kDxTile, r - j0); ks += 16) {
+      const int jc = ks + 2 * t;
+      const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc]);
+      const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc]);
+      const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(&uh[mr + g][jc + 8]);
+      const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(&uh[mr + g + 8][jc + 8]);
+      const uint32_t al0 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc]);
+      const uint32_t al1 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc]);
+      const uint32_t al2 = *reinterpret_cast<const uint32_t*>(&ul[mr + g][jc + 8]);
+      const uint32_t al3 = *reinterpret_cast<const uint32_t*>(&ul[mr + g + 8][jc + 8]);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int kk = kc + nt * 8 + g;
-      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&at[kk][jc]);
-      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&at[kk][jc + 8]);
-      mma_16816_bf16(acc[nt], ah0, ah1, ah2, ah3, b0, b1);
-      mma_16816_bf16(acc[nt], al0, al1, al2, al3, b0, b1);
+      for (int nt = 0; nt < 4; ++nt) {
+        const int kk = kc + nt * 8 + g;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&at[kk][jc]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&at[kk][jc + 8]);
+        mma_16816_bf16(acc[nt], ah0, ah1, ah2, ah3, b0, b1);
+        mma_16816_bf16(acc[nt], al0, al1, al2, al3, b0, b1);
+      }
     }
   }
   // acc[nt]: (row g, columns 2t, 2t+1) and (row g + 8, the same columns) of
@@ -161,7 +166,7 @@ cudaError_t launch_dropout_apply(const uint16_t* X, uint16_t* Xd, int64_t count,
 
 cudaError_t launch_dropout_dx(const float* dx32, const uint16_t* ducat, const uint16_t* A, void* out, int out_f32,
                               int M, int K, int r, const DropoutArgs& d, cudaStream_t stream) {
-  if (K % kDxTile != 0 || r > kDxTile) return cudaErrorInvalidValue;
+  if (K % kDxTile != 0 || r % 16 != 0 || r > 256) return cudaErrorInvalidValue;
   return launch_kernel(dropout_dx_kernel, dim3(K / kDxTile, (M + kDxTile - 1) / kDxTile), dim3(256), 0, stream,
                        dim3(1, 1, 1), dx32, ducat, A, out, out_f32, M, K, r, d);
 }

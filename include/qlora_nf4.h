@@ -177,7 +177,7 @@ QLORA_API qlora_status nf4_dequantize_centered(const uint8_t* codes, const uint8
  * Constraints: M >= 0 (0 = no-op), K % 64 == 0, N % 64 == 0, K >= 64,
  * N >= 64, M < 2^31, N*K < 2^40, r % 16 == 0 and 16 <= r <= 256 (ranks
  * above 64 run their rank-r products as chunks of 64).  The grouped calls
- * with more than one member and the LoRA dropout calls take r <= 64.
+ * with more than one member take r <= 64.
  * Accuracy: fp32 accumulation over exact bf16 inputs; relative Frobenius
  * error of Y within 2e-3 of the fp64 product on the same dequantised weights.
  */

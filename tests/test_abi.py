@@ -237,11 +237,13 @@ def test_dropout_rejects_bad_probability_before_touching_a_device():
              1 << 20, None, None) == SHAPE
     assert f(P(256), 64, w, P(256), P(256), 16, 1.0, 0.1, 7, None, P(256), 0, P(256), P(256), 1 << 20,
              None, None) == NULL
-    # LoRA dropout takes r <= 64 (its dX pass holds one 64-wide rank block)
-    assert f(P(256), 64, w, P(256), P(256), 128, 1.0, 0.1, 7, P(256), P(256), 0, P(256), P(256), 1 << 20,
+    # ranks as for the plain linear: up to 256 in steps of 16
+    assert f(P(256), 64, w, P(256), P(256), 272, 1.0, 0.1, 7, P(256), P(256), 0, P(256), P(256), 1 << 20,
              None, None) == SHAPE
-    assert g(P(256), P(256), P(256), 64, w, P(256), P(256), 128, 1.0, 0.1, 7, P(256), 0, P(256), P(256), P(256),
-             1 << 20, None, None) == SHAPE
+    assert f(P(256), 0, w, P(256), P(256), 144, 1.0, 0.1, 7, P(256), P(256), 0, P(256), P(256), 1 << 20,
+             None, None) == OK
+    assert g(P(256), P(256), P(256), 64, w, P(256), P(256), 80 + 4, 1.0, 0.1, 7, P(256), 0, P(256), P(256),
+             P(256), 1 << 20, None, None) == SHAPE
     assert q.qlora_bwd_dropout_workspace_size(4096, 4096, 4096, 64) == \
         q.qlora_bwd_workspace_size(4096, 4096, 4096, 64) + 4096 * 4096 * 4
 

@@ -1,7 +1,7 @@
 """GPU parity of the LoRA-dropout forward and backward against the CPU oracle
 (oracle/dropout.py): X_drop bit for bit, U / dA / dB within 1e-4 and Y / dX
 within 2e-3 relative Frobenius error, on the few-token, split-K, CTA-pair and
-single-CTA wide paths."""
+single-CTA wide paths, and for ranks above 64."""
 
 import numpy as np
 import pytest
@@ -32,7 +32,9 @@ def _case(M, N, K, r, seed=0):
 SHAPES = [(16, 320, 512, 16),     # few tokens (register path)
           (200, 512, 640, 32),    # split-K fused kernel
           (600, 512, 768, 64),    # CTA-pair kernels (rows % 256 == 0)
-          (1000, 384, 512, 64)]   # single-CTA wide kernel for the forward (384 rows)
+          (1000, 384, 512, 64),   # single-CTA wide kernel for the forward (384 rows)
+          (150, 384, 448, 144),   # a rank above 64 (chunks of 64 and 16; dX pass over three rank blocks)
+          (700, 512, 768, 256)]   # the widest rank on the CTA-pair kernels
 
 
 @pytest.mark.parametrize("shape", SHAPES)
